@@ -1,0 +1,92 @@
+"""ctypes view of the C ABI in include/ba.h (libba_b200.so).
+
+Argument marshalling only: every step of branch attention runs in the CUDA
+library.  Loading fails loudly when the library has not been built; there is
+no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libba_b200.so")
+
+BA_OK = 0
+BA_ERR_INVALID_ARG = -1
+BA_ERR_UNSUPPORTED = -2
+BA_ERR_CUDA = -3
+BA_ERR_TIMEOUT = -4
+BA_ERR_WORKSPACE = -5
+
+BA_MASK_CHAIN = 0
+BA_MASK_BLOCK = 1
+
+BA_WS_FWD = 0
+BA_WS_BWD = 1
+
+EXPORTED = (
+    "ba_workspace_size", "ba_main_fwd", "ba_branch_fwd", "ba_lse_merge", "ba_fused_fwd",
+    "ba_bwd", "ba_status_string", "ba_sync_status", "ba_plan_stats",
+)
+
+
+class BaProblem(ctypes.Structure):
+    _fields_ = [
+        ("S", ctypes.c_int), ("ndoc", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+        ("d", ctypes.c_int), ("Nb", ctypes.c_int), ("B", ctypes.c_int), ("mode", ctypes.c_int),
+        ("R", ctypes.c_int), ("scale", ctypes.c_float),
+        ("cu_seqlens_h", ctypes.c_void_p), ("cu_seqlens_d", ctypes.c_void_p),
+        ("anchors_h", ctypes.c_void_p), ("anchors_d", ctypes.c_void_p),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("qb", ctypes.c_void_p), ("kb", ctypes.c_void_p), ("vb", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class BAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it is missing (build it first)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is not built; run `python -m branch_attention_speculative_packed_b200.build` "
+                "(nvcc, sm_100a). There is no fallback path.")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(BaProblem)
+        vp, i32, i64p = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)
+        L.ba_workspace_size.argtypes = [P, i32]
+        L.ba_workspace_size.restype = ctypes.c_size_t
+        L.ba_main_fwd.argtypes = [P, vp, vp, vp]
+        L.ba_branch_fwd.argtypes = [P, vp, vp, vp]
+        L.ba_fused_fwd.argtypes = [P, vp, vp, vp, vp]
+        L.ba_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.ba_lse_merge.argtypes = [i32, i32, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                   i64p, vp, vp, ctypes.c_int64, vp]
+        L.ba_status_string.argtypes = [i32]
+        L.ba_status_string.restype = ctypes.c_char_p
+        L.ba_sync_status.argtypes = [vp]
+        L.ba_plan_stats.argtypes = [P, i64p, i64p, i64p]
+        for name in ("ba_main_fwd", "ba_branch_fwd", "ba_fused_fwd", "ba_bwd", "ba_lse_merge",
+                     "ba_sync_status", "ba_plan_stats"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().ba_status_string(int(status)).decode()
+
+
+def check(status: int, where: str) -> None:
+    if status != BA_OK:
+        raise BAError(status, where)

@@ -1,0 +1,477 @@
+// Branch-attention forward on sm_100a: tcgen05 MMA with TMEM accumulators,
+// TMA-staged tiles, warp-specialised pipeline.
+//
+// Paper: arXiv 2609.07108 §3.2 / Eq. 2 (rcap.io post, branch-attention
+// paragraph; cere-bro wiki, "Obstacle one, context parallelism").  One
+// persistent CTA per SM walks (row tile, query head) work items, longest
+// first.  For each item it streams the item's main key tiles (the causal
+// prefix [doc start, largest limit]) and, in the fused variant, the key tiles
+// of the branch-local keys, through one online softmax.  Visiting key tiles
+// one after another with a running (max, sum) is the same log-sum-exp merge
+// ring attention applies between ring steps (Eq. 2), so the main-sequence
+// component, the branch-local component and their merge all happen here.
+//
+// Roles (192 threads):
+//   warp 0      TMA producer: gathers the 128 query rows of the tile (one
+//               1-row box per row and 64 columns) and streams K/V key tiles
+//               through a 2-stage ring.
+//   warp 1      TMEM allocator and single-thread MMA issuer:
+//               S[sb] = Q K^T into one of two TMEM buffers, then O += P V.
+//   warps 2-5   softmax / epilogue, one query row per thread: load S from
+//               TMEM, mask by the row's key range, update the running max
+//               (lazily: O in TMEM is rescaled only when the max grows by
+//               more than 2^8), write P (bf16) to shared memory for the next
+//               MMA, and finally normalise O and write O and LSE.
+//
+// Shared memory (D = head dim): Q [128 x D] | 2 x (K [128 x D], V [128 x D])
+// | P [128 x 128], all bf16 in the 128-byte-swizzled layout TMA writes.
+// TMEM: S buffers at columns 0 and 128, O at column 256.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace ba {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColO = 256;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct Smem {
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kTileBytes = 128u * D * 2u;  // one 128-row bf16 tile
+  static constexpr uint32_t kK0 = kQ + kTileBytes;
+  static constexpr uint32_t kStageBytes = 2u * kTileBytes;  // K + V
+  static constexpr uint32_t kP = kK0 + kStages * kStageBytes;
+  static constexpr uint32_t kBar = kP + 128u * 128u * 2u;
+  // barriers: q_full, q_empty, kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, o_done, drain
+  static constexpr uint32_t kNumBars = 13;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base (4 B), abort (4 B)
+  static constexpr uint32_t kTotal = kMisc + 16u;
+  static constexpr uint32_t kAlloc = kTotal + 1024u;  // slack to align the base to 1024
+};
+
+struct Bars {
+  uint32_t q_full, q_empty, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full,
+      o_done, drain;
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQb,
+               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
+               const FwdArgs a) {
+  using L = Smem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  Bars bar;
+  {
+    uint32_t b = sbase + L::kBar;
+    bar.q_full = b; b += 8;
+    bar.q_empty = b; b += 8;
+    for (int i = 0; i < kStages; ++i) { bar.kv_full[i] = b; b += 8; }
+    for (int i = 0; i < kStages; ++i) { bar.kv_empty[i] = b; b += 8; }
+    for (int i = 0; i < 2; ++i) { bar.s_full[i] = b; b += 8; }
+    for (int i = 0; i < 2; ++i) { bar.s_empty[i] = b; b += 8; }
+    bar.p_full = b; b += 8;
+    bar.o_done = b; b += 8;
+    bar.drain = b;
+  }
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar.q_full, 1);
+    ptx::mbar_init(bar.q_empty, 1);
+    for (int i = 0; i < kStages; ++i) {
+      ptx::mbar_init(bar.kv_full[i], 1);
+      ptx::mbar_init(bar.kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar.s_full[i], 1);
+      ptx::mbar_init(bar.s_empty[i], 128);
+    }
+    ptx::mbar_init(bar.p_full, 128);
+    ptx::mbar_init(bar.o_done, 1);
+    ptx::mbar_init(bar.drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmQ);
+    ptx::prefetch_tmap(&tmQb);
+    ptx::prefetch_tmap(&tmK);
+    ptx::prefetch_tmap(&tmV);
+    ptx::prefetch_tmap(&tmKb);
+    ptx::prefetch_tmap(&tmVb);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(sbase + L::kMisc, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const int Hq = a.Hq;
+  const long long lim = a.wait_limit;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t kv_stage = 0, kv_phase = 0, q_phase = 0;
+    // Parity of each stage's last fill and whether it may still be in flight
+    // (for the abort drain); same for the query tile.
+    uint32_t pend_mask = 0, pend_par = 0, q_fills = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      const TileDesc td = a.tiles[a.order[item / Hq]];
+      const int h = item % Hq;
+      const int g = h / a.G;
+      int waited = 1;
+      if (lane == 0) waited = ptx::mbar_wait(bar.q_empty, q_phase ^ 1u, abort_flag, a.err, lim);
+      waited = __shfl_sync(0xffffffffu, waited, 0);
+      if (!waited) { ok = false; break; }
+      q_phase ^= 1u;
+      if (lane == 0) ptx::mbar_expect_tx(bar.q_full, L::kTileBytes);
+      ++q_fills;
+      __syncwarp();
+      for (int i = lane; i < 128; i += 32) {
+        const int r = a.row_table[td.row_base + i];
+        const void* map = &tmQ;
+        int y = -1;  // out of range: TMA fills zeros for padding rows
+        if (r >= 0 && r < a.S) {
+          y = r;
+        } else if (r >= a.S) {
+          map = &tmQb;
+          y = r - a.S;
+        }
+#pragma unroll
+        for (int cb = 0; cb < D / 64; ++cb)
+          ptx::tma_load_2d(sbase + L::kQ + cb * 16384u + i * 128u, map, bar.q_full, h * D + cb * 64, y);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
+        const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
+        for (int j = 0; j < nkv + nbr; ++j) {
+          if (!ptx::mbar_wait(bar.kv_empty[kv_stage], kv_phase ^ 1u, abort_flag, a.err, lim)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_expect_tx(bar.kv_full[kv_stage], 2u * L::kTileBytes);
+          const void* mk = &tmK;
+          const void* mv = &tmV;
+          int y;
+          if (j < nkv) {
+            y = td.doc_start + 128 * j;
+          } else {
+            y = td.br_lo + 128 * (j - nkv);
+            mk = &tmKb;
+            mv = &tmVb;
+          }
+          const uint32_t sk = sbase + L::kK0 + kv_stage * L::kStageBytes;
+          const uint32_t sv = sk + L::kTileBytes;
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb) {
+            ptx::tma_load_2d(sk + cb * 16384u, mk, bar.kv_full[kv_stage], g * D + cb * 64, y);
+            ptx::tma_load_2d(sv + cb * 16384u, mv, bar.kv_full[kv_stage], g * D + cb * 64, y);
+          }
+          pend_mask |= 1u << kv_stage;
+          pend_par = (pend_par & ~(1u << kv_stage)) | (kv_phase << kv_stage);
+          if (++kv_stage == kStages) { kv_stage = 0; kv_phase ^= 1u; }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    if (lane == 0 && *abort_flag) {
+      // Let our own copies in flight land before the CTA exits (bounded).
+      volatile int never = 0;
+      for (int i = 0; i < kStages; ++i)
+        if (pend_mask & (1u << i))
+          ptx::mbar_wait(bar.kv_full[i], (pend_par >> i) & 1u, &never, a.err, lim / 8);
+      if (q_fills) ptx::mbar_wait(bar.q_full, (q_fills - 1) & 1u, &never, a.err, lim / 8);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdPV = ptx::idesc_bf16_f32(128, D, false, true);
+      uint32_t kv_stage = 0, kv_phase = 0, q_phase = 0, p_phase = 0, s_cnt = 0;
+      bool ok = true;
+      const uint32_t sQ = sbase + L::kQ;
+      const uint32_t sP = sbase + L::kP;
+      auto issue_pv = [&](int jj, uint32_t stage) -> bool {
+        if (!ptx::mbar_wait(bar.p_full, p_phase, abort_flag, a.err, lim)) return false;
+        p_phase ^= 1u;
+        ptx::tc_fence_after();
+        const uint32_t sv = sbase + L::kK0 + stage * L::kStageBytes + L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ad = ptx::sdesc_sw128(sP + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
+          const uint64_t bd = ptx::sdesc_sw128(sv + kk * 2048u, 16384u, 1024u);
+          ptx::umma_ss(tmem + kColO, ad, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::umma_commit(bar.o_done);
+        ptx::umma_commit(bar.kv_empty[stage]);
+        return true;
+      };
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+        const TileDesc td = a.tiles[a.order[item / Hq]];
+        const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
+        const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
+        const int n = nkv + nbr;
+        if (!ptx::mbar_wait(bar.q_full, q_phase, abort_flag, a.err, lim)) { ok = false; break; }
+        q_phase ^= 1u;
+        ptx::tc_fence_after();
+        uint32_t prev_stage = 0;
+        for (int j = 0; j < n; ++j) {
+          if (!ptx::mbar_wait(bar.kv_full[kv_stage], kv_phase, abort_flag, a.err, lim)) { ok = false; break; }
+          const uint32_t sb = s_cnt & 1u;
+          const uint32_t sph = (s_cnt >> 1) & 1u;
+          if (!ptx::mbar_wait(bar.s_empty[sb], sph ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t sk = sbase + L::kK0 + kv_stage * L::kStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+            const uint64_t ad = ptx::sdesc_sw128(sQ + off, 16u, 1024u);
+            const uint64_t bd = ptx::sdesc_sw128(sk + off, 16u, 1024u);
+            ptx::umma_ss(tmem + kColS0 + sb * 128u, ad, bd, kIdS, kk > 0 ? 1u : 0u);
+          }
+          ptx::umma_commit(bar.s_full[sb]);
+          ++s_cnt;
+          if (j == n - 1) ptx::umma_commit(bar.q_empty);
+          if (j > 0 && !issue_pv(j - 1, prev_stage)) { ok = false; break; }
+          prev_stage = kv_stage;
+          if (++kv_stage == kStages) { kv_stage = 0; kv_phase ^= 1u; }
+        }
+        if (!ok) break;
+        if (!issue_pv(n - 1, prev_stage)) { ok = false; break; }
+      }
+      // Drain: every MMA this thread issued completes before TMEM is freed.
+      ptx::umma_commit(bar.drain);
+      volatile int never = 0;
+      ptx::mbar_wait(bar.drain, 0, &never, a.err, lim);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t sP = sbase + L::kP;
+    const float sl2 = a.scale_log2;
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      const TileDesc td = a.tiles[a.order[item / Hq]];
+      const int h = item % Hq;
+      const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
+      const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
+      const int n = nkv + nbr;
+      const int r = a.row_table[td.row_base + row];
+      int limit = td.doc_start;  // padding rows see one key: keeps their math finite
+      int blo = 0, bhi = 0;      // visible branch key rows [blo, bhi)
+      if (r >= 0 && r < a.S) {
+        limit = r;
+      } else if (r >= a.S) {
+        const int b = (r - a.S) / a.B;
+        const int t = (r - a.S) - b * a.B;
+        limit = a.anchors[b];
+        blo = b * a.B;
+        bhi = blo + (a.mode == 1 ? a.B : t + 1);
+      }
+      float m_used = -INFINITY;
+      float l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t sb = s_cnt & 1u;
+        const uint32_t sph = (s_cnt >> 1) & 1u;
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.s_full[sb], sph, abort_flag, a.err, lim))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tl + kColS0 + sb * 128u + c * 32u, sr[c]);
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar.s_empty[sb]);
+        ++s_cnt;
+        // visible columns [lo, hi) of this key tile
+        int lo, hi;
+        if (j < nkv) {
+          lo = 0;
+          hi = limit - (td.doc_start + 128 * j) + 1;
+        } else {
+          const int kr0 = td.br_lo + 128 * (j - nkv);
+          lo = blo - kr0;
+          hi = bhi - kr0;
+        }
+        lo = max(lo, 0);
+        hi = min(hi, 128);
+        float mx = -INFINITY;
+        if (lo == 0 && hi == 128) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[c][i]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int col = c * 32 + i;
+              const bool vis = col >= lo && col < hi;
+              if (!vis) sr[c][i] = __float_as_uint(-INFINITY);
+              mx = fmaxf(mx, __uint_as_float(sr[c][i]));
+            }
+        }
+        const float mxs = mx * sl2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (m_used == -INFINITY) {
+          m_used = mxs;
+        } else if (mxs > m_used + kRescaleThreshold) {
+          alpha = ptx::ex2(m_used - mxs);
+          m_used = mxs;
+          rescale = true;
+        }
+        const float neg_m = -m_used;
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p = ptx::ex2(fmaf(__uint_as_float(sr[c][i]), sl2, neg_m));
+            rs += p;
+            sr[c][i] = __float_as_uint(p);
+          }
+        l = l * alpha + rs;
+        if (j > 0) {
+          // P buffer and O are free once the previous P.V finished.
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done, o_cnt & 1u, abort_flag, a.err, lim))) {
+            ok = false;
+            break;
+          }
+          ++o_cnt;
+          ptx::tc_fence_after();
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t ov[32];
+              ptx::tmem_ld32(tl + kColO + c * 32u, ov);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              ptx::tmem_st32(tl + kColO + c * 32u, ov);
+            }
+            ptx::tmem_wait_st();
+          }
+        }
+        // P (bf16) -> shared memory, 128-byte-swizzled K-major rows.
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch) {
+          const int c = ch >> 2, i0 = (ch & 3) * 8;
+          const uint32_t w0 = ptx::pack_bf16x2(__uint_as_float(sr[c][i0 + 0]), __uint_as_float(sr[c][i0 + 1]));
+          const uint32_t w1 = ptx::pack_bf16x2(__uint_as_float(sr[c][i0 + 2]), __uint_as_float(sr[c][i0 + 3]));
+          const uint32_t w2 = ptx::pack_bf16x2(__uint_as_float(sr[c][i0 + 4]), __uint_as_float(sr[c][i0 + 5]));
+          const uint32_t w3 = ptx::pack_bf16x2(__uint_as_float(sr[c][i0 + 6]), __uint_as_float(sr[c][i0 + 7]));
+          const uint32_t addr = sP + (ch >> 3) * 16384u + row * 128u + ((((ch & 7) ^ (row & 7))) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
+                       "r"(w2), "r"(w3)
+                       : "memory");
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar.p_full);
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done, o_cnt & 1u, abort_flag, a.err, lim))) {
+        ok = false;
+        break;
+      }
+      ++o_cnt;
+      ptx::tc_fence_after();
+      const float inv_l = 1.f / l;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        ptx::tmem_ld32(tl + kColO + c * 32u, ov);
+        ptx::tmem_wait_ld();
+        if (r >= 0) {
+          if (a.out_bf16) {
+            __nv_bfloat16* dst = (r < a.S ? a.o + (int64_t(r) * Hq + h) * D
+                                          : a.ob + (int64_t(r - a.S) * Hq + h) * D) + c * 32;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint4 w;
+              w.x = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 0]) * inv_l, __uint_as_float(ov[q4 * 8 + 1]) * inv_l);
+              w.y = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 2]) * inv_l, __uint_as_float(ov[q4 * 8 + 3]) * inv_l);
+              w.z = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 4]) * inv_l, __uint_as_float(ov[q4 * 8 + 5]) * inv_l);
+              w.w = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 6]) * inv_l, __uint_as_float(ov[q4 * 8 + 7]) * inv_l);
+              reinterpret_cast<uint4*>(dst)[q4] = w;
+            }
+          } else {
+            float* dst = a.o_part + (int64_t(r) * Hq + h) * D + c * 32;
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+              float4 w;
+              w.x = __uint_as_float(ov[q4 * 4 + 0]) * inv_l;
+              w.y = __uint_as_float(ov[q4 * 4 + 1]) * inv_l;
+              w.z = __uint_as_float(ov[q4 * 4 + 2]) * inv_l;
+              w.w = __uint_as_float(ov[q4 * 4 + 3]) * inv_l;
+              reinterpret_cast<float4*>(dst)[q4] = w;
+            }
+          }
+        }
+      }
+      if (r >= 0) a.lse[int64_t(h) * a.lse_ld + r] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      ptx::tc_fence_before();
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_fwd_d(const FwdMaps& m, const FwdArgs& a, int num_sms, cudaStream_t stream) {
+  using L = Smem<D>;
+  static_assert(L::kAlloc <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::kAlloc));
+  if (e != cudaSuccess) return e;
+  const int grid = a.n_items < num_sms ? a.n_items : num_sms;
+  if (grid <= 0) return cudaSuccess;
+  fwd_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(m.q, m.qb, m.k, m.v, m.kb, m.vb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const FwdMaps& maps, const FwdArgs& a, int num_sms, cudaStream_t stream) {
+  if (a.d == 128) return launch_fwd_d<128>(maps, a, num_sms, stream);
+  if (a.d == 64) return launch_fwd_d<64>(maps, a, num_sms, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ba

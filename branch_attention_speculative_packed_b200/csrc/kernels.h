@@ -1,0 +1,62 @@
+// Launch wrappers of the device kernels (host side).  Every wrapper enqueues
+// on `stream` and returns the cudaError_t of the launch.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tile_desc.h"
+
+namespace ba {
+
+// ---------------------------------------------------------------- forward
+struct FwdArgs {
+  const int32_t* anchors;    // [Nb]
+  const int32_t* row_table;  // [ntiles * 128], -1 = padding
+  const TileDesc* tiles;     // [ntiles]
+  const int32_t* order;      // [ntiles], longest first
+  int S, Nb, B, mode, Hq, G, d;
+  int n_items;               // ntiles * Hq
+  float scale_log2;          // softmax scale * log2(e)
+  int with_branch;           // also visit the branch key tiles (fused forward)
+  int out_bf16;              // 1: bf16 o / ob; 0: fp32 o_part
+  float* o_part;             // [rows, Hq, d]
+  __nv_bfloat16* o;          // [S, Hq, d]
+  __nv_bfloat16* ob;         // [Nb*B, Hq, d]
+  float* lse;                // element (h, r) at lse[h * lse_ld + r]
+  int64_t lse_ld;
+  uint32_t* err;             // device error word
+  long long wait_limit;      // cycles per bounded wait
+};
+
+struct FwdMaps {
+  CUtensorMap q, qb, k, v, kb, vb;
+};
+
+cudaError_t launch_fwd(const FwdMaps& maps, const FwdArgs& a, int num_sms, cudaStream_t stream);
+
+// ---------------------------------------------------------------- planning
+cudaError_t launch_plan_rows(const int32_t* cu_seqlens, int ndoc, const int32_t* anchors, int S,
+                             int Nb, int B, int R, const ChunkDev* chunks, int32_t* row_table,
+                             int64_t n_slots, cudaStream_t stream);
+
+// ---------------------------------------------------------------- branch part / merge
+cudaError_t launch_branch_fwd(const __nv_bfloat16* qb, const __nv_bfloat16* kb,
+                              const __nv_bfloat16* vb, int Nb, int B, int mode, int Hq, int Hkv,
+                              int d, float scale, float* o_part, float* lse_part,
+                              cudaStream_t stream);
+
+struct MergeArgs {
+  int nparts, rows, H, d;
+  const float* o[16];
+  const float* lse[16];
+  int64_t lse_ld[16];
+  __nv_bfloat16* o_out;
+  float* lse_out;
+  int64_t lse_out_ld;
+};
+cudaError_t launch_lse_merge(const MergeArgs& a, cudaStream_t stream);
+
+}  // namespace ba

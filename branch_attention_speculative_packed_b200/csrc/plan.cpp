@@ -1,0 +1,206 @@
+// Host planner: validation, zigzag chunks, row tiles, longest-first order.
+#include "plan.h"
+
+#include <algorithm>
+#include <cstdint>
+#include <numeric>
+
+namespace ba {
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// First index i in [lo, hi) with a[i] >= x.
+int lower_bound_i(const int32_t* a, int lo, int hi, int64_t x) {
+  return static_cast<int>(std::lower_bound(a + lo, a + hi, x) - a);
+}
+
+}  // namespace
+
+ba_status validate(const ba_problem* p, bool need_tensors) {
+  if (!p) return BA_ERR_INVALID_ARG;
+  if (p->S < 1 || p->ndoc < 1 || p->ndoc > p->S) return BA_ERR_INVALID_ARG;
+  if (p->Hq < 1 || p->Hkv < 1 || p->Hq % p->Hkv != 0) return BA_ERR_INVALID_ARG;
+  if (p->d < 1 || p->Nb < 0 || p->R < 1 || p->R > 64) return BA_ERR_INVALID_ARG;
+  if (p->mode != BA_MASK_CHAIN && p->mode != BA_MASK_BLOCK) return BA_ERR_INVALID_ARG;
+  if (p->Nb > 0 && (p->B < 1 || p->B > 64)) return BA_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return BA_ERR_UNSUPPORTED;
+  // Row indices and head-major LSE offsets must fit the kernels' int32 row math.
+  const int64_t rows = (int64_t)p->S + (int64_t)p->Nb * (p->Nb > 0 ? p->B : 0);
+  if (rows >= (int64_t(1) << 31) - kRowsPerTile * 4) return BA_ERR_UNSUPPORTED;
+  if (!p->cu_seqlens_h || !p->cu_seqlens_d) return BA_ERR_INVALID_ARG;
+  if (p->Nb > 0 && (!p->anchors_h || !p->anchors_d)) return BA_ERR_INVALID_ARG;
+  const int32_t* cu = p->cu_seqlens_h;
+  if (cu[0] != 0 || cu[p->ndoc] != p->S) return BA_ERR_INVALID_ARG;
+  for (int i = 0; i < p->ndoc; ++i)
+    if (cu[i + 1] <= cu[i]) return BA_ERR_INVALID_ARG;  // empty or decreasing document
+  for (int b = 0; b < p->Nb; ++b) {
+    const int32_t a = p->anchors_h[b];
+    if (a < 0 || a >= p->S) return BA_ERR_INVALID_ARG;
+    if (b > 0 && a < p->anchors_h[b - 1]) return BA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(p->cu_seqlens_d) || (p->Nb > 0 && !aligned16(p->anchors_d)))
+    return BA_ERR_INVALID_ARG;
+  if (need_tensors) {
+    if (!p->q || !p->k || !p->v) return BA_ERR_INVALID_ARG;
+    if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v)) return BA_ERR_INVALID_ARG;
+    if (p->Nb > 0) {
+      if (!p->qb || !p->kb || !p->vb) return BA_ERR_INVALID_ARG;
+      if (!aligned16(p->qb) || !aligned16(p->kb) || !aligned16(p->vb)) return BA_ERR_INVALID_ARG;
+    }
+  }
+  return BA_OK;
+}
+
+void build_plan(const ba_problem* p, Plan* plan) {
+  const int S = p->S, R = p->R;
+  const int Nb = p->Nb, B = (p->Nb > 0 ? p->B : 0);
+  const int32_t* cu = p->cu_seqlens_h;
+  const int32_t* anc = p->anchors_h;
+  plan->S = S;
+  plan->Nb = Nb;
+  plan->B = B;
+  plan->R = R;
+  plan->ndoc = p->ndoc;
+  plan->chunks.clear();
+  plan->tiles.clear();
+  plan->chunks_dev.clear();
+  plan->n_tile_pairs = plan->n_branch_tile_pairs = plan->n_visible_pairs = 0;
+
+  // Exact visible pairs per head (counting rule of the definition).
+  int64_t vis = 0;
+  for (int i = 0; i < p->ndoc; ++i) {
+    const int64_t L = cu[i + 1] - cu[i];
+    vis += L * (L + 1) / 2;
+  }
+  for (int b = 0; b < Nb; ++b) {
+    const int di = static_cast<int>(std::upper_bound(cu, cu + p->ndoc + 1, anc[b]) - cu) - 1;
+    vis += int64_t(B) * (anc[b] - cu[di] + 1);
+    vis += (p->mode == BA_MASK_CHAIN) ? int64_t(B) * (B + 1) / 2 : int64_t(B) * B;
+  }
+  plan->n_visible_pairs = vis;
+
+  int tile_count = 0;
+  for (int di = 0; di < p->ndoc; ++di) {
+    const int s = cu[di], e = cu[di + 1];
+    const int64_t L = e - s;
+    for (int k = 0; k < 2 * R; ++k) {
+      Chunk c;
+      c.doc = di;
+      c.k = k;
+      c.rank = k < R ? k : 2 * R - 1 - k;
+      c.c0 = s + static_cast<int>((int64_t(k) * L) / (2 * R));
+      c.c1 = s + static_cast<int>((int64_t(k + 1) * L) / (2 * R));
+      c.b0 = Nb ? lower_bound_i(anc, 0, Nb, c.c0) : 0;
+      c.b1 = Nb ? lower_bound_i(anc, c.b0, Nb, c.c1) : 0;
+      c.n_rows = int64_t(c.c1 - c.c0) + int64_t(B) * (c.b1 - c.b0);
+      c.tile0 = tile_count;
+      c.ntiles = static_cast<int>((c.n_rows + kRowsPerTile - 1) / kRowsPerTile);
+      tile_count += c.ntiles;
+      plan->chunks.push_back(c);
+      ChunkDev cd;
+      cd.c0 = c.c0;
+      cd.b0 = c.b0;
+      cd.slot_base = c.tile0 * kRowsPerTile;
+      cd.pad = 0;
+      plan->chunks_dev.push_back(cd);
+
+      // merged index of main position q within the chunk
+      auto main_index = [&](int q) -> int64_t {
+        const int lb = Nb ? lower_bound_i(anc, c.b0, c.b1, q) : 0;
+        return int64_t(q - c.c0) + int64_t(B) * (lb - c.b0);
+      };
+      // limit of the row at merged index m: largest q in [c0, c1) with main_index(q) <= m
+      auto limit_at = [&](int64_t m) -> int {
+        int lo = c.c0, hi = c.c1 - 1;
+        while (lo < hi) {
+          const int mid = lo + (hi - lo + 1) / 2;
+          if (main_index(mid) <= m) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+      };
+      // first merged index of branch b's rows
+      auto branch_start = [&](int b) -> int64_t {
+        return int64_t(anc[b] - c.c0) + 1 + int64_t(B) * (b - c.b0);
+      };
+      for (int t = 0; t < c.ntiles; ++t) {
+        const int64_t m0 = int64_t(t) * kRowsPerTile;
+        const int64_t m1 = std::min<int64_t>(c.n_rows, m0 + kRowsPerTile);
+        TileDesc td;
+        td.row_base = (c.tile0 + t) * kRowsPerTile;
+        td.n_rows = static_cast<int32_t>(m1 - m0);
+        td.doc_start = s;
+        td.min_limit = limit_at(m0);
+        td.kv_end = limit_at(m1 - 1) + 1;
+        td.rank = c.rank;
+        td.br_lo = td.br_hi = 0;
+        if (c.b1 > c.b0) {
+          // branches whose rows [start, start + B) meet [m0, m1)
+          int lo = c.b0, hi = c.b1;  // first b with start(b) + B > m0
+          while (lo < hi) {
+            const int mid = (lo + hi) / 2;
+            if (branch_start(mid) + B > m0) hi = mid; else lo = mid + 1;
+          }
+          const int blo = lo;
+          lo = c.b0;
+          hi = c.b1;  // first b with start(b) >= m1
+          while (lo < hi) {
+            const int mid = (lo + hi) / 2;
+            if (branch_start(mid) >= m1) hi = mid; else lo = mid + 1;
+          }
+          const int bhi = lo;  // exclusive
+          if (bhi > blo) {
+            td.br_lo = blo * B;
+            td.br_hi = bhi * B;
+          }
+        }
+        const int64_t nkv = (int64_t(td.kv_end) - td.doc_start + kKeysPerTile - 1) / kKeysPerTile;
+        const int64_t nbr = (int64_t(td.br_hi) - td.br_lo + kKeysPerTile - 1) / kKeysPerTile;
+        plan->n_tile_pairs += nkv;
+        plan->n_branch_tile_pairs += std::max<int64_t>(0, nbr);
+        plan->tiles.push_back(td);
+      }
+    }
+  }
+  // Longest-processing-time-first order over the key tiles each row tile visits.
+  const int nt = static_cast<int>(plan->tiles.size());
+  plan->order.resize(nt);
+  std::iota(plan->order.begin(), plan->order.end(), 0);
+  std::vector<int64_t> cost(nt);
+  for (int i = 0; i < nt; ++i) {
+    const TileDesc& td = plan->tiles[i];
+    cost[i] = (int64_t(td.kv_end) - td.doc_start + kKeysPerTile - 1) / kKeysPerTile +
+              (int64_t(td.br_hi) - td.br_lo + kKeysPerTile - 1) / kKeysPerTile;
+  }
+  std::stable_sort(plan->order.begin(), plan->order.end(),
+                   [&](int a, int b) { return cost[a] > cost[b]; });
+}
+
+WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int which) {
+  WorkspaceLayout w;
+  const size_t nt = plan.tiles.size();
+  w.n_slots = int64_t(nt) * kRowsPerTile;
+  size_t off = 0;
+  w.tiles_off = off;
+  off = align_up(off + nt * sizeof(TileDesc), 256);
+  w.order_off = off;
+  off = align_up(off + nt * sizeof(int32_t), 256);
+  w.chunks_off = off;
+  off = align_up(off + plan.chunks_dev.size() * sizeof(ChunkDev), 256);
+  w.rows_off = off;
+  off = align_up(off + size_t(w.n_slots) * sizeof(int32_t), 256);
+  if (which == BA_WS_BWD) {
+    const size_t rows = size_t(p->S) + size_t(p->Nb) * (p->Nb > 0 ? p->B : 0);
+    w.dsum_off = off;
+    off = align_up(off + rows * p->Hq * sizeof(float), 256);
+    w.dq_off = off;
+    off = align_up(off + rows * p->Hq * p->d * sizeof(float), 256);
+  }
+  w.total = off;
+  return w;
+}
+
+}  // namespace ba

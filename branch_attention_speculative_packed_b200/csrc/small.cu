@@ -1,0 +1,254 @@
+// Small kernels: row-table scatter of the plan, the standalone branch-local
+// component (step a3) and the k-way LSE merge (step a4, Eq. 2).
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace ba {
+namespace {
+
+// ------------------------------------------------------------------ plan rows
+// Writes every concatenated row index r (main rows 0..S-1, then branch rows
+// S + b*B + t) into the slot of its row tile.  Within a zigzag chunk [c0, c1)
+// the rows are ordered by limit (main row p: p; branch row: its anchor), main
+// row first on ties, then branches in index order, depth-minor:
+//   main p:       m = (p - c0) + B * (#anchors in [c0, p))
+//   branch (b,t): m = (a_b - c0) + 1 + B * (b - b0) + t
+// The chunk of a position x in document [s, s+L) is the k with
+// floor(kL/2R) <= x - s < floor((k+1)L/2R).
+__global__ void plan_rows_kernel(const int32_t* __restrict__ cu, int ndoc,
+                                 const int32_t* __restrict__ anchors, int S, int Nb, int B, int R,
+                                 const ChunkDev* __restrict__ chunks, int32_t* __restrict__ rows,
+                                 int64_t n_slots) {
+  const int64_t total = int64_t(S) + int64_t(Nb) * B;
+  const int R2 = 2 * R;
+  for (int64_t r = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; r < total;
+       r += int64_t(gridDim.x) * blockDim.x) {
+    int lim, b = 0, t = 0;
+    const bool br = r >= S;
+    if (!br) {
+      lim = static_cast<int>(r);
+    } else {
+      const int64_t q = r - S;
+      b = static_cast<int>(q / B);
+      t = static_cast<int>(q - int64_t(b) * B);
+      lim = anchors[b];
+    }
+    int lo = 0, hi = ndoc - 1;  // last document with start <= lim
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cu[mid] <= lim) lo = mid; else hi = mid - 1;
+    }
+    const int s = cu[lo];
+    const int64_t L = cu[lo + 1] - s;
+    const int64_t x = lim - s;
+    int k = static_cast<int>((x * R2) / L);
+    while (k + 1 < R2 && (int64_t(k + 1) * L) / R2 <= x) ++k;
+    while (k > 0 && (int64_t(k) * L) / R2 > x) --k;
+    const ChunkDev c = chunks[int64_t(lo) * R2 + k];
+    int64_t m;
+    if (!br) {
+      int a0 = 0, a1 = Nb;  // first anchor >= lim
+      while (a0 < a1) {
+        const int mid = (a0 + a1) >> 1;
+        if (anchors[mid] < lim) a0 = mid + 1; else a1 = mid;
+      }
+      m = int64_t(lim - c.c0) + int64_t(B) * (a0 - c.b0);
+    } else {
+      m = int64_t(lim - c.c0) + 1 + int64_t(B) * (b - c.b0) + t;
+    }
+    const int64_t slot = int64_t(c.slot_base) + m;
+    if (slot >= 0 && slot < n_slots) rows[slot] = static_cast<int32_t>(r);
+  }
+}
+
+// ------------------------------------------------------------------ branch part
+// One block per (branch b, KV head g), one warp per query head of the group.
+// The branch's B keys and values of head g are staged in shared memory; each
+// warp walks the B rows of its head: scores against the visible branch keys
+// (chain: u <= t; block: all), softmax, O = P V.  Output fp32 O and LSE.
+template <int D>
+__global__ void branch_fwd_kernel(const __nv_bfloat16* __restrict__ qb,
+                                  const __nv_bfloat16* __restrict__ kb,
+                                  const __nv_bfloat16* __restrict__ vb, int Nb, int B, int mode,
+                                  int Hq, int Hkv, float scale, float* __restrict__ o_part,
+                                  float* __restrict__ lse_part) {
+  constexpr int E = D / 32;  // elements per lane
+  extern __shared__ float sm[];  // [2][B][D]
+  const int b = blockIdx.x / Hkv;
+  const int g = blockIdx.x % Hkv;
+  const int G = Hq / Hkv;
+  float* sk = sm;
+  float* sv = sm + B * D;
+  for (int i = threadIdx.x; i < B * D; i += blockDim.x) {
+    const int u = i / D, e = i % D;
+    const int64_t off = ((int64_t(b) * B + u) * Hkv + g) * D + e;
+    sk[i] = __bfloat162float(kb[off]);
+    sv[i] = __bfloat162float(vb[off]);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp >= G) return;
+  const int h = g * G + warp;
+  const int64_t nbr = int64_t(Nb) * B;
+  for (int t = 0; t < B; ++t) {
+    const int64_t row = int64_t(b) * B + t;
+    float qv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) qv[e] = __bfloat162float(qb[(row * Hq + h) * D + lane * E + e]);
+    const int nvis = mode == 1 ? B : t + 1;
+    float mx = -INFINITY, l = 0.f;
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int u = 0; u < nvis; ++u) {
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) s = fmaf(qv[e], sk[u * D + lane * E + e], s);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      s *= scale;
+      const float mn = fmaxf(mx, s);
+      const float c = expf(mx - mn);
+      const float p = expf(s - mn);
+      l = l * c + p;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = acc[e] * c + p * sv[u * D + lane * E + e];
+      mx = mn;
+    }
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int e = 0; e < E; ++e) o_part[(row * Hq + h) * D + lane * E + e] = acc[e] * inv;
+    if (lane == 0) lse_part[int64_t(h) * nbr + row] = mx + logf(l);
+  }
+}
+
+// ------------------------------------------------------------------ LSE merge
+// One warp per (head h, group of 32 rows).  Lane j first merges the LSEs of
+// row r0 + j (coalesced over rows), then the warp walks the 32 rows and each
+// lane rescales-and-adds a 16-byte slice of every part's O row (coalesced
+// over d), writing bf16 O and fp32 LSE.
+template <int D>
+__global__ void __launch_bounds__(256) lse_merge_kernel(const MergeArgs a) {
+  constexpr int E = D / 32;  // 4 (float4) for D=128, 2 (float2) for D=64
+  const int64_t groups = (int64_t(a.rows) + 31) / 32;
+  const int64_t nwarps = groups * a.H;
+  const int lane = threadIdx.x & 31;
+  for (int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32; w < nwarps;
+       w += (int64_t(gridDim.x) * blockDim.x) / 32) {
+    const int h = static_cast<int>(w % a.H);
+    const int64_t r0 = (w / a.H) * 32;
+    const int64_t my = r0 + lane;
+    const bool live = my < a.rows;
+    float lp[16];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      lp[p] = -INFINITY;
+      if (p < a.nparts && live) lp[p] = a.lse[p][int64_t(h) * a.lse_ld[p] + my];
+      mx = fmaxf(mx, lp[p]);
+    }
+    float Lr = -INFINITY;
+    float wt[16];
+    if (mx != -INFINITY) {
+      float tot = 0.f;
+#pragma unroll
+      for (int p = 0; p < 16; ++p) tot += (lp[p] == -INFINITY) ? 0.f : expf(lp[p] - mx);
+      Lr = mx + logf(tot);
+    }
+#pragma unroll
+    for (int p = 0; p < 16; ++p) wt[p] = (Lr == -INFINITY || lp[p] == -INFINITY) ? 0.f : expf(lp[p] - Lr);
+    if (live) a.lse_out[int64_t(h) * a.lse_out_ld + my] = Lr;
+    const int64_t left = int64_t(a.rows) - r0;
+    const int nr = left < 32 ? static_cast<int>(left) : 32;
+    for (int i = 0; i < nr; ++i) {
+      const int64_t base = ((r0 + i) * a.H + h) * D + lane * E;
+      float acc[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        if (p >= a.nparts) break;
+        const float wp = __shfl_sync(0xffffffffu, wt[p], i);
+        if constexpr (E == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(a.o[p] + base);
+          acc[0] = fmaf(wp, v.x, acc[0]);
+          acc[1] = fmaf(wp, v.y, acc[1]);
+          acc[2] = fmaf(wp, v.z, acc[2]);
+          acc[3] = fmaf(wp, v.w, acc[3]);
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(a.o[p] + base);
+          acc[0] = fmaf(wp, v.x, acc[0]);
+          acc[1] = fmaf(wp, v.y, acc[1]);
+        }
+      }
+      if constexpr (E == 4) {
+        uint2 o;
+        o.x = ptx::pack_bf16x2(acc[0], acc[1]);
+        o.y = ptx::pack_bf16x2(acc[2], acc[3]);
+        *reinterpret_cast<uint2*>(a.o_out + base) = o;
+      } else {
+        *reinterpret_cast<uint32_t*>(a.o_out + base) = ptx::pack_bf16x2(acc[0], acc[1]);
+      }
+    }
+  }
+}
+
+int grid_for(int64_t work, int per_block, int cap) {
+  int64_t g = (work + per_block - 1) / per_block;
+  if (g < 1) g = 1;
+  if (g > cap) g = cap;
+  return static_cast<int>(g);
+}
+
+}  // namespace
+
+cudaError_t launch_plan_rows(const int32_t* cu_seqlens, int ndoc, const int32_t* anchors, int S,
+                             int Nb, int B, int R, const ChunkDev* chunks, int32_t* row_table,
+                             int64_t n_slots, cudaStream_t stream) {
+  const int64_t total = int64_t(S) + int64_t(Nb) * B;
+  plan_rows_kernel<<<grid_for(total, 256, 148 * 16), 256, 0, stream>>>(
+      cu_seqlens, ndoc, anchors, S, Nb, B, R, chunks, row_table, n_slots);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_branch_fwd(const __nv_bfloat16* qb, const __nv_bfloat16* kb,
+                              const __nv_bfloat16* vb, int Nb, int B, int mode, int Hq, int Hkv,
+                              int d, float scale, float* o_part, float* lse_part,
+                              cudaStream_t stream) {
+  if (Nb == 0) return cudaSuccess;
+  const int G = Hq / Hkv;
+  const int threads = G * 32 < 64 ? 64 : G * 32;
+  const size_t smem = size_t(2) * B * d * sizeof(float);
+  const int64_t blocks = int64_t(Nb) * Hkv;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  if (d == 128) {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(branch_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+    branch_fwd_kernel<128><<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
+        qb, kb, vb, Nb, B, mode, Hq, Hkv, scale, o_part, lse_part);
+  } else {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(branch_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+    branch_fwd_kernel<64><<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
+        qb, kb, vb, Nb, B, mode, Hq, Hkv, scale, o_part, lse_part);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lse_merge(const MergeArgs& a, cudaStream_t stream) {
+  const int64_t warps = (int64_t(a.rows) + 31) / 32 * a.H;
+  const int grid = grid_for(warps, 8, 148 * 32);
+  if (a.d == 128)
+    lse_merge_kernel<128><<<grid, 256, 0, stream>>>(a);
+  else
+    lse_merge_kernel<64><<<grid, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ba

@@ -1,0 +1,31 @@
+// Plain structs shared by the host planner and the device kernels.
+#pragma once
+#include <cstdint>
+
+namespace ba {
+
+// One row tile: up to 128 query rows of one zigzag chunk, ordered by their
+// last visible main key ("limit"); ties put the main row first, then the
+// branch rows anchored there (branch-major, depth-minor).
+struct TileDesc {
+  int32_t row_base;   // first slot in the row table (tile index * 128)
+  int32_t n_rows;     // valid rows, 1..128 (slots beyond hold -1)
+  int32_t doc_start;  // first main key of the tile's document
+  int32_t kv_end;     // one past the largest limit in the tile
+  int32_t min_limit;  // smallest limit in the tile
+  int32_t br_lo;      // branch key rows (flattened b*B+u) the tile's branch
+  int32_t br_hi;      //   rows can see: [br_lo, br_hi); empty if br_lo >= br_hi
+  int32_t rank;       // owning virtual rank
+};
+static_assert(sizeof(TileDesc) == 32, "TileDesc must stay 32 bytes");
+
+// Per-chunk data the device row scatter needs.
+struct ChunkDev {
+  int32_t c0;        // first main position of the chunk
+  int32_t b0;        // first branch anchored in the chunk
+  int32_t slot_base; // row-table slot of merged index 0
+  int32_t pad;
+};
+static_assert(sizeof(ChunkDev) == 16, "ChunkDev must stay 16 bytes");
+
+}  // namespace ba

@@ -1,0 +1,191 @@
+/*
+ * ba.h -- branch attention for speculative-draft training on B200 (sm_100a).
+ *
+ * C ABI of libba_b200.so.  Plain pointers and sizes only.
+ *
+ * The operation.  Source: "Online Draft Co-Training for Speculative Decoding
+ * in Large-Scale, Long-Context RL Post-Training" (arXiv 2609.07108), §3.2 and
+ * Eq. 2, as described on the rcap.io post (paragraph on branch attention under
+ * context parallelism) and the evolve.pub review (Summary; FAQ on branch
+ * attention under CP).  A packed main sequence of S tokens (documents given by
+ * cu_seqlens, no padding) carries Nb draft branches; branch b hangs off the
+ * main position anchors[b] and has B rows.  Every query row attends with a
+ * softmax over its visible keys:
+ *   - main row i:        main keys j in [s(i), i]      (s = document start)
+ *   - branch row (b, t): main keys j in [s(a_b), a_b]  (causal prefix up to
+ *                        and including the anchor) plus its own branch keys
+ *                        (b, u) with u <= t (BA_MASK_CHAIN, EAGLE-3 training-
+ *                        time test) or all u < B (BA_MASK_BLOCK, DFlash-style
+ *                        block draft).
+ * Main rows never see branch keys; branches never see each other's keys.
+ * The library computes it the way the paper decomposes it: a causal
+ * main-sequence component over a load-balanced zigzag split (R virtual ranks
+ * on one GPU), a rank-local branch component, and the online-softmax
+ * (log-sum-exp) merge of the two, Eq. 2:
+ *     L = log(exp(L1) + exp(L2)),  O = exp(L1 - L) O1 + exp(L2 - L) O2.
+ * The backward pass (dQ, dK, dV through both parts) is not described on the
+ * pages; it is the textbook softmax-attention gradient of the same definition,
+ * recomputed from the merged LSE.
+ *
+ * Conventions (all entry points):
+ *   - Tensors are row-major with the last dimension contiguous:
+ *       q  bf16 [S, Hq, d]        k, v   bf16 [S, Hkv, d]
+ *       qb bf16 [Nb, B, Hq, d]    kb, vb bf16 [Nb, B, Hkv, d]
+ *     GQA: query head h uses KV head h / (Hq / Hkv).
+ *   - "Rows" are the S main rows followed by the Nb*B branch rows (b-major,
+ *     depth-minor).  LSE arrays are fp32 [Hq, rows] (head-major), natural log.
+ *   - Every device pointer must be 16-byte aligned.  Supported: d in {64, 128},
+ *     Hq % Hkv == 0, 1 <= B <= 64, 1 <= R <= 64.  anchors ascending (ties
+ *     allowed), each in [0, S).  Nb may be 0 (plain packed causal attention).
+ *   - scale <= 0 selects 1/sqrt(d).
+ *   - Ownership: the caller owns every buffer, including the workspace whose
+ *     size ba_workspace_size() returns.  The library allocates no device
+ *     memory on these paths and keeps no per-call state.
+ *   - Work is enqueued on `stream` and runs asynchronously.  Argument errors are
+ *     detected on the host before anything is enqueued.  A device-side bounded
+ *     wait that expires sets a device error word and the kernel returns;
+ *     ba_sync_status() reports it as BA_ERR_TIMEOUT.
+ *   - Results do not depend on R beyond floating-point summation order.
+ */
+#ifndef BA_B200_H
+#define BA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BA_API __attribute__((visibility("default")))
+#else
+#define BA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* ba_stream_t;
+
+typedef enum {
+  BA_OK = 0,
+  BA_ERR_INVALID_ARG = -1, /* bad size, pointer, layout or ordering */
+  BA_ERR_UNSUPPORTED = -2, /* valid but not implemented (e.g. d = 96) */
+  BA_ERR_CUDA = -3,        /* a CUDA runtime call failed */
+  BA_ERR_TIMEOUT = -4,     /* a device-side bounded wait expired */
+  BA_ERR_WORKSPACE = -5    /* workspace missing or too small */
+} ba_status;
+
+typedef enum {
+  BA_MASK_CHAIN = 0, /* EAGLE-3 training-time test: depth t sees branch keys u <= t */
+  BA_MASK_BLOCK = 1  /* DFlash-style block draft: all B keys of its own block */
+} ba_mask_mode;
+
+enum { BA_WS_FWD = 0, BA_WS_BWD = 1 };
+
+typedef struct {
+  int S;      /* packed main tokens (sum of document lengths), >= 1 */
+  int ndoc;   /* documents, >= 1; cu_seqlens has ndoc + 1 entries */
+  int Hq;     /* query heads */
+  int Hkv;    /* key/value heads, Hq % Hkv == 0 */
+  int d;      /* head dimension: 64 or 128 */
+  int Nb;     /* branches (may be 0) */
+  int B;      /* branch depth (chain) or block size (block) */
+  int mode;   /* ba_mask_mode */
+  int R;      /* virtual zigzag ranks, >= 1 */
+  float scale;/* softmax scale; <= 0 selects 1/sqrt(d) */
+  const int32_t* cu_seqlens_h; /* host copy, [ndoc + 1], 0 = c0 < c1 < ... = S */
+  const int32_t* cu_seqlens_d; /* device copy of the same */
+  const int32_t* anchors_h;    /* host copy, [Nb], ascending, in [0, S) */
+  const int32_t* anchors_d;    /* device copy of the same */
+  const void* q;  const void* k;  const void* v;   /* device, bf16 */
+  const void* qb; const void* kb; const void* vb;  /* device, bf16 (ignored if Nb == 0) */
+  void* workspace;        /* device, 256-byte aligned, caller-owned */
+  size_t workspace_bytes; /* its size */
+} ba_problem;
+
+/* Bytes of workspace that ba_main_fwd / ba_fused_fwd (which = BA_WS_FWD) or
+ * ba_bwd (which = BA_WS_BWD) need for this problem.  Returns 0 if the problem
+ * is invalid.  Host only; reads cu_seqlens_h and anchors_h. */
+BA_API size_t ba_workspace_size(const ba_problem* p, int which);
+
+/* Step a2: the causal main-sequence component of every row (main rows, then
+ * branch rows), i.e. each row against main keys [s(limit), limit] with
+ * limit = i for main row i and a_b for branch row (b, t), over the zigzag
+ * split into R virtual ranks.
+ *   o_part   device fp32 [S + Nb*B, Hq, d]: the normalised output of this
+ *            component alone (its softmax runs over main keys only)
+ *   lse_part device fp32 [Hq, S + Nb*B]: its log-sum-exp
+ * Needs ba_workspace_size(p, BA_WS_FWD) bytes of workspace.
+ * Paper: §3.2 (rcap.io post: the main-sequence part is computed by the
+ * existing packed, load-balanced zigzag ring attention). */
+BA_API ba_status ba_main_fwd(const ba_problem* p, float* o_part, float* lse_part, ba_stream_t stream);
+
+/* Step a3: the rank-local branch component: each branch row against its own
+ * branch keys only (chain: u <= t; block: all B).  Needs no workspace.
+ *   o_part   device fp32 [Nb*B, Hq, d]
+ *   lse_part device fp32 [Hq, Nb*B]
+ * Paper: §3.2 (rcap.io post; evolve.pub FAQ: the branch-local part is
+ * computed on the rank that holds the branch's anchor, so branch K/V never
+ * move). */
+BA_API ba_status ba_branch_fwd(const ba_problem* p, float* o_part, float* lse_part, ba_stream_t stream);
+
+/* Step a4: k-way online-softmax merge, Eq. 2, of nparts partial results over
+ * the same rows:  L = log sum_p exp(L_p),  O = sum_p exp(L_p - L) O_p.
+ * A partial with L_p = -inf is empty and contributes nothing; if all are
+ * empty the row gets O = 0, L = -inf.
+ *   o_parts    host array of nparts device pointers, each fp32 [rows, H, d]
+ *   lse_parts  host array of nparts device pointers; element (h, r) of part p
+ *              is lse_parts[p][h * lse_ld[p] + r]
+ *   lse_ld     host array of nparts head strides (>= rows)
+ *   o_out      device bf16 [rows, H, d] (round to nearest even)
+ *   lse_out    device fp32, element (h, r) at lse_out[h * lse_out_ld + r]
+ * 1 <= nparts <= 16; d in {64, 128}.  Needs no workspace.
+ * Paper: Eq. 2 (evolve.pub "Scope & Claims"); the rcap.io post calls it the
+ * log-sum-exp rule ring attention uses between ring steps. */
+BA_API ba_status ba_lse_merge(int nparts, int rows, int H, int d,
+                       const float* const* o_parts, const float* const* lse_parts,
+                       const int64_t* lse_ld, void* o_out, float* lse_out,
+                       int64_t lse_out_ld, ba_stream_t stream);
+
+/* Steps a2 + a3 + a4 in one persistent kernel: the branch-local keys are
+ * visited as extra key tiles of the same online softmax, so the Eq. 2 merge
+ * happens in registers and TMEM.
+ *   o    device bf16 [S, Hq, d]         final output of the main rows
+ *   ob   device bf16 [Nb, B, Hq, d]     final output of the branch rows
+ *   lse  device fp32 [Hq, S + Nb*B]     merged LSE (input to ba_bwd)
+ * Needs ba_workspace_size(p, BA_WS_FWD) bytes of workspace.
+ * Paper: §3.2; the cere-bro wiki page ("Obstacle one, context parallelism")
+ * describes the merge as happening within the ring pass itself. */
+BA_API ba_status ba_fused_fwd(const ba_problem* p, void* o, void* ob, float* lse, ba_stream_t stream);
+
+/* Backward (steps a5-a8; not on the pages): gradients of sum(O * dO) through
+ * both components, recomputed from the merged LSE.
+ *   o, ob, lse      the outputs of ba_fused_fwd
+ *   dout, doutb     bf16, layouts of o and ob
+ *   dq, dk, dv      bf16 [S, Hq, d], [S, Hkv, d], [S, Hkv, d]   (written)
+ *   dqb, dkb, dvb   bf16 [Nb, B, Hq, d], [Nb, B, Hkv, d] x2      (written)
+ * Needs ba_workspace_size(p, BA_WS_BWD) bytes of workspace (fp32 dQ
+ * accumulator, D = rowsum(dO * O), plan). */
+BA_API ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float* lse,
+                 const void* dout, const void* doutb, void* dq, void* dk, void* dv,
+                 void* dqb, void* dkb, void* dvb, ba_stream_t stream);
+
+/* Static description of a status code. */
+BA_API const char* ba_status_string(ba_status s);
+
+/* Synchronises `stream`, then reports (and clears) the device error word of
+ * the current device: BA_ERR_TIMEOUT if a bounded wait expired, BA_ERR_CUDA
+ * if the synchronisation failed, else BA_OK. */
+BA_API ba_status ba_sync_status(ba_stream_t stream);
+
+/* Planner statistics for a problem (host only, no GPU needed): number of row
+ * tiles, (row tile, key tile) pairs the forward kernel visits per query head,
+ * and the exact count of visible (row, key) pairs per query head.  Returns
+ * BA_ERR_INVALID_ARG for an invalid problem. */
+BA_API ba_status ba_plan_stats(const ba_problem* p, int64_t* n_row_tiles, int64_t* n_tile_pairs,
+                        int64_t* n_visible_pairs);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BA_B200_H */

@@ -18,7 +18,7 @@ page ("Obstacle one, context parallelism").
 The pages say a branch query sees the causal prefix of the main sequence up to
 its anchor plus a few branch-local keys, that the two pieces are computed
 separately and merged with the log-sum-exp rule ring attention uses between
-ring steps, and that nothing about the numerics changes.  So the method reaches,
+ring steps, and that the decomposition leaves the numerics unchanged.  So the method reaches,
 up to rounding order, plain masked softmax attention over the concatenated
 [main; branch] rows and keys.  The oracle writes that definition out:
 
@@ -139,6 +139,39 @@ def visible_mask(cu, anchors, B: int, mode: int) -> np.ndarray:
     return M
 
 
+class _Lazy:
+    """fp64 view of rows of a [N, H, d] array/tensor, or of the row-wise
+    concatenation of a main [S, H, d] and a branch [Nb, B, H, d] input,
+    converted only where read (keeps sampled-row checks at large S cheap)."""
+
+    def __init__(self, main, br=None):
+        self.main = main
+        self.S = main.shape[0]
+        self.br = None
+        if br is not None and br.shape[0] * br.shape[1] > 0:
+            self.br = br.reshape(br.shape[0] * br.shape[1], *br.shape[2:])
+
+    @staticmethod
+    def _take(x, idx, h):
+        if hasattr(x, "detach"):
+            import torch
+            t = x[torch.as_tensor(idx, dtype=torch.long), h]
+            return t.detach().cpu().to(torch.float64).numpy()
+        return np.asarray(x[idx, h], dtype=np.float64)
+
+    def rows(self, idx, h):
+        idx = np.asarray(idx, dtype=np.int64)
+        if self.br is None or (idx < self.S).all():
+            return self._take(self.main, idx, h)
+        out = np.empty((len(idx), self.main.shape[2]))
+        m = idx < self.S
+        if m.any():
+            out[m] = self._take(self.main, idx[m], h)
+        if (~m).any():
+            out[~m] = self._take(self.br, idx[~m] - self.S, h)
+        return out
+
+
 def _concat(main, br):
     """[S,H,d] and [Nb,B,H,d] -> [S+Nb*B, H, d]."""
     main = f64(main)
@@ -241,22 +274,29 @@ def _row_blocks(rows, cu, anchors, B, block):
         i = j
 
 
-def _block_scores(Qh, Kmain_g, Kbr_g, s0, lim, bid, dep, B, mode, sc):
+class _Window:
+    """Key rows gathered for one row block: main keys [s0, s0 + n) (``s0`` set)
+    or the listed branch key rows (``ids`` set)."""
+
+    def __init__(self, data, s0, ids=None):
+        self.data, self.s0, self.ids = data, s0, ids
+
+
+def _block_scores(Qh, Kmain, Kbr, s0, lim, bid, dep, B, mode, sc):
     """Scores of a row block against its visible keys: main keys [s0, max lim]
     (masked to each row's limit) and the branch keys of the block's branches
     (masked to each row's own branch and depth rule).  Returns
     (scores [nr, nk], main key index array, branch key index array)."""
     hi = int(lim.max())
     mk = np.arange(s0, hi + 1)
-    s_main = sc * (Qh @ Kmain_g[s0:hi + 1].T)
+    s_main = sc * (Qh @ Kmain.data.T)
     s_main = np.where(mk[None, :] <= lim[:, None], s_main, -np.inf)
-    ub = np.unique(bid[bid >= 0])
-    if len(ub) == 0:
+    if Kbr is None:
         return s_main, mk, np.zeros(0, dtype=np.int64)
-    bk = (ub[:, None] * B + np.arange(B)[None, :]).reshape(-1)  # flat branch key rows
+    bk = Kbr.ids
     kb_b = bk // B
     kb_u = bk % B
-    s_br = sc * (Qh @ Kbr_g[bk].T)
+    s_br = sc * (Qh @ Kbr.data.T)
     vis = (kb_b[None, :] == bid[:, None]) & ((mode == BLOCK) | (kb_u[None, :] <= dep[:, None]))
     s_br = np.where(vis, s_br, -np.inf)
     return np.concatenate([s_main, s_br], axis=1), mk, bk
@@ -266,7 +306,6 @@ def forward_rows(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None, rows=Non
                  heads=None, block=512):
     """O and LSE of the requested concatenated rows (default: all rows).
     Returns (rows [n], O [n, Hq, d], LSE [Hq, n]); heads outside ``heads`` are 0."""
-    q, k, v, qb, kb, vb = (f64(x) for x in (q, k, v, qb, kb, vb))
     S, Hq, d = q.shape
     Hkv = k.shape[1]
     Nb = qb.shape[0]
@@ -276,21 +315,27 @@ def forward_rows(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None, rows=Non
         rows = np.arange(S + Nb * B)
     rows = np.asarray(rows, dtype=np.int64)
     heads = list(range(Hq)) if heads is None else list(heads)
-    Qc = np.concatenate([q, qb.reshape(-1, Hq, d)], axis=0)
-    kbf = kb.reshape(-1, Hkv, d)
-    vbf = vb.reshape(-1, Hkv, d)
+    Qc = _Lazy(q, qb)
+    Km, Vm = _Lazy(k), _Lazy(v)
+    Kb, Vb = _Lazy(kb.reshape(-1, 1, Hkv, d)[:, 0] if Nb else k[:0]), _Lazy(vb.reshape(-1, 1, Hkv, d)[:, 0] if Nb else v[:0])
     pos = {int(r): n for n, r in enumerate(rows)}
     O = np.zeros((len(rows), Hq, d))
     L = np.full((Hq, len(rows)), np.nan)
     for r, s0, lim, bid, dep in _row_blocks(rows, cu, anchors, B, block):
         idx = np.array([pos[int(x)] for x in r])
+        hi = int(lim.max())
+        mk = np.arange(s0, hi + 1)
+        ub = np.unique(bid[bid >= 0])
+        bk = (ub[:, None] * B + np.arange(B)[None, :]).reshape(-1) if len(ub) else np.zeros(0, np.int64)
         for h in heads:
             g = h // G
-            s, mk, bk = _block_scores(Qc[r, h], k[:, g], kbf[:, g], s0, lim, bid, dep, B, mode, sc)
+            Kmain = _Window(Km.rows(mk, g), s0)
+            Kbr = _Window(Kb.rows(bk, g), None, bk) if len(bk) else None
+            s, _, _ = _block_scores(Qc.rows(r, h), Kmain, Kbr, s0, lim, bid, dep, B, mode, sc)
             m = s.max(axis=1, keepdims=True)
             e = np.exp(s - m)
             l = e.sum(axis=1, keepdims=True)
-            Vv = np.concatenate([v[mk, g], vbf[bk, g]], axis=0)
+            Vv = np.concatenate([Vm.rows(mk, g), Vb.rows(bk, g) if len(bk) else np.zeros((0, d))], axis=0)
             O[idx, h] = (e / l) @ Vv
             L[h, idx] = (m + np.log(l))[:, 0]
     return rows, O, L
@@ -302,7 +347,6 @@ def backward_rows(q, k, v, qb, kb, vb, do, dob, cu, anchors, B, mode, scale=None
     rows (default: all rows).  With dO zero outside ``rows`` this is the exact
     full gradient.  Returns (rows, dQ [n, Hq, d] of those rows,
     dk, dv [S,Hkv,d], dkb, dvb [Nb,B,Hkv,d]); only ``heads`` contribute."""
-    q, k, v, qb, kb, vb, do, dob = (f64(x) for x in (q, k, v, qb, kb, vb, do, dob))
     S, Hq, d = q.shape
     Hkv = k.shape[1]
     Nb = qb.shape[0]
@@ -312,33 +356,42 @@ def backward_rows(q, k, v, qb, kb, vb, do, dob, cu, anchors, B, mode, scale=None
         rows = np.arange(S + Nb * B)
     rows = np.asarray(rows, dtype=np.int64)
     heads = list(range(Hq)) if heads is None else list(heads)
-    Qc = np.concatenate([q, qb.reshape(-1, Hq, d)], axis=0)
-    dOc = np.concatenate([do, dob.reshape(-1, Hq, d)], axis=0)
-    kbf = kb.reshape(-1, Hkv, d)
-    vbf = vb.reshape(-1, Hkv, d)
-    dk = np.zeros_like(k)
-    dv = np.zeros_like(v)
-    dkbf = np.zeros_like(kbf)
-    dvbf = np.zeros_like(vbf)
+    Qc = _Lazy(q, qb)
+    dOc = _Lazy(do, dob)
+    Km, Vm = _Lazy(k), _Lazy(v)
+    Kb = _Lazy(kb.reshape(-1, 1, Hkv, d)[:, 0] if Nb else k[:0])
+    Vb = _Lazy(vb.reshape(-1, 1, Hkv, d)[:, 0] if Nb else v[:0])
+    dk = np.zeros((S, Hkv, d))
+    dv = np.zeros((S, Hkv, d))
+    dkbf = np.zeros((Nb * B, Hkv, d))
+    dvbf = np.zeros((Nb * B, Hkv, d))
     pos = {int(r): n for n, r in enumerate(rows)}
     dQ = np.zeros((len(rows), Hq, d))
     for r, s0, lim, bid, dep in _row_blocks(rows, cu, anchors, B, block):
         idx = np.array([pos[int(x)] for x in r])
+        hi = int(lim.max())
+        mk = np.arange(s0, hi + 1)
+        ub = np.unique(bid[bid >= 0])
+        bk = (ub[:, None] * B + np.arange(B)[None, :]).reshape(-1) if len(ub) else np.zeros(0, np.int64)
         for h in heads:
             g = h // G
-            s, mk, bk = _block_scores(Qc[r, h], k[:, g], kbf[:, g], s0, lim, bid, dep, B, mode, sc)
+            Km_g = Km.rows(mk, g)
+            Kb_g = Kb.rows(bk, g) if len(bk) else np.zeros((0, d))
+            Qh = Qc.rows(r, h)
+            s, _, _ = _block_scores(Qh, _Window(Km_g, s0), _Window(Kb_g, None, bk) if len(bk) else None,
+                                    s0, lim, bid, dep, B, mode, sc)
             m = s.max(axis=1, keepdims=True)
             e = np.exp(s - m)
             P = e / e.sum(axis=1, keepdims=True)
-            Kk = np.concatenate([k[mk, g], kbf[bk, g]], axis=0)
-            Vv = np.concatenate([v[mk, g], vbf[bk, g]], axis=0)
+            Kk = np.concatenate([Km_g, Kb_g], axis=0)
+            Vv = np.concatenate([Vm.rows(mk, g), Vb.rows(bk, g) if len(bk) else np.zeros((0, d))], axis=0)
             O = P @ Vv
-            dOh = dOc[r, h]
+            dOh = dOc.rows(r, h)
             Dv = (dOh * O).sum(axis=1, keepdims=True)
             dP = dOh @ Vv.T
             dS = P * (dP - Dv)
             dQ[idx, h] = sc * (dS @ Kk)
-            gk = sc * (dS.T @ Qc[r, h])
+            gk = sc * (dS.T @ Qh)
             gv = P.T @ dOh
             nm = len(mk)
             dk[mk, g] += gk[:nm]

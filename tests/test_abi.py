@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+include/ba.h declares, rejects invalid problems before launching anything,
+and its planner matches a Python restatement of the zigzag row tiling.
+No GPU needed."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ba():
+    from branch_attention_speculative_packed_b200 import build
+    build.build()
+    import branch_attention_speculative_packed_b200 as m
+    return m
+
+
+def _declared():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"BA_API\s+[\w\s\*]+?\b(ba_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(ba):
+    declared = _declared()
+    assert "ba_fused_fwd" in declared and "ba_bwd" in declared
+    L = ba.lib()
+    for name in declared:
+        assert hasattr(L, name), name
+    assert sorted(ba.EXPORTED) == sorted(declared) or set(ba.EXPORTED) <= set(declared)
+
+
+def test_status_strings(ba):
+    for s in (0, -1, -2, -3, -4, -5):
+        assert isinstance(ba.status_string(s), str) and ba.status_string(s)
+
+
+def _attn(ba, cu, anc, **kw):
+    args = dict(Hq=4, Hkv=2, d=128, B=3, mode=0, R=2, device="cpu")
+    args.update(kw)
+    return ba.BranchAttention(cu, anc, **args)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(cu=[0, 5, 5, 10], anc=[1]),          # empty document
+    dict(cu=[0, 6, 4, 10], anc=[1]),          # decreasing
+    dict(cu=[1, 5, 10], anc=[1]),             # does not start at 0
+    dict(cu=[0, 5, 10], anc=[3, 2]),          # anchors not ascending
+    dict(cu=[0, 5, 10], anc=[10]),            # anchor out of range
+    dict(cu=[0, 5, 10], anc=[-1]),            # negative anchor
+    dict(cu=[0, 5, 10], anc=[1], Hq=3),       # Hq % Hkv != 0
+    dict(cu=[0, 5, 10], anc=[1], R=0),        # no ranks
+    dict(cu=[0, 5, 10], anc=[1], R=65),       # too many ranks
+    dict(cu=[0, 5, 10], anc=[1], B=0),        # empty branches
+    dict(cu=[0, 5, 10], anc=[1], mode=2),     # unknown mask
+    dict(cu=[0, 5, 10], anc=[1], d=96),       # unsupported head dim
+])
+def test_invalid_problems_rejected(ba, bad):
+    bad = dict(bad)
+    cu, anc = bad.pop("cu"), bad.pop("anc")
+    a = _attn(ba, cu, anc, **bad)
+    with pytest.raises(ValueError):
+        a.workspace_size(ba.BA_WS_FWD)
+    with pytest.raises(ba.BAError):
+        a.plan_stats()
+
+
+def test_duplicate_anchors_accepted(ba):
+    a = _attn(ba, [0, 5, 10], [2, 2, 7])
+    assert a.workspace_size(ba.BA_WS_FWD) > 0
+
+
+# ---------------------------------------------------------------------------
+# planner restated in Python
+# ---------------------------------------------------------------------------
+
+def _restated_plan(cu, anc, B, R):
+    """Row tiles per zigzag chunk: rows sorted by (limit, main-before-branch,
+    branch index, depth), cut into 128-row tiles; a tile visits the main key
+    tiles [doc start, max limit] in steps of 128."""
+    cu = list(cu)
+    anc = list(anc)
+    S = cu[-1]
+    tiles = 0
+    pairs = 0
+    for (di, k, c0, c1, rank) in orc.zigzag_chunks(np.array(cu), R):
+        s = cu[di]
+        rows = [(p, 0, 0, 0) for p in range(c0, c1)]
+        rows += [(a, 1, b, t) for b, a in enumerate(anc) if c0 <= a < c1 for t in range(B)]
+        rows.sort()
+        for i in range(0, len(rows), 128):
+            tile = rows[i:i + 128]
+            tiles += 1
+            pairs += -(-(tile[-1][0] - s + 1) // 128)
+    return tiles, pairs
+
+
+@pytest.mark.parametrize("case", [
+    ([0, 256], [23, 43, 60, 72, 179, 200, 201, 255], 4, 2),
+    ([0, 3, 10, 700, 1000], list(range(0, 1000, 7)), 3, 4),
+    ([0, 1, 2, 3], [0, 1, 2], 2, 8),           # documents shorter than 2R
+    ([0, 500], [], 3, 3),                     # no branches
+    ([0, 300, 301], [299, 299, 300], 16, 1),  # duplicate anchors, anchor on 1-token doc
+])
+def test_planner_matches_restatement(ba, case):
+    cu, anc, B, R = case
+    a = _attn(ba, cu, anc, B=B, R=R)
+    st = a.plan_stats()
+    t, p = _restated_plan(cu, anc, B, R)
+    assert st["row_tiles"] == t
+    assert st["tile_pairs"] == p
+    assert st["visible_pairs"] == orc.visible_pair_count(np.array(cu), np.array(anc), B, 0)
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2, 3])
+def test_planner_on_workload_layouts(ba, idx):
+    cfg = wl.CONFIGS[idx]
+    cu, anc = wl.make_layout(idx)
+    a = ba.BranchAttention(cu, anc, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, B=cfg.B, mode=cfg.mode,
+                           R=cfg.R, device="cpu")
+    st = a.plan_stats()
+    assert st["visible_pairs"] == orc.visible_pair_count(cu.numpy(), anc.numpy(), cfg.B, cfg.mode)
+    if idx <= 2:
+        t, p = _restated_plan(cu.tolist(), anc.tolist(), cfg.B, cfg.R)
+        assert (st["row_tiles"], st["tile_pairs"]) == (t, p)
+    # every visible pair lies in a visited tile pair
+    assert st["tile_pairs"] * 128 * 128 >= st["visible_pairs"] - cfg.n_anchors * cfg.B * cfg.B
