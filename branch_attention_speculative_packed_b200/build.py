@@ -16,8 +16,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libba_b200.so")
-SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "small.cu", "plan.cpp"]
-HEADERS = ["kernels.h", "plan.h", "ptx.cuh", "tile_desc.h"]
+SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "bwd_dq.cu", "bwd_dkdv.cu", "small.cu", "plan.cpp"]
+HEADERS = ["kernels.h", "bwd_kernels.h", "plan.h", "ptx.cuh", "tile_desc.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "../../include/ba.h"
+#include "bwd_kernels.h"
 #include "kernels.h"
 #include "plan.h"
 
@@ -67,6 +68,7 @@ ba_status device_info(DeviceInfo* out) {
 // 2-D bf16 tensor map over a [rows, cols] row-major matrix, box [box_rows, 64]
 // with 128-byte swizzle.
 ba_status encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  // bf16 matrix [rows, cols], box [box_rows, 64 columns = 128 bytes], 128-byte swizzle
   if (rows < 1) rows = 1;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
@@ -265,7 +267,155 @@ ba_status ba_lse_merge(int nparts, int rows, int H, int d, const float* const* o
 
 ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float* lse,
                  const void* dout, const void* doutb, void* dq, void* dk, void* dv, void* dqb,
-                 void* dkb, void* dvb, ba_stream_t stream);
+                 void* dkb, void* dvb, ba_stream_t stream) {
+  ba_status s = validate(p, true);
+  if (s != BA_OK) return s;
+  const bool nb = p->Nb > 0;
+  const void* need[] = {o, lse, dout, dq, dk, dv};
+  for (const void* x : need)
+    if (!x || !aligned16(x)) return BA_ERR_INVALID_ARG;
+  if (nb) {
+    const void* needb[] = {ob, doutb, dqb, dkb, dvb};
+    for (const void* x : needb)
+      if (!x || !aligned16(x)) return BA_ERR_INVALID_ARG;
+  }
+  DeviceInfo di;
+  if ((s = device_info(&di)) != BA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Plan plan;
+  build_plan(p, &plan);
+  build_kv_plan(p, &plan);
+  const WorkspaceLayout w = workspace_layout(p, plan, BA_WS_BWD);
+  if ((s = check_workspace(p, w)) != BA_OK) return s;
+  if ((s = stage_plan(p, plan, w, st)) != BA_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  const size_t nkv = plan.kv_items.size();
+  if (nkv > 0 &&
+      (cudaMemcpyAsync(ws + w.kv_items_off, plan.kv_items.data(), nkv * sizeof(KvItem),
+                       cudaMemcpyHostToDevice, st) != cudaSuccess ||
+       cudaMemcpyAsync(ws + w.kv_order_off, plan.kv_order.data(), nkv * sizeof(int32_t),
+                       cudaMemcpyHostToDevice, st) != cudaSuccess))
+    return BA_ERR_CUDA;
+  const int64_t rows = int64_t(p->S) + int64_t(p->Nb) * plan.B;
+  const float scale = scale_of(p);
+  const int G = p->Hq / p->Hkv;
+  const int64_t items_q = int64_t(plan.tiles.size()) * p->Hq;
+  const int64_t items_kv = int64_t(nkv) * p->Hkv;
+  if (items_q > 0x7fffffff || items_kv > 0x7fffffff) return BA_ERR_UNSUPPORTED;
+
+  // 1. pre-pass
+  PrepArgs pa;
+  std::memset(&pa, 0, sizeof(pa));
+  pa.row_table = reinterpret_cast<const int32_t*>(ws + w.rows_off);
+  pa.anchors = p->anchors_d;
+  pa.q = static_cast<const __nv_bfloat16*>(p->q);
+  pa.qb = static_cast<const __nv_bfloat16*>(nb ? p->qb : p->q);
+  pa.o = static_cast<const __nv_bfloat16*>(o);
+  pa.ob = static_cast<const __nv_bfloat16*>(nb ? ob : o);
+  pa.dout = static_cast<const __nv_bfloat16*>(dout);
+  pa.dob = static_cast<const __nv_bfloat16*>(nb ? doutb : dout);
+  pa.lse = lse;
+  pa.S = p->S;
+  pa.B = plan.B > 0 ? plan.B : 1;
+  pa.mode = p->mode;
+  pa.Hq = p->Hq;
+  pa.rows = rows;
+  pa.n_slots = w.n_slots;
+  pa.qg = reinterpret_cast<__nv_bfloat16*>(ws + w.qg_off);
+  pa.dog = reinterpret_cast<__nv_bfloat16*>(ws + w.dog_off);
+  pa.ls = reinterpret_cast<float*>(ws + w.ls_off);
+  pa.ds = reinterpret_cast<float*>(ws + w.ds_off);
+  pa.drow = reinterpret_cast<float*>(ws + w.drow_off);
+  pa.meta = reinterpret_cast<SlotMeta*>(ws + w.meta_off);
+  if (launch_bwd_prep(pa, p->d, st) != cudaSuccess) return BA_ERR_CUDA;
+
+  // tensor maps
+  const int64_t qcols = int64_t(p->Hq) * p->d, kcols = int64_t(p->Hkv) * p->d;
+  const int64_t nb_rows_map = nb ? int64_t(p->Nb) * plan.B : p->S;
+  DqMaps dm;
+  DkdvMaps km;
+  if (encode_2d(&dm.qg, pa.qg, w.n_slots, qcols, 128) != BA_OK ||
+      encode_2d(&dm.dog, pa.dog, w.n_slots, qcols, 128) != BA_OK ||
+      encode_2d(&dm.k, p->k, p->S, kcols, 128) != BA_OK ||
+      encode_2d(&dm.v, p->v, p->S, kcols, 128) != BA_OK ||
+      encode_2d(&dm.kb, nb ? p->kb : p->k, nb_rows_map, kcols, 128) != BA_OK ||
+      encode_2d(&dm.vb, nb ? p->vb : p->v, nb_rows_map, kcols, 128) != BA_OK ||
+      encode_2d(&km.qg, pa.qg, w.n_slots, qcols, 64) != BA_OK ||
+      encode_2d(&km.dog, pa.dog, w.n_slots, qcols, 64) != BA_OK)
+    return BA_ERR_CUDA;
+  km.k = dm.k;
+  km.v = dm.v;
+
+  // 2. dQ (main and branch keys)
+  DqArgs qa;
+  std::memset(&qa, 0, sizeof(qa));
+  qa.tiles = reinterpret_cast<const TileDesc*>(ws + w.tiles_off);
+  qa.order = reinterpret_cast<const int32_t*>(ws + w.order_off);
+  qa.meta = pa.meta;
+  qa.ls = pa.ls;
+  qa.ds = pa.ds;
+  qa.S = p->S;
+  qa.Hq = p->Hq;
+  qa.G = G;
+  qa.d = p->d;
+  qa.n_slots = w.n_slots;
+  qa.n_items = static_cast<int>(items_q);
+  qa.with_branch = nb ? 1 : 0;
+  qa.scale_log2 = scale * 1.4426950408889634f;
+  qa.scale = scale;
+  qa.dq = static_cast<__nv_bfloat16*>(dq);
+  qa.dqb = static_cast<__nv_bfloat16*>(nb ? dqb : dq);
+  qa.err = di.err;
+  qa.wait_limit = kWaitLimitCycles;
+  if (launch_bwd_dq(dm, qa, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
+
+  // 3. dK, dV of the main keys
+  DkdvArgs ka;
+  std::memset(&ka, 0, sizeof(ka));
+  ka.items = reinterpret_cast<const KvItem*>(ws + w.kv_items_off);
+  ka.order = reinterpret_cast<const int32_t*>(ws + w.kv_order_off);
+  ka.tiles = qa.tiles;
+  ka.meta = pa.meta;
+  ka.ls = pa.ls;
+  ka.ds = pa.ds;
+  ka.Hq = p->Hq;
+  ka.Hkv = p->Hkv;
+  ka.G = G;
+  ka.d = p->d;
+  ka.n_slots = w.n_slots;
+  ka.n_items = static_cast<int>(items_kv);
+  ka.scale_log2 = qa.scale_log2;
+  ka.scale = scale;
+  ka.dk = static_cast<__nv_bfloat16*>(dk);
+  ka.dv = static_cast<__nv_bfloat16*>(dv);
+  ka.err = di.err;
+  ka.wait_limit = kWaitLimitCycles;
+  if (launch_bwd_dkdv(km, ka, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
+
+  // 4. dK, dV of the branch keys
+  if (nb) {
+    BranchBwdArgs ba_;
+    std::memset(&ba_, 0, sizeof(ba_));
+    ba_.qb = static_cast<const __nv_bfloat16*>(p->qb);
+    ba_.kb = static_cast<const __nv_bfloat16*>(p->kb);
+    ba_.vb = static_cast<const __nv_bfloat16*>(p->vb);
+    ba_.dob = static_cast<const __nv_bfloat16*>(doutb);
+    ba_.lse = lse;
+    ba_.drow = pa.drow;
+    ba_.S = p->S;
+    ba_.Nb = p->Nb;
+    ba_.B = p->B;
+    ba_.mode = p->mode;
+    ba_.Hq = p->Hq;
+    ba_.Hkv = p->Hkv;
+    ba_.rows = rows;
+    ba_.scale = scale;
+    ba_.dkb = static_cast<__nv_bfloat16*>(dkb);
+    ba_.dvb = static_cast<__nv_bfloat16*>(dvb);
+    if (launch_branch_bwd(ba_, p->d, st) != cudaSuccess) return BA_ERR_CUDA;
+  }
+  return BA_OK;
+}
 
 const char* ba_status_string(ba_status s) {
   switch (s) {

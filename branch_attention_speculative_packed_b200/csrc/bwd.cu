@@ -1,8 +1,191 @@
-// Backward pass (placeholder until the tcgen05 backward lands).
-#include "../../include/ba.h"
+// Backward pass: pre-pass, branch-local dK/dV and the host orchestration of
+// ba_bwd.  The pages do not describe the backward; it is the softmax-attention
+// gradient of the same masked attention, recomputed from the merged LSE:
+//   D_i = <dO_i, O_i>,  P_ij = exp(s_ij - L_i),  dS_ij = P_ij (<dO_i, v_j> - D_i)
+//   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,  dV_j = sum_i P_ij dO_i
+// With the merged L and D, each component's backward is plain attention
+// backward restricted to that component's keys, and the two add; no separate
+// backward of the Eq. 2 merge is needed.
+//
+// Kernels, in launch order:
+//   1. bwd_prep (HBM-bound): D = rowsum(dO * O); Q and dO gathered into
+//      row-tile slot order (so both tensor-core passes load whole tiles with
+//      plain TMA boxes); per-slot log2-scaled L, D and key-range metadata.
+//   2. bwd_dq (tcgen05, query-stationary): dQ over main and branch keys.
+//   3. bwd_dkdv (tcgen05, key-stationary): dK, dV of the main keys.
+//   4. branch_bwd (SIMT): dK, dV of the branch keys (a handful of pairs each).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
 
-extern "C" ba_status ba_bwd(const ba_problem*, const void*, const void*, const float*,
-                            const void*, const void*, void*, void*, void*, void*, void*, void*,
-                            ba_stream_t) {
-  return BA_ERR_UNSUPPORTED;
+#include <cmath>
+#include <cstring>
+
+#include "../../include/ba.h"
+#include "bwd_kernels.h"
+#include "plan.h"
+
+namespace ba {
+namespace {
+
+// ------------------------------------------------------------------ pre-pass
+// One group of D/8 threads per (slot, head); each thread moves 16 bytes of
+// the row.  Slots are the row-table entries (tile * 128 + i).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepArgs a) {
+  constexpr int TPR = D / 8;  // threads per (slot, head)
+  const int64_t pairs = a.n_slots * a.Hq;
+  const int sub = threadIdx.x % TPR;
+  const int64_t stride = (int64_t(gridDim.x) * blockDim.x) / TPR;
+  for (int64_t pr = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / TPR; pr < pairs; pr += stride) {
+    const int64_t slot = pr / a.Hq;
+    const int h = static_cast<int>(pr % a.Hq);
+    const int r = a.row_table[slot];
+    uint4 qv = make_uint4(0, 0, 0, 0), dv = make_uint4(0, 0, 0, 0);
+    float dsum = 0.f;
+    if (r >= 0) {
+      const bool br = r >= a.S;
+      const int64_t rr = br ? r - a.S : r;
+      const int64_t off = (rr * a.Hq + h) * D + sub * 8;
+      qv = *reinterpret_cast<const uint4*>((br ? a.qb : a.q) + off);
+      dv = *reinterpret_cast<const uint4*>((br ? a.dob : a.dout) + off);
+      const uint4 ov = *reinterpret_cast<const uint4*>((br ? a.ob : a.o) + off);
+      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(d2[i]);
+        const float2 y = __bfloat1622float2(o2[i]);
+        dsum = fmaf(x.x, y.x, dsum);
+        dsum = fmaf(x.y, y.y, dsum);
+      }
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off, TPR);
+    const int64_t goff = (slot * a.Hq + h) * D + sub * 8;
+    *reinterpret_cast<uint4*>(a.qg + goff) = qv;
+    *reinterpret_cast<uint4*>(a.dog + goff) = dv;
+    if (sub == 0) {
+      const int64_t hs = int64_t(h) * a.n_slots + slot;
+      if (r >= 0) {
+        a.ls[hs] = a.lse[int64_t(h) * a.rows + r] * 1.4426950408889634f;
+        a.ds[hs] = dsum;
+        a.drow[int64_t(h) * a.rows + r] = dsum;
+      } else {
+        a.ls[hs] = INFINITY;  // padding: P = exp2(s - inf) = 0
+        a.ds[hs] = 0.f;
+      }
+      if (h == 0) {
+        SlotMeta m;
+        m.limit = -1;
+        m.blo = m.bhi = 0;
+        m.row = r;
+        if (r >= 0 && r < a.S) {
+          m.limit = r;
+        } else if (r >= a.S) {
+          const int b = (r - a.S) / a.B;
+          const int t = (r - a.S) - b * a.B;
+          m.limit = a.anchors[b];
+          m.blo = b * a.B;
+          m.bhi = m.blo + (a.mode == 1 ? a.B : t + 1);
+        }
+        a.meta[slot] = m;
+      }
+    }
+  }
 }
+
+// ------------------------------------------------------------------ branch dK/dV
+// One block per (branch b, KV head g); one warp per branch key u (strided).
+// Lane l holds elements [l*E, l*E + E) of k_u, v_u and of the accumulators.
+// For every query head of the group and every row t that sees u:
+//   s = scale <q_t, k_u>, P = exp(s - L_t), dS = P (<dO_t, v_u> - D_t),
+//   dV_u += P dO_t, dK_u += scale dS q_t.
+template <int D>
+__global__ void branch_bwd_kernel(const BranchBwdArgs a) {
+  constexpr int E = D / 32;
+  const int b = blockIdx.x / a.Hkv;
+  const int g = blockIdx.x % a.Hkv;
+  const int G = a.Hq / a.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  const int64_t base_row = int64_t(a.S) + int64_t(b) * a.B;  // concatenated row of (b, 0)
+  for (int u = warp; u < a.B; u += nw) {
+    const int64_t ku = ((int64_t(b) * a.B + u) * a.Hkv + g) * D + lane * E;
+    float kf[E], vf[E], dk[E], dv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      kf[e] = __bfloat162float(a.kb[ku + e]);
+      vf[e] = __bfloat162float(a.vb[ku + e]);
+      dk[e] = 0.f;
+      dv[e] = 0.f;
+    }
+    for (int hh = 0; hh < G; ++hh) {
+      const int h = g * G + hh;
+      for (int t = (a.mode == 1 ? 0 : u); t < a.B; ++t) {
+        const int64_t qo = ((int64_t(b) * a.B + t) * a.Hq + h) * D + lane * E;
+        float qf[E], df[E];
+        float s = 0.f, dp = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          qf[e] = __bfloat162float(a.qb[qo + e]);
+          df[e] = __bfloat162float(a.dob[qo + e]);
+          s = fmaf(qf[e], kf[e], s);
+          dp = fmaf(df[e], vf[e], dp);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          s += __shfl_xor_sync(0xffffffffu, s, off);
+          dp += __shfl_xor_sync(0xffffffffu, dp, off);
+        }
+        const int64_t row = base_row + t;
+        const float P = expf(s * a.scale - a.lse[int64_t(h) * a.rows + row]);
+        const float dS = P * (dp - a.drow[int64_t(h) * a.rows + row]);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          dv[e] = fmaf(P, df[e], dv[e]);
+          dk[e] = fmaf(dS, qf[e], dk[e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      a.dkb[ku + e] = __float2bfloat16_rn(dk[e] * a.scale);
+      a.dvb[ku + e] = __float2bfloat16_rn(dv[e]);
+    }
+  }
+}
+
+int grid_cap(int64_t work, int per_block, int cap) {
+  int64_t g = (work + per_block - 1) / per_block;
+  if (g < 1) g = 1;
+  if (g > cap) g = cap;
+  return static_cast<int>(g);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_prep(const PrepArgs& a, int d, cudaStream_t st) {
+  const int tpr = d / 8;
+  const int64_t threads = a.n_slots * a.Hq * tpr;
+  const int grid = grid_cap(threads, 256, 148 * 32);
+  if (d == 128)
+    bwd_prep_kernel<128><<<grid, 256, 0, st>>>(a);
+  else
+    bwd_prep_kernel<64><<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_branch_bwd(const BranchBwdArgs& a, int d, cudaStream_t st) {
+  if (a.Nb == 0) return cudaSuccess;
+  const int64_t blocks = int64_t(a.Nb) * a.Hkv;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  const int warps = a.B < 8 ? a.B : 8;
+  if (d == 128)
+    branch_bwd_kernel<128><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(a);
+  else
+    branch_bwd_kernel<64><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ba

@@ -1,0 +1,415 @@
+// dK/dV pass of the backward on sm_100a (key-stationary, tcgen05 + TMEM).
+//
+// One persistent CTA per SM walks (main key tile, KV head) items, most work
+// first.  The item's K and V tiles (128 keys) stay in shared memory; the CTA
+// visits every row tile that can see them (a contiguous range of the plan's
+// tiles), for each of the G query heads of the KV head, in halves of 64 rows:
+//   S^T  = K Q^T      [128 keys x 64 rows]  -> TMEM (two buffers)
+//   dP^T = V dO^T     [128 x 64]            -> TMEM (two buffers)
+//   threads (one key per thread): P^T = exp2(S^T*scale*log2e - L*log2e) where
+//       key <= the row's limit, dS^T = P^T (dP^T - D)  -> shared memory (bf16)
+//   dV += P^T dO,  dK += dS^T Q             -> TMEM accumulators
+// and finally dK * scale and dV are written as bf16 for the keys this item
+// owns (a key tile may run past its document's end; those keys belong to the
+// next document's items and are not written here).
+//
+// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-5
+// one key row each.  TMEM: dK 0..127, dV 128..255, S^T 256 / 320, dP^T 384 / 448.
+// Shared memory: K | V | 3 stages of (Q half, dO half, L, D, slot metadata) |
+// P^T | dS^T.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "bwd_kernels.h"
+#include "ptx.cuh"
+
+namespace ba {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 3;
+constexpr int kHalf = 64;  // query rows per sub-tile
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;
+
+template <int D>
+struct Smem {
+  static constexpr uint32_t kKVBytes = 128u * D * 2u;       // K or V tile
+  static constexpr uint32_t kHalfBytes = kHalf * D * 2u;    // Q or dO half tile
+  static constexpr uint32_t kMetaBytes = kHalf * (4u + 4u + 16u);  // L, D, SlotMeta
+  static constexpr uint32_t kStageBytes = ((2u * kHalfBytes + kMetaBytes) + 1023u) / 1024u * 1024u;
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = kK + kKVBytes;
+  static constexpr uint32_t kStage0 = kV + kKVBytes;
+  static constexpr uint32_t kPT = kStage0 + kStages * kStageBytes;
+  static constexpr uint32_t kDST = kPT + 128u * kHalf * 2u;
+  static constexpr uint32_t kBar = kDST + 128u * kHalf * 2u;
+  // kv_full, kv_empty, st_full[3], st_empty[3], sd_full[2], sd_empty[2], pd_full, pd_free,
+  // acc_full, acc_free, drain
+  static constexpr uint32_t kNumBars = 19;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8u;
+  static constexpr uint32_t kTotal = kMisc + 16u;
+  static constexpr uint32_t kAlloc = kTotal + 1024u;
+  // offsets inside a stage
+  static constexpr uint32_t kSQ = 0, kSDO = kHalfBytes, kSL = 2u * kHalfBytes;
+  static constexpr uint32_t kSD = kSL + kHalf * 4u, kSM = kSD + kHalf * 4u;
+  static constexpr uint32_t kStageTx = 2u * kHalfBytes + kMetaBytes;
+};
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                    const DkdvArgs a) {
+  using L = Smem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t b0 = sbase + L::kBar;
+  const uint32_t bar_kv_full = b0, bar_kv_empty = b0 + 8;
+  auto bar_st_full = [&](uint32_t s) { return b0 + 16 + 8 * s; };
+  auto bar_st_empty = [&](uint32_t s) { return b0 + 40 + 8 * s; };
+  auto bar_sd_full = [&](uint32_t s) { return b0 + 64 + 8 * s; };
+  auto bar_sd_empty = [&](uint32_t s) { return b0 + 80 + 8 * s; };
+  const uint32_t bar_pd_full = b0 + 96, bar_pd_free = b0 + 104;
+  const uint32_t bar_acc_full = b0 + 112, bar_acc_free = b0 + 120, bar_drain = b0 + 128;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar_kv_full, 1);
+    ptx::mbar_init(bar_kv_empty, 1);
+    for (uint32_t i = 0; i < kStages; ++i) {
+      ptx::mbar_init(bar_st_full(i), 1);
+      ptx::mbar_init(bar_st_empty(i), 1);
+    }
+    for (uint32_t i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar_sd_full(i), 1);
+      ptx::mbar_init(bar_sd_empty(i), 128);
+    }
+    ptx::mbar_init(bar_pd_full, 128);
+    ptx::mbar_init(bar_pd_free, 1);
+    ptx::mbar_init(bar_acc_full, 1);
+    ptx::mbar_init(bar_acc_free, 128);
+    ptx::mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmK);
+    ptx::prefetch_tmap(&tmV);
+    ptx::prefetch_tmap(&tmQ);
+    ptx::prefetch_tmap(&tmDO);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(sbase + L::kMisc, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int G = a.G;
+  const long long lim = a.wait_limit;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t kv_phase = 0, st = 0, st_phase = 0;
+      uint32_t pend_mask = 0, pend_par = 0, kv_fills = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+        const KvItem it = a.items[a.order[item / a.Hkv]];
+        const int g = item % a.Hkv;
+        if (!ptx::mbar_wait(bar_kv_empty, kv_phase ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+        kv_phase ^= 1u;
+        ptx::mbar_expect_tx(bar_kv_full, 2u * L::kKVBytes);
+        ++kv_fills;
+#pragma unroll
+        for (int cb = 0; cb < D / 64; ++cb) {
+          ptx::tma_load_2d(sbase + L::kK + cb * 16384u, &tmK, bar_kv_full, g * D + cb * 64, it.key0);
+          ptx::tma_load_2d(sbase + L::kV + cb * 16384u, &tmV, bar_kv_full, g * D + cb * 64, it.key0);
+        }
+        for (int ti = 0; ti < it.t_count && ok; ++ti) {
+          const TileDesc td = a.tiles[it.t_first + ti];
+          const int nh = (td.n_rows + kHalf - 1) / kHalf;
+          for (int hh = 0; hh < G && ok; ++hh) {
+            const int h = g * G + hh;
+            for (int half = 0; half < nh; ++half) {
+              if (!ptx::mbar_wait(bar_st_empty(st), st_phase ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+              const uint32_t sb = sbase + L::kStage0 + st * L::kStageBytes;
+              const int slot0 = td.row_base + half * kHalf;
+              ptx::mbar_expect_tx(bar_st_full(st), L::kStageTx);
+#pragma unroll
+              for (int cb = 0; cb < D / 64; ++cb) {
+                ptx::tma_load_2d(sb + L::kSQ + cb * 8192u, &tmQ, bar_st_full(st), h * D + cb * 64, slot0);
+                ptx::tma_load_2d(sb + L::kSDO + cb * 8192u, &tmDO, bar_st_full(st), h * D + cb * 64, slot0);
+              }
+              bulk_load(sb + L::kSL, a.ls + int64_t(h) * a.n_slots + slot0, kHalf * 4u, bar_st_full(st));
+              bulk_load(sb + L::kSD, a.ds + int64_t(h) * a.n_slots + slot0, kHalf * 4u, bar_st_full(st));
+              bulk_load(sb + L::kSM, a.meta + slot0, kHalf * 16u, bar_st_full(st));
+              pend_mask |= 1u << st;
+              pend_par = (pend_par & ~(1u << st)) | (st_phase << st);
+              if (++st == kStages) { st = 0; st_phase ^= 1u; }
+            }
+          }
+        }
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        for (int i = 0; i < kStages; ++i)
+          if (pend_mask & (1u << i))
+            ptx::mbar_wait(bar_st_full(i), (pend_par >> i) & 1u, &never, a.err, lim / 8);
+        if (kv_fills) ptx::mbar_wait(bar_kv_full, (kv_fills - 1) & 1u, &never, a.err, lim / 8);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, kHalf, false, false);
+      constexpr uint32_t kIdG = ptx::idesc_bf16_f32(128, D, false, true);
+      uint32_t kv_phase = 0, st = 0, st_phase = 0, pd_phase = 0, acc_phase = 0, sd_cnt = 0;
+      bool ok = true;
+      const uint32_t sK = sbase + L::kK, sV = sbase + L::kV;
+      const uint32_t sPT = sbase + L::kPT, sDST = sbase + L::kDST;
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+        const KvItem it = a.items[a.order[item / a.Hkv]];
+        if (!ptx::mbar_wait(bar_kv_full, kv_phase, abort_flag, a.err, lim)) { ok = false; break; }
+        kv_phase ^= 1u;
+        ptx::tc_fence_after();
+        bool first_grad = true;
+        uint32_t prev_st = 0;
+        bool have_prev = false;
+        auto issue_grad = [&](uint32_t stg) -> bool {
+          if (!ptx::mbar_wait(bar_pd_full, pd_phase, abort_flag, a.err, lim)) return false;
+          pd_phase ^= 1u;
+          if (first_grad) {  // the previous item's epilogue has read dK / dV
+            if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim)) return false;
+            acc_phase ^= 1u;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sb = sbase + L::kStage0 + stg * L::kStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < kHalf / 16; ++kk) {
+            const uint32_t acc = (!first_grad || kk > 0) ? 1u : 0u;
+            ptx::umma_ss(tmem + kColDV, ptx::sdesc_sw128(sPT + kk * 32u, 16u, 1024u),
+                         ptx::sdesc_sw128(sb + L::kSDO + kk * 2048u, 8192u, 1024u), kIdG, acc);
+            ptx::umma_ss(tmem + kColDK, ptx::sdesc_sw128(sDST + kk * 32u, 16u, 1024u),
+                         ptx::sdesc_sw128(sb + L::kSQ + kk * 2048u, 8192u, 1024u), kIdG, acc);
+          }
+          first_grad = false;
+          ptx::umma_commit(bar_pd_free);
+          ptx::umma_commit(bar_st_empty(stg));
+          return true;
+        };
+        for (int ti = 0; ti < it.t_count && ok; ++ti) {
+          const TileDesc td = a.tiles[it.t_first + ti];
+          const int nh = (td.n_rows + kHalf - 1) / kHalf;
+          for (int hh = 0; hh < G && ok; ++hh) {
+            for (int half = 0; half < nh; ++half) {
+              if (!ptx::mbar_wait(bar_st_full(st), st_phase, abort_flag, a.err, lim)) { ok = false; break; }
+              const uint32_t b = sd_cnt & 1u;
+              const uint32_t bph = (sd_cnt >> 1) & 1u;
+              if (!ptx::mbar_wait(bar_sd_empty(b), bph ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+              ptx::tc_fence_after();
+              const uint32_t sb = sbase + L::kStage0 + st * L::kStageBytes;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t offA = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                const uint32_t offB = (kk >> 2) * 8192u + (kk & 3) * 32u;
+                ptx::umma_ss(tmem + kColS + b * kHalf, ptx::sdesc_sw128(sK + offA, 16u, 1024u),
+                             ptx::sdesc_sw128(sb + L::kSQ + offB, 16u, 1024u), kIdS, kk > 0 ? 1u : 0u);
+              }
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t offA = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                const uint32_t offB = (kk >> 2) * 8192u + (kk & 3) * 32u;
+                ptx::umma_ss(tmem + kColDP + b * kHalf, ptx::sdesc_sw128(sV + offA, 16u, 1024u),
+                             ptx::sdesc_sw128(sb + L::kSDO + offB, 16u, 1024u), kIdS, kk > 0 ? 1u : 0u);
+              }
+              ptx::umma_commit(bar_sd_full(b));
+              ++sd_cnt;
+              if (have_prev && !issue_grad(prev_st)) { ok = false; break; }
+              prev_st = st;
+              have_prev = true;
+              if (++st == kStages) { st = 0; st_phase ^= 1u; }
+            }
+          }
+        }
+        if (!ok) break;
+        if (have_prev && !issue_grad(prev_st)) { ok = false; break; }
+        if (first_grad) {  // no gradient MMA in this item: still pair the epilogue handshake
+          if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+          acc_phase ^= 1u;
+        }
+        ptx::umma_commit(bar_kv_empty);
+        ptx::umma_commit(bar_acc_full);
+      }
+      ptx::umma_commit(bar_drain);
+      volatile int never = 0;
+      ptx::mbar_wait(bar_drain, 0, &never, a.err, lim);
+    }
+  } else {
+    // ------------------------------------------------------------ P^T, dS^T / epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // key row within the tile
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t sPT = sbase + L::kPT, sDST = sbase + L::kDST;
+    const float sl2 = a.scale_log2;
+    uint32_t st = 0, sd_cnt = 0, pd_cnt = 0, acc_cnt = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      const KvItem it = a.items[a.order[item / a.Hkv]];
+      const int g = item % a.Hkv;
+      const int kp = it.key0 + row;  // this thread's key position
+      bool any = false;
+      for (int ti = 0; ti < it.t_count && ok; ++ti) {
+        const TileDesc td = a.tiles[it.t_first + ti];
+        const int nh = (td.n_rows + kHalf - 1) / kHalf;
+        for (int hh = 0; hh < G && ok; ++hh) {
+          for (int half = 0; half < nh; ++half) {
+            const uint32_t b = sd_cnt & 1u;
+            const uint32_t bph = (sd_cnt >> 1) & 1u;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_sd_full(b), bph, abort_flag, a.err, lim))) {
+              ok = false;
+              break;
+            }
+            ++sd_cnt;
+            ptx::tc_fence_after();
+            uint32_t sv[2][32], pv[2][32];
+            ptx::tmem_ld32(tl + kColS + b * kHalf, sv[0]);
+            ptx::tmem_ld32(tl + kColS + b * kHalf + 32u, sv[1]);
+            ptx::tmem_ld32(tl + kColDP + b * kHalf, pv[0]);
+            ptx::tmem_ld32(tl + kColDP + b * kHalf + 32u, pv[1]);
+            ptx::tmem_wait_ld();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar_sd_empty(b));
+            const uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
+            const float* Ls = reinterpret_cast<const float*>(sb + L::kSL);
+            const float* Ds = reinterpret_cast<const float*>(sb + L::kSD);
+            const SlotMeta* Ms = reinterpret_cast<const SlotMeta*>(sb + L::kSM);
+            // P^T and dS^T of this key row over the 64 query rows
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int col = c * 32 + i;
+                const bool vis = kp <= Ms[col].limit;
+                const float p = vis ? ptx::ex2(fmaf(__uint_as_float(sv[c][i]), sl2, -Ls[col])) : 0.f;
+                sv[c][i] = __float_as_uint(p);
+                pv[c][i] = __float_as_uint(p * (__uint_as_float(pv[c][i]) - Ds[col]));
+              }
+            if (pd_cnt > 0) {
+              // the previous sub-tile's gradient MMAs have read P^T / dS^T
+              if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_pd_free, (pd_cnt - 1) & 1u, abort_flag, a.err, lim))) {
+                ok = false;
+                break;
+              }
+            }
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              const int c = ch >> 2, i0 = (ch & 3) * 8;
+              const uint32_t off = row * 128u + (((ch ^ (row & 7))) << 4);
+              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPT + off),
+                           "r"(ptx::pack_bf16x2(__uint_as_float(sv[c][i0 + 0]), __uint_as_float(sv[c][i0 + 1]))),
+                           "r"(ptx::pack_bf16x2(__uint_as_float(sv[c][i0 + 2]), __uint_as_float(sv[c][i0 + 3]))),
+                           "r"(ptx::pack_bf16x2(__uint_as_float(sv[c][i0 + 4]), __uint_as_float(sv[c][i0 + 5]))),
+                           "r"(ptx::pack_bf16x2(__uint_as_float(sv[c][i0 + 6]), __uint_as_float(sv[c][i0 + 7])))
+                           : "memory");
+              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sDST + off),
+                           "r"(ptx::pack_bf16x2(__uint_as_float(pv[c][i0 + 0]), __uint_as_float(pv[c][i0 + 1]))),
+                           "r"(ptx::pack_bf16x2(__uint_as_float(pv[c][i0 + 2]), __uint_as_float(pv[c][i0 + 3]))),
+                           "r"(ptx::pack_bf16x2(__uint_as_float(pv[c][i0 + 4]), __uint_as_float(pv[c][i0 + 5]))),
+                           "r"(ptx::pack_bf16x2(__uint_as_float(pv[c][i0 + 6]), __uint_as_float(pv[c][i0 + 7])))
+                           : "memory");
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar_pd_full);
+            ++pd_cnt;
+            any = true;
+            if (++st == kStages) st = 0;
+          }
+        }
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_acc_full, acc_cnt & 1u, abort_flag, a.err, lim))) {
+        ok = false;
+        break;
+      }
+      ++acc_cnt;
+      ptx::tc_fence_after();
+      const bool own = kp < it.key_end && any;
+      const bool zero = kp < it.key_end && !any;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* out = which == 0 ? a.dk : a.dv;
+        const float mul = which == 0 ? a.scale : 1.f;
+        const uint32_t col0 = which == 0 ? kColDK : kColDV;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          ptx::tmem_ld32(tl + col0 + c * 32u, v);
+          ptx::tmem_wait_ld();
+          if (own || zero) {
+            __nv_bfloat16* dst = out + (int64_t(kp) * a.Hkv + g) * D + c * 32;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint4 wv;
+              const float z = zero ? 0.f : mul;
+              wv.x = ptx::pack_bf16x2(__uint_as_float(v[q4 * 8 + 0]) * z, __uint_as_float(v[q4 * 8 + 1]) * z);
+              wv.y = ptx::pack_bf16x2(__uint_as_float(v[q4 * 8 + 2]) * z, __uint_as_float(v[q4 * 8 + 3]) * z);
+              wv.z = ptx::pack_bf16x2(__uint_as_float(v[q4 * 8 + 4]) * z, __uint_as_float(v[q4 * 8 + 5]) * z);
+              wv.w = ptx::pack_bf16x2(__uint_as_float(v[q4 * 8 + 6]) * z, __uint_as_float(v[q4 * 8 + 7]) * z);
+              reinterpret_cast<uint4*>(dst)[q4] = wv;
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar_acc_free);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const DkdvMaps& m, const DkdvArgs& a, int num_sms, cudaStream_t st) {
+  using L = Smem<D>;
+  static_assert(L::kAlloc <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::kAlloc));
+  if (e != cudaSuccess) return e;
+  const int grid = a.n_items < num_sms ? a.n_items : num_sms;
+  if (grid <= 0) return cudaSuccess;
+  bwd_dkdv_kernel<D><<<grid, kThreads, L::kAlloc, st>>>(m.k, m.v, m.qg, m.dog, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_dkdv(const DkdvMaps& m, const DkdvArgs& a, int num_sms, cudaStream_t st) {
+  if (a.d == 128) return launch_d<128>(m, a, num_sms, st);
+  if (a.d == 64) return launch_d<64>(m, a, num_sms, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ba

@@ -179,6 +179,41 @@ void build_plan(const ba_problem* p, Plan* plan) {
                    [&](int a, int b) { return cost[a] > cost[b]; });
 }
 
+void build_kv_plan(const ba_problem* p, Plan* plan) {
+  plan->kv_items.clear();
+  plan->n_kv_pairs = 0;
+  const int32_t* cu = p->cu_seqlens_h;
+  const int nt = static_cast<int>(plan->tiles.size());
+  int t = 0;
+  for (int di = 0; di < p->ndoc; ++di) {
+    const int s = cu[di], e = cu[di + 1];
+    // row tiles of this document: contiguous, kv_end non-decreasing
+    const int t_lo = t;
+    while (t < nt && plan->tiles[t].doc_start == s) ++t;
+    const int t_hi = t;
+    for (int k0 = s; k0 < e; k0 += kKeysPerTile) {
+      int lo = t_lo, hi = t_hi;  // first tile with kv_end > k0
+      while (lo < hi) {
+        const int mid = (lo + hi) / 2;
+        if (plan->tiles[mid].kv_end > k0) hi = mid; else lo = mid + 1;
+      }
+      KvItem it;
+      it.key0 = k0;
+      it.key_end = std::min(e, k0 + kKeysPerTile);
+      it.t_first = lo;
+      it.t_count = t_hi - lo;
+      plan->n_kv_pairs += it.t_count;
+      plan->kv_items.push_back(it);
+    }
+  }
+  const int nk = static_cast<int>(plan->kv_items.size());
+  plan->kv_order.resize(nk);
+  std::iota(plan->kv_order.begin(), plan->kv_order.end(), 0);
+  std::stable_sort(plan->kv_order.begin(), plan->kv_order.end(), [&](int a, int b) {
+    return plan->kv_items[a].t_count > plan->kv_items[b].t_count;
+  });
+}
+
 WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int which) {
   WorkspaceLayout w;
   const size_t nt = plan.tiles.size();
@@ -194,10 +229,25 @@ WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int whic
   off = align_up(off + size_t(w.n_slots) * sizeof(int32_t), 256);
   if (which == BA_WS_BWD) {
     const size_t rows = size_t(p->S) + size_t(p->Nb) * (p->Nb > 0 ? p->B : 0);
-    w.dsum_off = off;
+    const size_t slots = size_t(w.n_slots);
+    // key tiles: one per 128 keys of each document, at most S/128 + ndoc
+    const size_t nkv = size_t(p->S) / kKeysPerTile + p->ndoc;
+    w.kv_items_off = off;
+    off = align_up(off + nkv * sizeof(KvItem), 256);
+    w.kv_order_off = off;
+    off = align_up(off + nkv * sizeof(int32_t), 256);
+    w.qg_off = off;
+    off = align_up(off + slots * p->Hq * p->d * 2, 1024);
+    w.dog_off = off;
+    off = align_up(off + slots * p->Hq * p->d * 2, 1024);
+    w.ls_off = off;
+    off = align_up(off + slots * p->Hq * sizeof(float), 256);
+    w.ds_off = off;
+    off = align_up(off + slots * p->Hq * sizeof(float), 256);
+    w.meta_off = off;
+    off = align_up(off + slots * sizeof(SlotMeta), 256);
+    w.drow_off = off;
     off = align_up(off + rows * p->Hq * sizeof(float), 256);
-    w.dq_off = off;
-    off = align_up(off + rows * p->Hq * p->d * sizeof(float), 256);
   }
   w.total = off;
   return w;

@@ -36,6 +36,9 @@ struct Plan {
   std::vector<TileDesc> tiles;     // in position order
   std::vector<int32_t> order;      // tile indices, longest (most key tiles) first
   std::vector<ChunkDev> chunks_dev;
+  std::vector<KvItem> kv_items;    // key tiles of the dK/dV pass
+  std::vector<int32_t> kv_order;   // kv item indices, most row tiles first
+  int64_t n_kv_pairs = 0;          // (key tile, row tile) pairs of the dK/dV pass
   int64_t n_tile_pairs = 0;        // main key tiles visited, per query head
   int64_t n_branch_tile_pairs = 0; // branch key tiles visited (fused forward), per head
   int64_t n_visible_pairs = 0;     // exact visible (row, key) pairs per head
@@ -49,10 +52,18 @@ ba_status validate(const ba_problem* p, bool need_tensors);
 // Precondition: validate(p, ...) == BA_OK.
 void build_plan(const ba_problem* p, Plan* plan);
 
+// Builds the key-tile list of the dK/dV pass (after build_plan).
+void build_kv_plan(const ba_problem* p, Plan* plan);
+
 // Workspace layout shared by the forward and backward paths.
 struct WorkspaceLayout {
   size_t tiles_off = 0, order_off = 0, chunks_off = 0, rows_off = 0;
-  size_t dsum_off = 0, dq_off = 0;   // backward only
+  // backward only
+  size_t kv_items_off = 0, kv_order_off = 0;
+  size_t qg_off = 0, dog_off = 0;    // Q and dO gathered into slot order, bf16 [slots, Hq, d]
+  size_t ls_off = 0, ds_off = 0;     // log2-scaled LSE and D = rowsum(dO*O), fp32 [Hq, slots]
+  size_t meta_off = 0;               // SlotMeta [slots]
+  size_t drow_off = 0;               // D in row order, fp32 [Hq, rows]
   size_t total = 0;
   int64_t n_slots = 0;               // row-table entries (ntiles * 128)
 };

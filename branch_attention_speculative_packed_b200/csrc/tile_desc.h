@@ -28,4 +28,23 @@ struct ChunkDev {
 };
 static_assert(sizeof(ChunkDev) == 16, "ChunkDev must stay 16 bytes");
 
+// One main key tile of the key-stationary dK/dV pass: 128 keys of one
+// document and the row tiles (a contiguous range) whose rows can see them.
+struct KvItem {
+  int32_t key0;     // first key (packed main position), document start + 128 j
+  int32_t key_end;  // one past the last key this item owns: min(doc end, key0 + 128)
+  int32_t t_first;  // first row tile with a row whose limit >= key0
+  int32_t t_count;  // row tiles to visit: [t_first, t_first + t_count)
+};
+static_assert(sizeof(KvItem) == 16, "KvItem must stay 16 bytes");
+
+// Per row-table slot metadata written by the backward pre-pass.
+struct SlotMeta {
+  int32_t limit;  // last visible main key (-1 for padding)
+  int32_t blo;    // visible branch key rows [blo, bhi) (flattened b*B+u)
+  int32_t bhi;
+  int32_t row;    // concatenated row index (-1 for padding)
+};
+static_assert(sizeof(SlotMeta) == 16, "SlotMeta must stay 16 bytes");
+
 }  // namespace ba
