@@ -1,0 +1,416 @@
+"""Benchmark: branch-attention forward + backward on B200.
+
+One step = ba_fused_fwd + ba_bwd (fused main-sequence + branch-local
+attention with the in-kernel Eq. 2 merge, then dQ/dK/dV through both parts)
+over one synthetic packed batch shaped like the 64K-token EAGLE-3
+training-time-test workload: S = 65536 packed tokens in 16 log-normal
+documents (mean 4096), a depth-3 chain branch at every main position, GQA
+32/8, d = 128, bf16, R = 8 virtual zigzag ranks.
+
+Metric: useful TFLOPS = 14 * d * P * Hq / step time, P = exact visible
+(row, key) pairs per query head (forward 4 d P Hq, backward 2.5x that).
+Inputs (several GB) are far larger than L2, so no flush between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1: launched under torchrun, one process per GPU, each rank runs its own
+independent batch (different seed), no collective on the data path; the
+reported value is the whole job's useful FLOPs / max-over-ranks time
+("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "branch-attn fwd+bwd useful TFLOPS at 64K tokens; % of B200 BF16 dense peak"
+WORKLOAD_INDEX = 3  # the 64K-token EAGLE-3 configuration
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling)."""
+    return 7919 * rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="ba_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # samples under load: the upper half of the power draw
+        pmed = statistics.median(power)
+        load = [s for s, p in zip(sm, power) if p >= pmed] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx), "samples": len(sm),
+                "power_w_max": max(power), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the same workload
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(target_s: float = 15.0):
+    """Times the oracle (as it stands) on the host: full forward + backward of
+    whole documents of the 64K workload, one KV group (4 query heads), adding
+    documents until about ``target_s`` seconds of CPU work.  Returns the same
+    metric (useful TFLOPS) over that sample."""
+    import numpy as np
+    import oracle as orc
+    import workloads as wl
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    cfg = wl.CONFIGS[WORKLOAD_INDEX]
+    prob = wl.make_problem(WORKLOAD_INDEX, device="cpu")
+    cu = prob.cu_seqlens.numpy()
+    anc = prob.anchors.numpy()
+    G = cfg.Hq // cfg.Hkv
+    heads = list(range(G))
+    q = prob.q[:, :G]
+    k = prob.k[:, :1]
+    v = prob.v[:, :1]
+    qb = prob.qb[:, :, :G]
+    kb = prob.kb[:, :, :1]
+    vb = prob.vb[:, :, :1]
+    do = prob.do[:, :G]
+    dob = prob.dob[:, :, :G]
+    S = int(cu[-1])
+    lengths = np.diff(cu)
+    order = np.argsort(lengths)  # shortest documents first: bounded steps
+    t0 = time.perf_counter()
+    done_pairs = 0
+    docs = 0
+    for di in order:
+        s, e = int(cu[di]), int(cu[di + 1])
+        branch_rows = [S + b * cfg.B + t for b in range(len(anc)) if s <= anc[b] < e for t in range(cfg.B)]
+        rows = np.concatenate([np.arange(s, e), np.array(branch_rows, dtype=np.int64)])
+        orc.forward_rows(q, k, v, qb, kb, vb, cu, anc, cfg.B, cfg.mode, rows=rows)
+        orc.backward_rows(q, k, v, qb, kb, vb, do, dob, cu, anc, cfg.B, cfg.mode, rows=rows)
+        L = e - s
+        nb = int(((anc >= s) & (anc < e)).sum())
+        pre = int(((anc[(anc >= s) & (anc < e)]) - s + 1).sum()) * cfg.B
+        done_pairs += L * (L + 1) // 2 + pre + nb * cfg.B * (cfg.B + 1) // 2
+        docs += 1
+        if time.perf_counter() - t0 >= target_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = 14.0 * cfg.d * done_pairs * len(heads)
+    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 oracle fwd+bwd of {docs} whole document(s) of the 64K workload "
+                      f"(shortest first), 1 KV group = {len(heads)} query heads, "
+                      f"{done_pairs} visible pairs/head, {dt:.1f} s",
+            "seconds": dt}
+
+
+# ---------------------------------------------------------------------------
+# GPU benchmark
+# ---------------------------------------------------------------------------
+
+def kernel_flops(kind: str, d: int, pairs: int, Hq: int) -> float:
+    """Algorithmic FLOPs of one launch of a tensor-core kernel over the
+    visible pairs: forward 2 GEMMs (QK^T, PV), dQ pass 3 (QK^T, dO V^T, dS K),
+    dK/dV pass 4 (K Q^T, V dO^T, P^T dO, dS^T Q); 2 d FLOPs per pair and GEMM."""
+    g = {"fused_fwd": 2, "bwd_dq": 3, "bwd_dkdv": 4}[kind]
+    return 2.0 * g * d * pairs * Hq
+
+
+def run_gpu(args):
+    import torch
+    import branch_attention_speculative_packed_b200 as ba
+    import workloads as wl
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = wl.CONFIGS[WORKLOAD_INDEX]
+    base = wl.make_problem(WORKLOAD_INDEX, device="cpu", with_grad_inputs=False) if False else None
+    # draw on the device (rank-dependent seed for weak scaling)
+    cu, anc = wl.make_layout(WORKLOAD_INDEX)
+    prob = wl._draw(cfg, wl.seed_of(WORKLOAD_INDEX) + rank_seed_offset(rank), cu, anc, dev, True)
+    a = ba.BranchAttention(cu, anc, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, B=cfg.B, mode=cfg.mode,
+                           R=cfg.R, device=dev)
+    stats = a.plan_stats()
+    P = stats["visible_pairs"]
+    useful = 14.0 * cfg.d * P * cfg.Hq
+    S, Nb = prob.S, prob.Nb
+    o = torch.empty_like(prob.q)
+    ob = torch.empty(Nb, cfg.B, cfg.Hq, cfg.d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(cfg.Hq, a.rows, dtype=torch.float32, device=dev)
+    grads = (torch.empty_like(prob.q), torch.empty_like(prob.k), torch.empty_like(prob.v),
+             torch.empty_like(prob.qb), torch.empty_like(prob.kb), torch.empty_like(prob.vb))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        a.fused_fwd(prob.q, prob.k, prob.v, prob.qb, prob.kb, prob.vb, out=(o, ob, lse))
+        a.bwd(prob.q, prob.k, prob.v, prob.qb, prob.kb, prob.vb, o, ob, lse, prob.do, prob.dob,
+              out=grads)
+
+    for _ in range(args.warmup):
+        step()
+    ba.sync_status()
+    # ------------------------------------------------------------ timed region
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ba.profile_enable(True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ba.profile_enable(False)
+    clocks = sampler.stop()
+    ms_local = ev0.elapsed_time(ev1)
+    prof = ba.profile_collect()
+    ba.sync_status()
+    ms_max = max_over_ranks(ms_local, world, dev)
+    ms_per_step = ms_max / args.steps
+    total_useful = sum_over_ranks(useful, world, dev)
+    value = total_useful * args.steps / (ms_max / 1e3) / 1e12
+
+    # ------------------------------------------------------------ roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    per_kernel = {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches": v[1], "share": None}
+                  for k, v in prof.items()}
+    tot = sum(v[0] for v in prof.values()) or 1.0
+    for k, v in prof.items():
+        per_kernel[k]["share"] = v[0] / tot
+    tensor_kernels = [k for k in ("fused_fwd", "bwd_dq", "bwd_dkdv") if k in prof]
+    dom = max(tensor_kernels, key=lambda k: prof[k][0])
+    dom_ms = per_kernel[dom]["ms_per_launch"]
+    achieved = kernel_flops(dom, cfg.d, P, cfg.Hq) / (dom_ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    launches = sum(v[1] for v in prof.values())
+
+    # ------------------------------------------------------------ end to end (host buffers)
+    host = {}
+    for name in ("q", "k", "v", "qb", "kb", "vb", "do", "dob"):
+        host[name] = getattr(prob, name).cpu().pin_memory()
+    outs_h = [t.new_empty(t.shape, device="cpu").pin_memory() for t in (o, ob, lse) + grads]
+    dev_in = {name: torch.empty_like(getattr(prob, name)) for name in host}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+
+    def e2e_step():
+        for name, t in host.items():
+            dev_in[name].copy_(t, non_blocking=True)
+        a.fused_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["qb"], dev_in["kb"], dev_in["vb"],
+                    out=(o, ob, lse))
+        a.bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["qb"], dev_in["kb"], dev_in["vb"], o, ob,
+              lse, dev_in["do"], dev_in["dob"], out=grads)
+        for dst, src in zip(outs_h, (o, ob, lse) + grads):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_steps = max(2, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    e2e_value = total_useful * e2e_steps / (e2e_ms / 1e3) / 1e12
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOPS",
+        "pct_of_peak": round(100.0 * value / (peak * world), 2),
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name + ": " + cfg.description, "S": cfg.S, "ndoc": cfg.ndoc,
+                   "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d, "branches": Nb, "B": cfg.B,
+                   "mask": "chain", "R": cfg.R, "visible_pairs_per_head": P,
+                   "useful_flop_per_step": useful, "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": None, "peak_source": f"{peak_src} bf16_tflops_sustained"},
+        "kernels": {k: {"ms": round(v["ms_per_launch"], 4), "launches": v["launches"],
+                        "share": round(v["share"], 4)} for k, v in per_kernel.items()},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        try:
+            result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        except Exception as e:  # keep the GPU line even if the host leg fails
+            result["cpu_baseline"] = {"error": repr(e)}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle on the host cores, same metric and
+    workload, each step a bounded sample (whole documents, one KV group)."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    vals = []
+    for _ in range(args.warmup):
+        cpu_baseline(min(args.cpu_seconds, 5.0))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(args.cpu_seconds))
+    dt = time.perf_counter() - t0
+    value = statistics.median(v["value"] for v in vals)
+    cfg_name = "eagle3_64k"
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg_name, "parallelism": "host cores (oracle)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": vals[0]["cores"],
+                         "kind": "oracle", "sample": vals[0]["sample"]},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "b200":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

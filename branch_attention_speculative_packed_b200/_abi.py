@@ -27,7 +27,8 @@ BA_WS_BWD = 1
 
 EXPORTED = (
     "ba_workspace_size", "ba_main_fwd", "ba_branch_fwd", "ba_lse_merge", "ba_fused_fwd",
-    "ba_bwd", "ba_status_string", "ba_sync_status", "ba_plan_stats",
+    "ba_bwd", "ba_status_string", "ba_sync_status", "ba_plan_stats", "ba_profile_enable",
+    "ba_profile_collect", "ba_last_error_word",
 )
 
 
@@ -47,7 +48,12 @@ class BaProblem(ctypes.Structure):
 class BAError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        extra = ""
+        if status == BA_ERR_TIMEOUT:
+            w = int(lib().ba_last_error_word())
+            extra = (f" [kernel {(w >> 24) & 0x7f}, role {(w >> 16) & 0xff}, "
+                     f"wait site {(w >> 8) & 0xff}, parity {w & 1}]")
+        super().__init__(f"{where}: {status_string(status)} (status {status}){extra}")
 
 
 _lib = None
@@ -76,6 +82,13 @@ def lib() -> ctypes.CDLL:
         L.ba_status_string.restype = ctypes.c_char_p
         L.ba_sync_status.argtypes = [vp]
         L.ba_plan_stats.argtypes = [P, i64p, i64p, i64p]
+        L.ba_last_error_word.argtypes = []
+        L.ba_last_error_word.restype = ctypes.c_uint32
+        L.ba_profile_enable.argtypes = [i32]
+        L.ba_profile_enable.restype = None
+        L.ba_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                                         ctypes.POINTER(ctypes.c_int), i32]
+        L.ba_profile_collect.restype = ctypes.c_int
         for name in ("ba_main_fwd", "ba_branch_fwd", "ba_fused_fwd", "ba_bwd", "ba_lse_merge",
                      "ba_sync_status", "ba_plan_stats"):
             getattr(L, name).restype = ctypes.c_int
@@ -90,3 +103,21 @@ def status_string(status: int) -> str:
 def check(status: int, where: str) -> None:
     if status != BA_OK:
         raise BAError(status, where)
+
+
+def profile_enable(on: bool) -> None:
+    """Bracket every kernel launch of the library with CUDA events (benchmarks)."""
+    lib().ba_profile_enable(1 if on else 0)
+
+
+def profile_collect() -> dict:
+    """{kernel name: (total ms, launches)} of the launches recorded since the
+    last collect (waits for their events)."""
+    cap = 32
+    names = (ctypes.c_char_p * cap)()
+    ms = (ctypes.c_double * cap)()
+    n = (ctypes.c_int * cap)()
+    k = lib().ba_profile_collect(names, ms, n, cap)
+    if k < 0:
+        raise RuntimeError("ba_profile_collect: event query failed")
+    return {names[i].decode(): (ms[i], n[i]) for i in range(min(k, cap))}

@@ -4,7 +4,10 @@
 
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "../../include/ba.h"
 #include "bwd_kernels.h"
@@ -83,6 +86,37 @@ ba_status encode_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// ------------------------------------------------------------------ profiling
+struct ProfRecord {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof;
+
+// Brackets one kernel launch with events on `st` while profiling is enabled.
+struct ProfScope {
+  ProfRecord rec{nullptr, nullptr, nullptr};
+  cudaStream_t st;
+  ProfScope(const char* name, cudaStream_t s) : st(s) {
+    if (!g_prof_on) return;
+    if (cudaEventCreate(&rec.start) != cudaSuccess) return;
+    if (cudaEventCreate(&rec.stop) != cudaSuccess) {
+      cudaEventDestroy(rec.start);
+      return;
+    }
+    rec.name = name;
+    cudaEventRecord(rec.start, st);
+  }
+  ~ProfScope() {
+    if (!rec.name) return;
+    cudaEventRecord(rec.stop, st);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.push_back(rec);
+  }
+};
+
 float scale_of(const ba_problem* p) {
   return p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->d));
 }
@@ -103,6 +137,7 @@ ba_status stage_plan(const ba_problem* p, const Plan& plan, const WorkspaceLayou
       cudaMemsetAsync(ws + w.rows_off, 0xFF, size_t(w.n_slots) * sizeof(int32_t), st) !=
           cudaSuccess)
     return BA_ERR_CUDA;
+  ProfScope prof("plan_rows", st);
   if (launch_plan_rows(p->cu_seqlens_d, p->ndoc, p->anchors_d, p->S, p->Nb, plan.B, p->R,
                        reinterpret_cast<const ChunkDev*>(ws + w.chunks_off),
                        reinterpret_cast<int32_t*>(ws + w.rows_off), w.n_slots,
@@ -178,6 +213,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   a.lse_ld = rows;
   a.err = di.err;
   a.wait_limit = kWaitLimitCycles;
+  ProfScope prof(fused ? "fused_fwd" : "main_fwd", st);
   if (launch_fwd(maps, a, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
   return BA_OK;
 }
@@ -224,6 +260,7 @@ ba_status ba_branch_fwd(const ba_problem* p, float* o_part, float* lse_part, ba_
   if (!o_part || !lse_part || !aligned16(o_part) || !aligned16(lse_part)) return BA_ERR_INVALID_ARG;
   DeviceInfo di;
   if ((s = device_info(&di)) != BA_OK) return s;
+  ProfScope prof("branch_fwd", reinterpret_cast<cudaStream_t>(stream));
   if (launch_branch_fwd(static_cast<const __nv_bfloat16*>(p->qb),
                         static_cast<const __nv_bfloat16*>(p->kb),
                         static_cast<const __nv_bfloat16*>(p->vb), p->Nb, p->B, p->mode, p->Hq,
@@ -260,6 +297,7 @@ ba_status ba_lse_merge(int nparts, int rows, int H, int d, const float* const* o
   DeviceInfo di;
   ba_status s = device_info(&di);
   if (s != BA_OK) return s;
+  ProfScope prof("lse_merge", reinterpret_cast<cudaStream_t>(stream));
   if (launch_lse_merge(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return BA_ERR_CUDA;
   return BA_OK;
@@ -327,7 +365,10 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   pa.ds = reinterpret_cast<float*>(ws + w.ds_off);
   pa.drow = reinterpret_cast<float*>(ws + w.drow_off);
   pa.meta = reinterpret_cast<SlotMeta*>(ws + w.meta_off);
-  if (launch_bwd_prep(pa, p->d, st) != cudaSuccess) return BA_ERR_CUDA;
+  {
+    ProfScope prof("bwd_prep", st);
+    if (launch_bwd_prep(pa, p->d, st) != cudaSuccess) return BA_ERR_CUDA;
+  }
 
   // tensor maps
   const int64_t qcols = int64_t(p->Hq) * p->d, kcols = int64_t(p->Hkv) * p->d;
@@ -367,7 +408,10 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   qa.dqb = static_cast<__nv_bfloat16*>(nb ? dqb : dq);
   qa.err = di.err;
   qa.wait_limit = kWaitLimitCycles;
-  if (launch_bwd_dq(dm, qa, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
+  {
+    ProfScope prof("bwd_dq", st);
+    if (launch_bwd_dq(dm, qa, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
+  }
 
   // 3. dK, dV of the main keys
   DkdvArgs ka;
@@ -390,7 +434,10 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   ka.dv = static_cast<__nv_bfloat16*>(dv);
   ka.err = di.err;
   ka.wait_limit = kWaitLimitCycles;
-  if (launch_bwd_dkdv(km, ka, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
+  {
+    ProfScope prof("bwd_dkdv", st);
+    if (launch_bwd_dkdv(km, ka, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
+  }
 
   // 4. dK, dV of the branch keys
   if (nb) {
@@ -412,6 +459,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
     ba_.scale = scale;
     ba_.dkb = static_cast<__nv_bfloat16*>(dkb);
     ba_.dvb = static_cast<__nv_bfloat16*>(dvb);
+    ProfScope prof("branch_bwd", st);
     if (launch_branch_bwd(ba_, p->d, st) != cudaSuccess) return BA_ERR_CUDA;
   }
   return BA_OK;
@@ -429,12 +477,55 @@ const char* ba_status_string(ba_status s) {
   return "unknown status";
 }
 
+void ba_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+}
+
+int ba_profile_collect(const char** names, double* total_ms, int* launches, int cap) {
+  std::vector<ProfRecord> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    recs.swap(g_prof);
+  }
+  std::map<std::string, std::pair<double, int>> acc;
+  std::map<std::string, const char*> name_of;
+  bool ok = true;
+  for (const ProfRecord& r : recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess)
+      ok = false;
+    auto& e = acc[r.name];
+    e.first += ms;
+    e.second += 1;
+    name_of[r.name] = r.name;
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  int i = 0;
+  for (const auto& kv : acc) {
+    if (i < cap) {
+      if (names) names[i] = name_of[kv.first];
+      if (total_ms) total_ms[i] = kv.second.first;
+      if (launches) launches[i] = kv.second.second;
+    }
+    ++i;
+  }
+  return ok ? i : -1;
+}
+
+static uint32_t g_last_error_word = 0;
+
+uint32_t ba_last_error_word(void) { return g_last_error_word; }
+
 ba_status ba_sync_status(ba_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return BA_ERR_CUDA;
   uint32_t word = 0;
   if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return BA_ERR_CUDA;
   if (word != 0) {
+    g_last_error_word = word;
     const uint32_t zero = 0;
     cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
     return BA_ERR_TIMEOUT;

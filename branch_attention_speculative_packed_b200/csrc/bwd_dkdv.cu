@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
         const KvItem it = a.items[a.order[item / a.Hkv]];
         const int g = item % a.Hkv;
-        if (!ptx::mbar_wait(bar_kv_empty, kv_phase ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+        if (!ptx::mbar_wait(bar_kv_empty, kv_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 0, 1))) { ok = false; break; }
         kv_phase ^= 1u;
         ptx::mbar_expect_tx(bar_kv_full, 2u * L::kKVBytes);
         ++kv_fills;
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int hh = 0; hh < G && ok; ++hh) {
             const int h = g * G + hh;
             for (int half = 0; half < nh; ++half) {
-              if (!ptx::mbar_wait(bar_st_empty(st), st_phase ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+              if (!ptx::mbar_wait(bar_st_empty(st), st_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 0, 2))) { ok = false; break; }
               const uint32_t sb = sbase + L::kStage0 + st * L::kStageBytes;
               const int slot0 = td.row_base + half * kHalf;
               ptx::mbar_expect_tx(bar_st_full(st), L::kStageTx);
@@ -185,17 +185,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sPT = sbase + L::kPT, sDST = sbase + L::kDST;
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
         const KvItem it = a.items[a.order[item / a.Hkv]];
-        if (!ptx::mbar_wait(bar_kv_full, kv_phase, abort_flag, a.err, lim)) { ok = false; break; }
+        if (!ptx::mbar_wait(bar_kv_full, kv_phase, abort_flag, a.err, lim, ptx::wait_site(3, 1, 3))) { ok = false; break; }
         kv_phase ^= 1u;
         ptx::tc_fence_after();
         bool first_grad = true;
         uint32_t prev_st = 0;
         bool have_prev = false;
         auto issue_grad = [&](uint32_t stg) -> bool {
-          if (!ptx::mbar_wait(bar_pd_full, pd_phase, abort_flag, a.err, lim)) return false;
+          if (!ptx::mbar_wait(bar_pd_full, pd_phase, abort_flag, a.err, lim, ptx::wait_site(3, 1, 4))) return false;
           pd_phase ^= 1u;
           if (first_grad) {  // the previous item's epilogue has read dK / dV
-            if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim)) return false;
+            if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 5))) return false;
             acc_phase ^= 1u;
           }
           ptx::tc_fence_after();
@@ -218,10 +218,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nh = (td.n_rows + kHalf - 1) / kHalf;
           for (int hh = 0; hh < G && ok; ++hh) {
             for (int half = 0; half < nh; ++half) {
-              if (!ptx::mbar_wait(bar_st_full(st), st_phase, abort_flag, a.err, lim)) { ok = false; break; }
+              if (!ptx::mbar_wait(bar_st_full(st), st_phase, abort_flag, a.err, lim, ptx::wait_site(3, 1, 6))) { ok = false; break; }
               const uint32_t b = sd_cnt & 1u;
               const uint32_t bph = (sd_cnt >> 1) & 1u;
-              if (!ptx::mbar_wait(bar_sd_empty(b), bph ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+              if (!ptx::mbar_wait(bar_sd_empty(b), bph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 7))) { ok = false; break; }
               ptx::tc_fence_after();
               const uint32_t sb = sbase + L::kStage0 + st * L::kStageBytes;
 #pragma unroll
@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (have_prev && !issue_grad(prev_st)) { ok = false; break; }
         if (first_grad) {  // no gradient MMA in this item: still pair the epilogue handshake
-          if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+          if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 8))) { ok = false; break; }
           acc_phase ^= 1u;
         }
         ptx::umma_commit(bar_kv_empty);
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t sPT = sbase + L::kPT, sDST = sbase + L::kDST;
     const float sl2 = a.scale_log2;
-    uint32_t st = 0, sd_cnt = 0, pd_cnt = 0, acc_cnt = 0;
+    uint32_t st = 0, st_phase = 0, sd_cnt = 0, pd_cnt = 0, acc_cnt = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
       const KvItem it = a.items[a.order[item / a.Hkv]];
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int half = 0; half < nh; ++half) {
             const uint32_t b = sd_cnt & 1u;
             const uint32_t bph = (sd_cnt >> 1) & 1u;
-            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_sd_full(b), bph, abort_flag, a.err, lim))) {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_sd_full(b), bph, abort_flag, a.err, lim, ptx::wait_site(3, 2, 9)))) {
               ok = false;
               break;
             }
@@ -295,6 +295,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_wait_ld();
             ptx::tc_fence_before();
             ptx::mbar_arrive(bar_sd_empty(b));
+            // the stage's L, D and metadata landed (TMA completion, seen by this thread)
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_st_full(st), st_phase, abort_flag, a.err, lim, ptx::wait_site(3, 2, 12)))) {
+              ok = false;
+              break;
+            }
             const uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
             const float* Ls = reinterpret_cast<const float*>(sb + L::kSL);
             const float* Ds = reinterpret_cast<const float*>(sb + L::kSD);
@@ -312,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             if (pd_cnt > 0) {
               // the previous sub-tile's gradient MMAs have read P^T / dS^T
-              if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_pd_free, (pd_cnt - 1) & 1u, abort_flag, a.err, lim))) {
+              if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_pd_free, (pd_cnt - 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(3, 2, 10)))) {
                 ok = false;
                 break;
               }
@@ -339,13 +344,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_arrive(bar_pd_full);
             ++pd_cnt;
             any = true;
-            if (++st == kStages) st = 0;
+            if (++st == kStages) { st = 0; st_phase ^= 1u; }
           }
         }
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_acc_full, acc_cnt & 1u, abort_flag, a.err, lim))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_acc_full, acc_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(3, 2, 11)))) {
         ok = false;
         break;
       }

@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileDesc td = a.tiles[a.order[item / Hq]];
         const int h = item % Hq;
         const int g = h / a.G;
-        if (!ptx::mbar_wait(bar_q_empty, q_phase ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+        if (!ptx::mbar_wait(bar_q_empty, q_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 0, 1))) { ok = false; break; }
         q_phase ^= 1u;
         ptx::mbar_expect_tx(bar_q_full, 2u * L::kTileBytes);
         ++q_fills;
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
         for (int j = 0; j < nkv + nbr; ++j) {
-          if (!ptx::mbar_wait(bar_kv_empty(kv_stage), kv_phase ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+          if (!ptx::mbar_wait(bar_kv_empty(kv_stage), kv_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 0, 2))) { ok = false; break; }
           ptx::mbar_expect_tx(bar_kv_full(kv_stage), 2u * L::kTileBytes);
           const void* mk = &tmK;
           const void* mv = &tmV;
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       const uint32_t sQ = sbase + L::kQ, sDO = sbase + L::kDO, sDS = sbase + L::kDS;
       auto issue_dq = [&](int jj, uint32_t stage) -> bool {
-        if (!ptx::mbar_wait(bar_ds_full, ds_phase, abort_flag, a.err, lim)) return false;
+        if (!ptx::mbar_wait(bar_ds_full, ds_phase, abort_flag, a.err, lim, ptx::wait_site(2, 1, 3))) return false;
         ds_phase ^= 1u;
         ptx::tc_fence_after();
         const uint32_t sk = sbase + L::kK0 + stage * L::kStageBytes;
@@ -192,15 +192,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
         const int n = nkv + nbr;
-        if (!ptx::mbar_wait(bar_q_full, q_phase, abort_flag, a.err, lim)) { ok = false; break; }
+        if (!ptx::mbar_wait(bar_q_full, q_phase, abort_flag, a.err, lim, ptx::wait_site(2, 1, 4))) { ok = false; break; }
         q_phase ^= 1u;
         ptx::tc_fence_after();
         uint32_t prev_stage = 0;
         for (int j = 0; j < n; ++j) {
-          if (!ptx::mbar_wait(bar_kv_full(kv_stage), kv_phase, abort_flag, a.err, lim)) { ok = false; break; }
+          if (!ptx::mbar_wait(bar_kv_full(kv_stage), kv_phase, abort_flag, a.err, lim, ptx::wait_site(2, 1, 5))) { ok = false; break; }
           const uint32_t sb = s_cnt & 1u;
           const uint32_t sph = (s_cnt >> 1) & 1u;
-          if (!ptx::mbar_wait(bar_s_empty(sb), sph ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+          if (!ptx::mbar_wait(bar_s_empty(sb), sph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 1, 6))) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t sk = sbase + L::kK0 + kv_stage * L::kStageBytes;
           const uint32_t sv = sk + L::kTileBytes;
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ptx::umma_commit(bar_s_full(sb));
           ++s_cnt;
-          if (!ptx::mbar_wait(bar_dp_empty, dp_phase ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+          if (!ptx::mbar_wait(bar_dp_empty, dp_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 1, 7))) { ok = false; break; }
           dp_phase ^= 1u;
           ptx::tc_fence_after();
 #pragma unroll
@@ -256,8 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j) {
         const uint32_t sb = s_cnt & 1u;
         const uint32_t sph = (s_cnt >> 1) & 1u;
-        bool w = ptx::mbar_wait(bar_s_full(sb), sph, abort_flag, a.err, lim);
-        w = w && ptx::mbar_wait(bar_dp_full, dp_cnt & 1u, abort_flag, a.err, lim);
+        bool w = ptx::mbar_wait(bar_s_full(sb), sph, abort_flag, a.err, lim, ptx::wait_site(2, 2, 8));
+        w = w && ptx::mbar_wait(bar_dp_full, dp_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 9));
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         ++dp_cnt;
         ptx::tc_fence_after();
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         lo = max(lo, 0);
         hi = min(hi, 128);
         if (j > 0) {
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_ds_free, ds_cnt & 1u, abort_flag, a.err, lim))) {
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_ds_free, ds_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 10)))) {
             ok = false;
             break;
           }
@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_ds_free, ds_cnt & 1u, abort_flag, a.err, lim))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_ds_free, ds_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 11)))) {
         ok = false;
         break;
       }

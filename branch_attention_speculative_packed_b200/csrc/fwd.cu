@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int h = item % Hq;
       const int g = h / a.G;
       int waited = 1;
-      if (lane == 0) waited = ptx::mbar_wait(bar.q_empty, q_phase ^ 1u, abort_flag, a.err, lim);
+      if (lane == 0) waited = ptx::mbar_wait(bar.q_empty, q_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(1, 0, 1));
       waited = __shfl_sync(0xffffffffu, waited, 0);
       if (!waited) { ok = false; break; }
       q_phase ^= 1u;
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
         for (int j = 0; j < nkv + nbr; ++j) {
-          if (!ptx::mbar_wait(bar.kv_empty[kv_stage], kv_phase ^ 1u, abort_flag, a.err, lim)) {
+          if (!ptx::mbar_wait(bar.kv_empty[kv_stage], kv_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(1, 0, 2))) {
             ok = false;
             break;
           }
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sQ = sbase + L::kQ;
       const uint32_t sP = sbase + L::kP;
       auto issue_pv = [&](int jj, uint32_t stage) -> bool {
-        if (!ptx::mbar_wait(bar.p_full, p_phase, abort_flag, a.err, lim)) return false;
+        if (!ptx::mbar_wait(bar.p_full, p_phase, abort_flag, a.err, lim, ptx::wait_site(1, 1, 3))) return false;
         p_phase ^= 1u;
         ptx::tc_fence_after();
         const uint32_t sv = sbase + L::kK0 + stage * L::kStageBytes + L::kTileBytes;
@@ -234,15 +234,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
         const int n = nkv + nbr;
-        if (!ptx::mbar_wait(bar.q_full, q_phase, abort_flag, a.err, lim)) { ok = false; break; }
+        if (!ptx::mbar_wait(bar.q_full, q_phase, abort_flag, a.err, lim, ptx::wait_site(1, 1, 4))) { ok = false; break; }
         q_phase ^= 1u;
         ptx::tc_fence_after();
         uint32_t prev_stage = 0;
         for (int j = 0; j < n; ++j) {
-          if (!ptx::mbar_wait(bar.kv_full[kv_stage], kv_phase, abort_flag, a.err, lim)) { ok = false; break; }
+          if (!ptx::mbar_wait(bar.kv_full[kv_stage], kv_phase, abort_flag, a.err, lim, ptx::wait_site(1, 1, 5))) { ok = false; break; }
           const uint32_t sb = s_cnt & 1u;
           const uint32_t sph = (s_cnt >> 1) & 1u;
-          if (!ptx::mbar_wait(bar.s_empty[sb], sph ^ 1u, abort_flag, a.err, lim)) { ok = false; break; }
+          if (!ptx::mbar_wait(bar.s_empty[sb], sph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(1, 1, 6))) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t sk = sbase + L::kK0 + kv_stage * L::kStageBytes;
 #pragma unroll
@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j) {
         const uint32_t sb = s_cnt & 1u;
         const uint32_t sph = (s_cnt >> 1) & 1u;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.s_full[sb], sph, abort_flag, a.err, lim))) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.s_full[sb], sph, abort_flag, a.err, lim, ptx::wait_site(1, 2, 7)))) {
           ok = false;
           break;
         }
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = l * alpha + rs;
         if (j > 0) {
           // P buffer and O are free once the previous P.V finished.
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done, o_cnt & 1u, abort_flag, a.err, lim))) {
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done, o_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 8)))) {
             ok = false;
             break;
           }
@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done, o_cnt & 1u, abort_flag, a.err, lim))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done, o_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 9)))) {
         ok = false;
         break;
       }

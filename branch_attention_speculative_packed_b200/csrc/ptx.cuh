@@ -38,22 +38,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Device error word codes.
-enum : uint32_t { kErrTimeout = 1u };
+// Device error word: 0 = no error.  A bounded wait that expires stores
+// 0x80000000 | (kernel << 24) | (role << 16) | (wait site << 8) | (parity)
+// unless an earlier error is already recorded.
+enum : uint32_t { kErrTimeout = 0x80000000u };
+__host__ __device__ constexpr uint32_t wait_site(uint32_t kernel, uint32_t role, uint32_t site) {
+  return kErrTimeout | (kernel << 24) | (role << 16) | (site << 8);
+}
 
 // Bounded wait on an mbarrier phase.  Gives up after ~`limit_cycles` SM
 // cycles or when another role of the CTA has raised `abort`; on expiry it
-// records the timeout in the device error word, raises `abort` and returns
-// false.  Never traps.
+// records where it gave up in the device error word, raises `abort` and
+// returns false.  Never traps.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* err, long long limit_cycles) {
+                                          uint32_t* err, long long limit_cycles,
+                                          uint32_t site = kErrTimeout) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > limit_cycles) {
-      atomicOr(err, kErrTimeout);
+      atomicCAS(err, 0u, site | (parity & 1u));
       *abort = 1;
       return false;
     }

@@ -178,12 +178,33 @@ BA_API const char* ba_status_string(ba_status s);
  * if the synchronisation failed, else BA_OK. */
 BA_API ba_status ba_sync_status(ba_stream_t stream);
 
+/* The device error word that the last failing ba_sync_status() reported
+ * (0 if none): bit 31 set for an expired bounded wait, bits 24-30 the kernel
+ * (1 forward, 2 dQ pass, 3 dK/dV pass), bits 16-23 the role (0 TMA producer,
+ * 1 MMA issuer, 2 softmax / gradient threads), bits 8-15 the wait site in that
+ * role, bit 0 the phase parity waited for.  For diagnosing a timeout. */
+BA_API uint32_t ba_last_error_word(void);
+
 /* Planner statistics for a problem (host only, no GPU needed): number of row
  * tiles, (row tile, key tile) pairs the forward kernel visits per query head,
  * and the exact count of visible (row, key) pairs per query head.  Returns
  * BA_ERR_INVALID_ARG for an invalid problem. */
 BA_API ba_status ba_plan_stats(const ba_problem* p, int64_t* n_row_tiles, int64_t* n_tile_pairs,
                         int64_t* n_visible_pairs);
+
+/* Kernel timing for benchmarks (no counterpart on the pages).  While enabled,
+ * every kernel the library launches is bracketed by two CUDA events recorded
+ * on the launching stream; the library creates and destroys these events
+ * itself (host-side handles, no device memory).  Enabling and disabling are
+ * not thread-safe with respect to concurrent calls of the library. */
+BA_API void ba_profile_enable(int on);
+
+/* Waits for the recorded events, sums the elapsed time per kernel name, writes
+ * up to `cap` entries (name, total milliseconds, number of launches) and
+ * forgets the records.  Returns the number of distinct kernel names (may be
+ * larger than cap), or -1 if an event query failed.  Names are static strings
+ * owned by the library. */
+BA_API int ba_profile_collect(const char** names, double* total_ms, int* launches, int cap);
 
 #ifdef __cplusplus
 }
