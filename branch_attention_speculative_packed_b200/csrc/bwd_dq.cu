@@ -317,6 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          : "memory");
           }
         }
+        ++s_cnt;
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar_ds_full);
