@@ -36,6 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "branch-attn fwd+bwd useful TFLOPS at 64K tokens; % of B200 BF16 dense peak"
 WORKLOAD_INDEX = 3  # the 64K-token EAGLE-3 configuration
+REFERENCE_PREFIX = 640  # tokens per reference-arm step: about 3 s of oracle time
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -146,11 +147,13 @@ class ClockSampler:
 # CPU baseline: the fp64 oracle on a bounded sample of the same workload
 # ---------------------------------------------------------------------------
 
-def cpu_baseline(target_s: float = 15.0):
+def cpu_baseline(target_s: float = 15.0, prefix: int = 0):
     """Times the oracle (as it stands) on the host: full forward + backward of
     whole documents of the 64K workload, one KV group (4 query heads), adding
-    documents until about ``target_s`` seconds of CPU work.  Returns the same
-    metric (useful TFLOPS) over that sample."""
+    documents until about ``target_s`` seconds of CPU work (``prefix`` > 0:
+    only the first ``prefix`` tokens of the shortest document, a shorter
+    document of the same layout).  Returns the same metric (useful TFLOPS)
+    over that sample."""
     import numpy as np
     import oracle as orc
     import workloads as wl
@@ -160,50 +163,56 @@ def cpu_baseline(target_s: float = 15.0):
     except Exception:  # pragma: no cover
         threads = 1
     cfg = wl.CONFIGS[WORKLOAD_INDEX]
-    prob = wl.make_problem(WORKLOAD_INDEX, device="cpu")
-    cu = prob.cu_seqlens.numpy()
-    anc = prob.anchors.numpy()
+    cu_t, anc_t = wl.make_layout(WORKLOAD_INDEX)
+    cu = cu_t.numpy()
+    anc = anc_t.numpy()
     G = cfg.Hq // cfg.Hkv
     heads = list(range(G))
-    q = prob.q[:, :G]
-    k = prob.k[:, :1]
-    v = prob.v[:, :1]
-    qb = prob.qb[:, :, :G]
-    kb = prob.kb[:, :, :1]
-    vb = prob.vb[:, :, :1]
-    do = prob.do[:, :G]
-    dob = prob.dob[:, :, :G]
-    S = int(cu[-1])
     lengths = np.diff(cu)
     order = np.argsort(lengths)  # shortest documents first: bounded steps
-    t0 = time.perf_counter()
+    dt = 0.0
     done_pairs = 0
     docs = 0
     for di in order:
         s, e = int(cu[di]), int(cu[di + 1])
-        branch_rows = [S + b * cfg.B + t for b in range(len(anc)) if s <= anc[b] < e for t in range(cfg.B)]
-        rows = np.concatenate([np.arange(s, e), np.array(branch_rows, dtype=np.int64)])
-        orc.forward_rows(q, k, v, qb, kb, vb, cu, anc, cfg.B, cfg.mode, rows=rows)
-        orc.backward_rows(q, k, v, qb, kb, vb, do, dob, cu, anc, cfg.B, cfg.mode, rows=rows)
-        L = e - s
-        nb = int(((anc >= s) & (anc < e)).sum())
-        pre = int(((anc[(anc >= s) & (anc < e)]) - s + 1).sum()) * cfg.B
-        done_pairs += L * (L + 1) // 2 + pre + nb * cfg.B * (cfg.B + 1) // 2
+        if prefix > 0:
+            e = min(e, s + prefix)
+        a_doc = anc[(anc >= s) & (anc < e)] - s
+        # one document of the workload, one KV group (G query heads), same draws' law
+        sub = wl.make_custom([e - s], a_doc.tolist(), Hq=G, Hkv=1, d=cfg.d, B=cfg.B, mode=cfg.mode,
+                             seed=wl.seed_of(WORKLOAD_INDEX) + int(di))
+        scu = sub.cu_seqlens.numpy()
+        sanc = sub.anchors.numpy()
+        t0 = time.perf_counter()
+        orc.forward_rows(sub.q, sub.k, sub.v, sub.qb, sub.kb, sub.vb, scu, sanc, cfg.B, cfg.mode)
+        orc.backward_rows(sub.q, sub.k, sub.v, sub.qb, sub.kb, sub.vb, sub.do, sub.dob, scu, sanc,
+                          cfg.B, cfg.mode)
+        dt += time.perf_counter() - t0
+        done_pairs += orc.visible_pair_count(scu, sanc, cfg.B, cfg.mode)
         docs += 1
-        if time.perf_counter() - t0 >= target_s:
+        if dt >= target_s or prefix > 0:
             break
-    dt = time.perf_counter() - t0
     flops = 14.0 * cfg.d * done_pairs * len(heads)
     return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
-            "sample": f"fp64 oracle fwd+bwd of {docs} whole document(s) of the 64K workload "
-                      f"(shortest first), 1 KV group = {len(heads)} query heads, "
-                      f"{done_pairs} visible pairs/head, {dt:.1f} s",
+            "sample": f"fp64 oracle fwd+bwd (row-set form) of {docs} "
+                      f"{'document prefix of ' + str(prefix) + ' tokens' if prefix else 'whole document(s)'} "
+                      f"of the 64K workload's layout (shortest first), 1 KV group = {len(heads)} query "
+                      f"heads, {done_pairs} visible pairs/head, {dt:.1f} s of oracle time",
             "seconds": dt}
 
 
 # ---------------------------------------------------------------------------
 # GPU benchmark
 # ---------------------------------------------------------------------------
+
+def workload_config(world: int) -> dict:
+    import workloads as wl
+    cfg = wl.CONFIGS[WORKLOAD_INDEX]
+    return {"workload": cfg.name + ": " + cfg.description, "S": cfg.S, "ndoc": cfg.ndoc,
+            "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d, "branches": cfg.n_anchors, "B": cfg.B,
+            "mask": "chain", "R": cfg.R, "l2": "inputs larger than L2 (no flush)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
 
 def kernel_flops(kind: str, d: int, pairs: int, Hq: int) -> float:
     """Algorithmic FLOPs of one launch of a tensor-core kernel over the
@@ -227,7 +236,6 @@ def run_gpu(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     cfg = wl.CONFIGS[WORKLOAD_INDEX]
-    base = wl.make_problem(WORKLOAD_INDEX, device="cpu", with_grad_inputs=False) if False else None
     # draw on the device (rank-dependent seed for weak scaling)
     cu, anc = wl.make_layout(WORKLOAD_INDEX)
     prob = wl._draw(cfg, wl.seed_of(WORKLOAD_INDEX) + rank_seed_offset(rank), cu, anc, dev, True)
@@ -339,11 +347,8 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": cfg.name + ": " + cfg.description, "S": cfg.S, "ndoc": cfg.ndoc,
-                   "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d, "branches": Nb, "B": cfg.B,
-                   "mask": "chain", "R": cfg.R, "visible_pairs_per_head": P,
-                   "useful_flop_per_step": useful, "l2": "inputs larger than L2 (no flush)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": dict(workload_config(world), visible_pairs_per_head=P,
+                       useful_flop_per_step=useful),
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": None, "peak_source": f"{peak_src} bf16_tflops_sustained"},
@@ -375,19 +380,18 @@ def run_reference(args):
         return
     vals = []
     for _ in range(args.warmup):
-        cpu_baseline(min(args.cpu_seconds, 5.0))
+        cpu_baseline(prefix=REFERENCE_PREFIX)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        vals.append(cpu_baseline(args.cpu_seconds))
+        vals.append(cpu_baseline(prefix=REFERENCE_PREFIX))
     dt = time.perf_counter() - t0
     value = statistics.median(v["value"] for v in vals)
-    cfg_name = "eagle3_64k"
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg_name, "parallelism": "host cores (oracle)"},
+        "config": workload_config(world),
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": vals[0]["cores"],
                          "kind": "oracle", "sample": vals[0]["sample"]},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
