@@ -18,6 +18,7 @@ BA_ERR_UNSUPPORTED = -2
 BA_ERR_CUDA = -3
 BA_ERR_TIMEOUT = -4
 BA_ERR_WORKSPACE = -5
+BA_ERR_SCRATCH_LIMIT = -6
 
 BA_MASK_CHAIN = 0
 BA_MASK_BLOCK = 1
@@ -28,7 +29,7 @@ BA_WS_BWD = 1
 EXPORTED = (
     "ba_workspace_size", "ba_main_fwd", "ba_branch_fwd", "ba_lse_merge", "ba_fused_fwd",
     "ba_bwd", "ba_status_string", "ba_sync_status", "ba_plan_stats", "ba_profile_enable",
-    "ba_profile_collect", "ba_last_error_word",
+    "ba_profile_collect", "ba_last_error_word", "ba_fused_fwd_noalloc",
 )
 
 
@@ -75,6 +76,7 @@ def lib() -> ctypes.CDLL:
         L.ba_main_fwd.argtypes = [P, vp, vp, vp]
         L.ba_branch_fwd.argtypes = [P, vp, vp, vp]
         L.ba_fused_fwd.argtypes = [P, vp, vp, vp, vp]
+        L.ba_fused_fwd_noalloc.argtypes = [P, vp, vp, vp, vp]
         L.ba_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.ba_lse_merge.argtypes = [i32, i32, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                    i64p, vp, vp, ctypes.c_int64, vp]
@@ -89,7 +91,8 @@ def lib() -> ctypes.CDLL:
         L.ba_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
                                          ctypes.POINTER(ctypes.c_int), i32]
         L.ba_profile_collect.restype = ctypes.c_int
-        for name in ("ba_main_fwd", "ba_branch_fwd", "ba_fused_fwd", "ba_bwd", "ba_lse_merge",
+        for name in ("ba_main_fwd", "ba_branch_fwd", "ba_fused_fwd", "ba_fused_fwd_noalloc", "ba_bwd",
+                     "ba_lse_merge",
                      "ba_sync_status", "ba_plan_stats"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L

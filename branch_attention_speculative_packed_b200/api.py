@@ -109,6 +109,15 @@ class BranchAttention:
                                       _ptr(lse), _stream(stream)), "ba_fused_fwd")
         return o, ob, lse
 
+    def fused_fwd_noalloc(self, q, k, v, qb, kb, vb, out, stream=None):
+        """ba_fused_fwd for callers that cannot allocate: scratch comes from the
+        library's static device array (no workspace); outputs must be given."""
+        o, ob, lse = out
+        p = self._problem(q, k, v, qb, kb, vb)
+        check(_abi.lib().ba_fused_fwd_noalloc(ctypes.byref(p), _ptr(o), _ptr(ob) if self.Nb else None,
+                                              _ptr(lse), _stream(stream)), "ba_fused_fwd_noalloc")
+        return o, ob, lse
+
     def main_fwd(self, q, k, v, qb, kb, vb, stream=None):
         """Step a2: (o_part fp32 [rows,Hq,d], lse_part fp32 [Hq,rows])."""
         dev = q.device

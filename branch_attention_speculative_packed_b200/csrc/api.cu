@@ -473,6 +473,8 @@ const char* ba_status_string(ba_status s) {
     case BA_ERR_CUDA: return "CUDA runtime error";
     case BA_ERR_TIMEOUT: return "device-side bounded wait expired";
     case BA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case BA_ERR_SCRATCH_LIMIT:
+      return "problem needs more scratch than the library's static array holds (BA_STATIC_SCRATCH_BYTES)";
   }
   return "unknown status";
 }
@@ -534,3 +536,45 @@ ba_status ba_sync_status(ba_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Entry point that allocates nothing: ba_fused_fwd with its scratch in a
+// file-scope device array (see ba_fused_fwd_noalloc in include/ba.h).
+namespace ba {
+namespace {
+
+static __device__ __align__(256) uint8_t g_static_scratch[BA_STATIC_SCRATCH_BYTES];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64] = {nullptr};
+
+// Device address of g_static_scratch on the current device, looked up once
+// per device.  In host code the symbol itself is only a host-side stand-in.
+ba_status static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return BA_ERR_CUDA;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return BA_OK;
+}
+
+}  // namespace
+}  // namespace ba
+
+extern "C" ba_status ba_fused_fwd_noalloc(const ba_problem* p, void* o, void* ob, float* lse,
+                                           ba_stream_t stream) {
+  ba_status s = validate(p, true);
+  if (s != BA_OK) return s;
+  if (ba_workspace_size(p, BA_WS_FWD) > BA_STATIC_SCRATCH_BYTES) return BA_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  if ((s = static_scratch(&scratch)) != BA_OK) return s;
+  ba_problem q = *p;
+  q.workspace = scratch;
+  q.workspace_bytes = BA_STATIC_SCRATCH_BYTES;
+  return ba_fused_fwd(&q, o, ob, lse, stream);
+}

@@ -72,7 +72,8 @@ typedef enum {
   BA_ERR_UNSUPPORTED = -2, /* valid but not implemented (e.g. d = 96) */
   BA_ERR_CUDA = -3,        /* a CUDA runtime call failed */
   BA_ERR_TIMEOUT = -4,     /* a device-side bounded wait expired */
-  BA_ERR_WORKSPACE = -5    /* workspace missing or too small */
+  BA_ERR_WORKSPACE = -5,   /* workspace missing or too small */
+  BA_ERR_SCRATCH_LIMIT = -6 /* problem needs more than the static scratch array holds */
 } ba_status;
 
 typedef enum {
@@ -157,6 +158,34 @@ BA_API ba_status ba_lse_merge(int nparts, int rows, int H, int d,
  * Paper: §3.2; the cere-bro wiki page ("Obstacle one, context parallelism")
  * describes the merge as happening within the ring pass itself. */
 BA_API ba_status ba_fused_fwd(const ba_problem* p, void* o, void* ob, float* lse, ba_stream_t stream);
+
+/* ba_fused_fwd for callers that cannot allocate device memory.  The paper has
+ * no counterpart; this is a deployment convenience.  Some callers cannot call
+ * cudaMalloc or hand the library a freshly allocated workspace: a runtime
+ * whose allocator owns every byte of device memory and forbids side
+ * allocations, code running under a strict device-memory budget fixed at
+ * start-up, or a caller that must not trigger an allocation's implicit
+ * synchronisation in the middle of a stream.  This entry point computes
+ * exactly what ba_fused_fwd computes (same kernels, same plan, same outputs)
+ * but takes its scratch space (the plan: tile table, order, chunk table and
+ * row table) from a file-scope device array inside the library instead of
+ * p->workspace, which is ignored along with p->workspace_bytes.
+ *   - Capacity: BA_STATIC_SCRATCH_BYTES (8 MiB), enough for problems of up to
+ *     about 1.9 million rows (S + Nb*B).  Every GPU that loads the library
+ *     holds this array until the process exits.  A problem whose plan needs
+ *     more returns BA_ERR_SCRATCH_LIMIT before anything is enqueued.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on that device.
+ *   - All calls share the one array, and it keeps the last call's contents.
+ *     Each call rewrites every part of it that it reads (the row table is
+ *     reset to -1 on every call), so nothing relies on earlier contents.
+ *     Calls whose work overlaps on the GPU (different streams, or different
+ *     host threads, on the same device) race on the array: serialise them.
+ *   - Allocates no device memory and calls no allocating library routine. */
+#define BA_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+BA_API ba_status ba_fused_fwd_noalloc(const ba_problem* p, void* o, void* ob, float* lse,
+                                      ba_stream_t stream);
 
 /* Backward (steps a5-a8; not on the pages): gradients of sum(O * dO) through
  * both components, recomputed from the merged LSE.
