@@ -35,7 +35,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "branch-attn fwd+bwd useful TFLOPS at 64K tokens; % of B200 BF16 dense peak"
-WORKLOAD_INDEX = 3  # the 64K-token EAGLE-3 configuration
+WORKLOAD_INDEX = 3  # the 64K-token EAGLE-3 configuration (the headline)
 REFERENCE_PREFIX = 640  # tokens per reference-arm step: about 3 s of oracle time
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -205,12 +205,13 @@ def cpu_baseline(target_s: float = 15.0, prefix: int = 0):
 # GPU benchmark
 # ---------------------------------------------------------------------------
 
-def workload_config(world: int) -> dict:
+def workload_config(world: int, index: int = WORKLOAD_INDEX) -> dict:
     import workloads as wl
-    cfg = wl.CONFIGS[WORKLOAD_INDEX]
+    cfg = wl.CONFIGS[index]
     return {"workload": cfg.name + ": " + cfg.description, "S": cfg.S, "ndoc": cfg.ndoc,
             "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d, "branches": cfg.n_anchors, "B": cfg.B,
-            "mask": "chain", "R": cfg.R, "l2": "inputs larger than L2 (no flush)",
+            "mask": "chain" if cfg.mode == wl.CHAIN else "block", "R": cfg.R,
+            "l2": "inputs larger than L2 (no flush)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
@@ -235,10 +236,11 @@ def run_gpu(args):
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
-    cfg = wl.CONFIGS[WORKLOAD_INDEX]
+    widx = args.workload_index
+    cfg = wl.CONFIGS[widx]
     # draw on the device (rank-dependent seed for weak scaling)
-    cu, anc = wl.make_layout(WORKLOAD_INDEX)
-    prob = wl._draw(cfg, wl.seed_of(WORKLOAD_INDEX) + rank_seed_offset(rank), cu, anc, dev, True)
+    cu, anc = wl.make_layout(widx)
+    prob = wl._draw(cfg, wl.seed_of(widx) + rank_seed_offset(rank), cu, anc, dev, True)
     a = ba.BranchAttention(cu, anc, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, B=cfg.B, mode=cfg.mode,
                            R=cfg.R, device=dev)
     stats = a.plan_stats()
@@ -347,7 +349,7 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": dict(workload_config(world), visible_pairs_per_head=P,
+        "config": dict(workload_config(world, widx), visible_pairs_per_head=P,
                        useful_flop_per_step=useful),
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
@@ -359,7 +361,7 @@ def run_gpu(args):
         "gpu_launches": launches,
         "clocks": clocks,
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and widx == WORKLOAD_INDEX:
         try:
             result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
         except Exception as e:  # keep the GPU line even if the host leg fails
@@ -407,7 +409,17 @@ def main():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="eagle3_64k",
+                    help="configuration name (default: the 64K headline); others are parity-test "
+                         "sizes, useful for small profiling captures")
     args = ap.parse_args()
+    import workloads as wl
+    names = [c.name for c in wl.CONFIGS]
+    if args.workload not in names:
+        ap.error(f"--workload must be one of {names}")
+    args.workload_index = names.index(args.workload)
+    if args.impl == "reference" and args.workload_index != WORKLOAD_INDEX:
+        ap.error("the reference arm times the 64K headline workload only")
     if args.warmup < 3 and args.impl == "b200":
         args.warmup = 3
     if args.impl == "reference":
