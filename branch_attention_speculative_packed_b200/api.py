@@ -93,6 +93,14 @@ class BranchAttention:
                                        ctypes.byref(b), ctypes.byref(c)), "ba_plan_stats")
         return {"row_tiles": a.value, "tile_pairs": b.value, "visible_pairs": c.value}
 
+    def rank_work(self):
+        """(row tile, main key tile) pairs owned by each of the R virtual ranks."""
+        buf = (ctypes.c_int64 * self.R)()
+        n = _abi.lib().ba_plan_rank_work(ctypes.byref(self._problem()), buf, self.R)
+        if n < 0:
+            check(n, "ba_plan_rank_work")
+        return list(buf)
+
     # ------------------------------------------------------------------ forward
     def fused_fwd(self, q, k, v, qb, kb, vb, out=None, stream=None):
         """Steps a2+a3+a4: returns (o bf16 [S,Hq,d], ob bf16 [Nb,B,Hq,d], lse fp32 [Hq,rows])."""

@@ -138,7 +138,7 @@ ba_status stage_plan(const ba_problem* p, const Plan& plan, const WorkspaceLayou
           cudaSuccess)
     return BA_ERR_CUDA;
   ProfScope prof("plan_rows", st);
-  if (launch_plan_rows(p->cu_seqlens_d, p->ndoc, p->anchors_d, p->S, p->Nb, plan.B, p->R,
+  if (launch_plan_rows(p->cu_seqlens_d, p->ndoc, p->anchors_d, p->S, p->Nb, plan.B,
                        reinterpret_cast<const ChunkDev*>(ws + w.chunks_off),
                        reinterpret_cast<int32_t*>(ws + w.rows_off), w.n_slots,
                        st) != cudaSuccess)
@@ -245,6 +245,16 @@ ba_status ba_plan_stats(const ba_problem* p, int64_t* n_row_tiles, int64_t* n_ti
   return BA_OK;
 }
 
+int ba_plan_rank_work(const ba_problem* p, int64_t* pairs, int cap) {
+  ba_status s = validate(p, false);
+  if (s != BA_OK) return s;
+  Plan plan;
+  build_plan(p, &plan);
+  for (int r = 0; r < cap && r < p->R; ++r)
+    if (pairs) pairs[r] = plan.rank_pairs[r];
+  return p->R;
+}
+
 ba_status ba_main_fwd(const ba_problem* p, float* o_part, float* lse_part, ba_stream_t stream) {
   return run_fwd(p, false, o_part, nullptr, nullptr, lse_part, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -331,8 +341,9 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   if (nkv > 0 &&
       (cudaMemcpyAsync(ws + w.kv_items_off, plan.kv_items.data(), nkv * sizeof(KvItem),
                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
-       cudaMemcpyAsync(ws + w.kv_order_off, plan.kv_order.data(), nkv * sizeof(int32_t),
-                       cudaMemcpyHostToDevice, st) != cudaSuccess))
+       cudaMemcpyAsync(ws + w.kv_order_off, plan.kv_order.data(),
+                       plan.kv_order.size() * sizeof(int32_t), cudaMemcpyHostToDevice,
+                       st) != cudaSuccess))
     return BA_ERR_CUDA;
   const int64_t rows = int64_t(p->S) + int64_t(p->Nb) * plan.B;
   const float scale = scale_of(p);

@@ -130,8 +130,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pend_mask = 0, pend_par = 0, kv_fills = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-        const KvItem it = a.items[a.order[item / a.Hkv]];
-        const int g = item % a.Hkv;
+        const int code = a.order[item];
+        const KvItem it = a.items[code / a.Hkv];
+        const int g = code % a.Hkv;
         if (!ptx::mbar_wait(bar_kv_empty, kv_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 0, 1))) { ok = false; break; }
         kv_phase ^= 1u;
         ptx::mbar_expect_tx(bar_kv_full, 2u * L::kKVBytes);
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tma_load_2d(sbase + L::kV + cb * 16384u, &tmV, bar_kv_full, g * D + cb * 64, it.key0);
         }
         for (int ti = 0; ti < it.t_count && ok; ++ti) {
-          const TileDesc td = a.tiles[it.t_first + ti];
+          const TileDesc td = a.tiles[it.t_first + it.t_count - 1 - ti];
           const int nh = (td.n_rows + kHalf - 1) / kHalf;
           for (int hh = 0; hh < G && ok; ++hh) {
             const int h = g * G + hh;
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sK = sbase + L::kK, sV = sbase + L::kV;
       const uint32_t sPT = sbase + L::kPT, sDST = sbase + L::kDST;
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-        const KvItem it = a.items[a.order[item / a.Hkv]];
+        const KvItem it = a.items[a.order[item] / a.Hkv];
         if (!ptx::mbar_wait(bar_kv_full, kv_phase, abort_flag, a.err, lim, ptx::wait_site(3, 1, 3))) { ok = false; break; }
         kv_phase ^= 1u;
         ptx::tc_fence_after();
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         for (int ti = 0; ti < it.t_count && ok; ++ti) {
-          const TileDesc td = a.tiles[it.t_first + ti];
+          const TileDesc td = a.tiles[it.t_first + it.t_count - 1 - ti];
           const int nh = (td.n_rows + kHalf - 1) / kHalf;
           for (int hh = 0; hh < G && ok; ++hh) {
             for (int half = 0; half < nh; ++half) {
@@ -270,12 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t st = 0, st_phase = 0, sd_cnt = 0, pd_cnt = 0, acc_cnt = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-      const KvItem it = a.items[a.order[item / a.Hkv]];
-      const int g = item % a.Hkv;
+      const int code = a.order[item];
+      const KvItem it = a.items[code / a.Hkv];
+      const int g = code % a.Hkv;
       const int kp = it.key0 + row;  // this thread's key position
       bool any = false;
       for (int ti = 0; ti < it.t_count && ok; ++ti) {
-        const TileDesc td = a.tiles[it.t_first + ti];
+        const TileDesc td = a.tiles[it.t_first + it.t_count - 1 - ti];
         const int nh = (td.n_rows + kHalf - 1) / kHalf;
         for (int hh = 0; hh < G && ok; ++hh) {
           for (int half = 0; half < nh; ++half) {

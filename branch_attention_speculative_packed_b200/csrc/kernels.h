@@ -39,7 +39,7 @@ cudaError_t launch_fwd(const FwdMaps& maps, const FwdArgs& a, int num_sms, cudaS
 
 // ---------------------------------------------------------------- planning
 cudaError_t launch_plan_rows(const int32_t* cu_seqlens, int ndoc, const int32_t* anchors, int S,
-                             int Nb, int B, int R, const ChunkDev* chunks, int32_t* row_table,
+                             int Nb, int B, const ChunkDev* docs, int32_t* row_table,
                              int64_t n_slots, cudaStream_t stream);
 
 // ---------------------------------------------------------------- branch part / merge

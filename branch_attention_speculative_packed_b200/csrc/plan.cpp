@@ -69,6 +69,7 @@ void build_plan(const ba_problem* p, Plan* plan) {
   plan->tiles.clear();
   plan->chunks_dev.clear();
   plan->n_tile_pairs = plan->n_branch_tile_pairs = plan->n_visible_pairs = 0;
+  plan->rank_pairs.assign(R, 0);
 
   // Exact visible pairs per head (counting rule of the definition).
   int64_t vis = 0;
@@ -87,6 +88,8 @@ void build_plan(const ba_problem* p, Plan* plan) {
   for (int di = 0; di < p->ndoc; ++di) {
     const int s = cu[di], e = cu[di + 1];
     const int64_t L = e - s;
+    // Zigzag chunks of this document and their owning virtual ranks.
+    const size_t chunk0 = plan->chunks.size();
     for (int k = 0; k < 2 * R; ++k) {
       Chunk c;
       c.doc = di;
@@ -97,73 +100,84 @@ void build_plan(const ba_problem* p, Plan* plan) {
       c.b0 = Nb ? lower_bound_i(anc, 0, Nb, c.c0) : 0;
       c.b1 = Nb ? lower_bound_i(anc, c.b0, Nb, c.c1) : 0;
       c.n_rows = int64_t(c.c1 - c.c0) + int64_t(B) * (c.b1 - c.b0);
-      c.tile0 = tile_count;
-      c.ntiles = static_cast<int>((c.n_rows + kRowsPerTile - 1) / kRowsPerTile);
-      tile_count += c.ntiles;
+      c.tile0 = c.ntiles = 0;
       plan->chunks.push_back(c);
-      ChunkDev cd;
-      cd.c0 = c.c0;
-      cd.b0 = c.b0;
-      cd.slot_base = c.tile0 * kRowsPerTile;
-      cd.pad = 0;
-      plan->chunks_dev.push_back(cd);
-
-      // merged index of main position q within the chunk
-      auto main_index = [&](int q) -> int64_t {
-        const int lb = Nb ? lower_bound_i(anc, c.b0, c.b1, q) : 0;
-        return int64_t(q - c.c0) + int64_t(B) * (lb - c.b0);
-      };
-      // limit of the row at merged index m: largest q in [c0, c1) with main_index(q) <= m
-      auto limit_at = [&](int64_t m) -> int {
-        int lo = c.c0, hi = c.c1 - 1;
-        while (lo < hi) {
-          const int mid = lo + (hi - lo + 1) / 2;
-          if (main_index(mid) <= m) lo = mid; else hi = mid - 1;
-        }
-        return lo;
-      };
-      // first merged index of branch b's rows
-      auto branch_start = [&](int b) -> int64_t {
-        return int64_t(anc[b] - c.c0) + 1 + int64_t(B) * (b - c.b0);
-      };
-      for (int t = 0; t < c.ntiles; ++t) {
-        const int64_t m0 = int64_t(t) * kRowsPerTile;
-        const int64_t m1 = std::min<int64_t>(c.n_rows, m0 + kRowsPerTile);
-        TileDesc td;
-        td.row_base = (c.tile0 + t) * kRowsPerTile;
-        td.n_rows = static_cast<int32_t>(m1 - m0);
-        td.doc_start = s;
-        td.min_limit = limit_at(m0);
-        td.kv_end = limit_at(m1 - 1) + 1;
-        td.rank = c.rank;
-        td.br_lo = td.br_hi = 0;
-        if (c.b1 > c.b0) {
-          // branches whose rows [start, start + B) meet [m0, m1)
-          int lo = c.b0, hi = c.b1;  // first b with start(b) + B > m0
-          while (lo < hi) {
-            const int mid = (lo + hi) / 2;
-            if (branch_start(mid) + B > m0) hi = mid; else lo = mid + 1;
-          }
-          const int blo = lo;
-          lo = c.b0;
-          hi = c.b1;  // first b with start(b) >= m1
-          while (lo < hi) {
-            const int mid = (lo + hi) / 2;
-            if (branch_start(mid) >= m1) hi = mid; else lo = mid + 1;
-          }
-          const int bhi = lo;  // exclusive
-          if (bhi > blo) {
-            td.br_lo = blo * B;
-            td.br_hi = bhi * B;
-          }
-        }
-        const int64_t nkv = (int64_t(td.kv_end) - td.doc_start + kKeysPerTile - 1) / kKeysPerTile;
-        const int64_t nbr = (int64_t(td.br_hi) - td.br_lo + kKeysPerTile - 1) / kKeysPerTile;
-        plan->n_tile_pairs += nkv;
-        plan->n_branch_tile_pairs += std::max<int64_t>(0, nbr);
-        plan->tiles.push_back(td);
-      }
     }
+    // Row tiles over the document's rows in limit order (main row p, then the
+    // branch rows anchored at p).  A tile may cross a zigzag chunk edge; it is
+    // owned by the virtual rank whose chunk holds its first row.
+    const int b0 = Nb ? lower_bound_i(anc, 0, Nb, s) : 0;
+    const int b1 = Nb ? lower_bound_i(anc, b0, Nb, e) : 0;
+    const int64_t n_rows = L + int64_t(B) * (b1 - b0);
+    const int ntiles = static_cast<int>((n_rows + kRowsPerTile - 1) / kRowsPerTile);
+    ChunkDev cd;
+    cd.c0 = s;
+    cd.b0 = b0;
+    cd.slot_base = tile_count * kRowsPerTile;
+    cd.pad = 0;
+    plan->chunks_dev.push_back(cd);
+    // merged index of main position q within the document
+    auto main_index = [&](int q) -> int64_t {
+      const int lb = Nb ? lower_bound_i(anc, b0, b1, q) : 0;
+      return int64_t(q - s) + int64_t(B) * (lb - b0);
+    };
+    // limit of the row at merged index m: largest q in [s, e) with main_index(q) <= m
+    auto limit_at = [&](int64_t m) -> int {
+      int lo = s, hi = e - 1;
+      while (lo < hi) {
+        const int mid = lo + (hi - lo + 1) / 2;
+        if (main_index(mid) <= m) lo = mid; else hi = mid - 1;
+      }
+      return lo;
+    };
+    // first merged index of branch b's rows
+    auto branch_start = [&](int b) -> int64_t {
+      return int64_t(anc[b] - s) + 1 + int64_t(B) * (b - b0);
+    };
+    for (int t = 0; t < ntiles; ++t) {
+      const int64_t m0 = int64_t(t) * kRowsPerTile;
+      const int64_t m1 = std::min<int64_t>(n_rows, m0 + kRowsPerTile);
+      TileDesc td;
+      td.row_base = (tile_count + t) * kRowsPerTile;
+      td.n_rows = static_cast<int32_t>(m1 - m0);
+      td.doc_start = s;
+      td.min_limit = limit_at(m0);
+      td.kv_end = limit_at(m1 - 1) + 1;
+      td.rank = 0;
+      for (int k = 0; k < 2 * R; ++k) {
+        const Chunk& c = plan->chunks[chunk0 + k];
+        if (c.c0 <= td.min_limit && td.min_limit < c.c1) td.rank = c.rank;
+      }
+      td.br_lo = td.br_hi = 0;
+      if (b1 > b0) {
+        // branches whose rows [start, start + B) meet [m0, m1)
+        int lo = b0, hi = b1;  // first b with start(b) + B > m0
+        while (lo < hi) {
+          const int mid = (lo + hi) / 2;
+          if (branch_start(mid) + B > m0) hi = mid; else lo = mid + 1;
+        }
+        const int blo = lo;
+        lo = b0;
+        hi = b1;  // first b with start(b) >= m1
+        while (lo < hi) {
+          const int mid = (lo + hi) / 2;
+          if (branch_start(mid) >= m1) hi = mid; else lo = mid + 1;
+        }
+        const int bhi = lo;  // exclusive
+        if (bhi > blo) {
+          td.br_lo = blo * B;
+          td.br_hi = bhi * B;
+        }
+      }
+      const int64_t nkv = (int64_t(td.kv_end) - td.doc_start + kKeysPerTile - 1) / kKeysPerTile;
+      const int64_t nbr = (int64_t(td.br_hi) - td.br_lo + kKeysPerTile - 1) / kKeysPerTile;
+      plan->n_tile_pairs += nkv;
+      plan->n_branch_tile_pairs += std::max<int64_t>(0, nbr);
+      plan->rank_pairs.resize(R, 0);
+      plan->rank_pairs[td.rank] += nkv;
+      plan->tiles.push_back(td);
+    }
+    tile_count += ntiles;
   }
   // Longest-processing-time-first order over the key tiles each row tile visits.
   const int nt = static_cast<int>(plan->tiles.size());
@@ -206,12 +220,28 @@ void build_kv_plan(const ba_problem* p, Plan* plan) {
       plan->kv_items.push_back(it);
     }
   }
-  const int nk = static_cast<int>(plan->kv_items.size());
-  plan->kv_order.resize(nk);
-  std::iota(plan->kv_order.begin(), plan->kv_order.end(), 0);
-  std::stable_sort(plan->kv_order.begin(), plan->kv_order.end(), [&](int a, int b) {
-    return plan->kv_items[a].t_count > plan->kv_items[b].t_count;
+  // Work order: documents longest first, then KV head, then key tiles in
+  // order, so the CTAs running at the same time share one (document, KV head)
+  // and stream the same query tiles through L2.  Entry = item * Hkv + head.
+  plan->kv_order.clear();
+  std::vector<int> docs(p->ndoc);
+  std::iota(docs.begin(), docs.end(), 0);
+  std::stable_sort(docs.begin(), docs.end(), [&](int a, int b) {
+    return (cu[a + 1] - cu[a]) > (cu[b + 1] - cu[b]);
   });
+  std::vector<int> first_item(p->ndoc + 1, 0);
+  {
+    int k = 0;
+    for (int di = 0; di < p->ndoc; ++di) {
+      first_item[di] = k;
+      k += (cu[di + 1] - cu[di] + kKeysPerTile - 1) / kKeysPerTile;
+    }
+    first_item[p->ndoc] = k;
+  }
+  for (int di : docs)
+    for (int g = 0; g < p->Hkv; ++g)
+      for (int k = first_item[di]; k < first_item[di + 1]; ++k)
+        plan->kv_order.push_back(k * p->Hkv + g);
 }
 
 WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int which) {
@@ -235,7 +265,7 @@ WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int whic
     w.kv_items_off = off;
     off = align_up(off + nkv * sizeof(KvItem), 256);
     w.kv_order_off = off;
-    off = align_up(off + nkv * sizeof(int32_t), 256);
+    off = align_up(off + nkv * p->Hkv * sizeof(int32_t), 256);
     w.qg_off = off;
     off = align_up(off + slots * p->Hq * p->d * 2, 1024);
     w.dog_off = off;

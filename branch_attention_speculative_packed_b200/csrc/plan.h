@@ -27,7 +27,7 @@ struct Chunk {
   int c0, c1;   // main positions [c0, c1)
   int b0, b1;   // branches whose anchor lies in [c0, c1)
   int64_t n_rows;
-  int tile0, ntiles;  // tiles of this chunk: [tile0, tile0 + ntiles)
+  int tile0, ntiles;  // unused: row tiles are cut per document
 };
 
 struct Plan {
@@ -36,8 +36,9 @@ struct Plan {
   std::vector<TileDesc> tiles;     // in position order
   std::vector<int32_t> order;      // tile indices, longest (most key tiles) first
   std::vector<ChunkDev> chunks_dev;
+  std::vector<int64_t> rank_pairs; // main (row tile, key tile) pairs per virtual rank
   std::vector<KvItem> kv_items;    // key tiles of the dK/dV pass
-  std::vector<int32_t> kv_order;   // kv item indices, most row tiles first
+  std::vector<int32_t> kv_order;   // work order: kv item * Hkv + KV head
   int64_t n_kv_pairs = 0;          // (key tile, row tile) pairs of the dK/dV pass
   int64_t n_tile_pairs = 0;        // main key tiles visited, per query head
   int64_t n_branch_tile_pairs = 0; // branch key tiles visited (fused forward), per head

@@ -12,19 +12,17 @@ namespace {
 
 // ------------------------------------------------------------------ plan rows
 // Writes every concatenated row index r (main rows 0..S-1, then branch rows
-// S + b*B + t) into the slot of its row tile.  Within a zigzag chunk [c0, c1)
-// the rows are ordered by limit (main row p: p; branch row: its anchor), main
-// row first on ties, then branches in index order, depth-minor:
-//   main p:       m = (p - c0) + B * (#anchors in [c0, p))
-//   branch (b,t): m = (a_b - c0) + 1 + B * (b - b0) + t
-// The chunk of a position x in document [s, s+L) is the k with
-// floor(kL/2R) <= x - s < floor((k+1)L/2R).
+// S + b*B + t) into its slot of the row table.  Within a document starting at
+// s the rows are ordered by limit (main row p: p; branch row: its anchor),
+// main row first on ties, then branches in index order, depth-minor:
+//   main p:       m = (p - s) + B * (#anchors in [s, p))
+//   branch (b,t): m = (a_b - s) + 1 + B * (b - b0) + t
+// where b0 is the document's first branch.
 __global__ void plan_rows_kernel(const int32_t* __restrict__ cu, int ndoc,
-                                 const int32_t* __restrict__ anchors, int S, int Nb, int B, int R,
-                                 const ChunkDev* __restrict__ chunks, int32_t* __restrict__ rows,
+                                 const int32_t* __restrict__ anchors, int S, int Nb, int B,
+                                 const ChunkDev* __restrict__ docs, int32_t* __restrict__ rows,
                                  int64_t n_slots) {
   const int64_t total = int64_t(S) + int64_t(Nb) * B;
-  const int R2 = 2 * R;
   for (int64_t r = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; r < total;
        r += int64_t(gridDim.x) * blockDim.x) {
     int lim, b = 0, t = 0;
@@ -42,13 +40,7 @@ __global__ void plan_rows_kernel(const int32_t* __restrict__ cu, int ndoc,
       const int mid = (lo + hi + 1) >> 1;
       if (cu[mid] <= lim) lo = mid; else hi = mid - 1;
     }
-    const int s = cu[lo];
-    const int64_t L = cu[lo + 1] - s;
-    const int64_t x = lim - s;
-    int k = static_cast<int>((x * R2) / L);
-    while (k + 1 < R2 && (int64_t(k + 1) * L) / R2 <= x) ++k;
-    while (k > 0 && (int64_t(k) * L) / R2 > x) --k;
-    const ChunkDev c = chunks[int64_t(lo) * R2 + k];
+    const ChunkDev c = docs[lo];
     int64_t m;
     if (!br) {
       int a0 = 0, a1 = Nb;  // first anchor >= lim
@@ -207,11 +199,11 @@ int grid_for(int64_t work, int per_block, int cap) {
 }  // namespace
 
 cudaError_t launch_plan_rows(const int32_t* cu_seqlens, int ndoc, const int32_t* anchors, int S,
-                             int Nb, int B, int R, const ChunkDev* chunks, int32_t* row_table,
+                             int Nb, int B, const ChunkDev* docs, int32_t* row_table,
                              int64_t n_slots, cudaStream_t stream) {
   const int64_t total = int64_t(S) + int64_t(Nb) * B;
   plan_rows_kernel<<<grid_for(total, 256, 148 * 16), 256, 0, stream>>>(
-      cu_seqlens, ndoc, anchors, S, Nb, B, R, chunks, row_table, n_slots);
+      cu_seqlens, ndoc, anchors, S, Nb, B, docs, row_table, n_slots);
   return cudaGetLastError();
 }
 

@@ -4,9 +4,10 @@
 
 namespace ba {
 
-// One row tile: up to 128 query rows of one zigzag chunk, ordered by their
-// last visible main key ("limit"); ties put the main row first, then the
-// branch rows anchored there (branch-major, depth-minor).
+// One row tile: up to 128 query rows of one document, ordered by their last
+// visible main key ("limit"); ties put the main row first, then the branch
+// rows anchored there (branch-major, depth-minor).  The tile belongs to the
+// virtual rank whose zigzag chunk holds its first row.
 struct TileDesc {
   int32_t row_base;   // first slot in the row table (tile index * 128)
   int32_t n_rows;     // valid rows, 1..128 (slots beyond hold -1)
@@ -19,10 +20,10 @@ struct TileDesc {
 };
 static_assert(sizeof(TileDesc) == 32, "TileDesc must stay 32 bytes");
 
-// Per-chunk data the device row scatter needs.
+// Per-document data the device row scatter needs.
 struct ChunkDev {
-  int32_t c0;        // first main position of the chunk
-  int32_t b0;        // first branch anchored in the chunk
+  int32_t c0;        // first main position of the document
+  int32_t b0;        // first branch anchored in the document
   int32_t slot_base; // row-table slot of merged index 0
   int32_t pad;
 };

@@ -235,6 +235,14 @@ BA_API void ba_profile_enable(int on);
  * owned by the library. */
 BA_API int ba_profile_collect(const char** names, double* total_ms, int* launches, int cap);
 
+/* Work per virtual rank of the zigzag split (host only, no GPU needed):
+ * writes, for r < min(cap, R), the number of (row tile, main key tile) pairs
+ * of the row tiles owned by virtual rank r, and returns R (or a negative
+ * status for an invalid problem).  A row tile is owned by the rank whose
+ * zigzag chunk holds its first row.  With the zigzag split these totals are
+ * nearly equal (the pages: the split balances the triangular causal work). */
+BA_API int ba_plan_rank_work(const ba_problem* p, int64_t* pairs, int cap);
+
 #ifdef __cplusplus
 }
 #endif

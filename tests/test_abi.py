@@ -87,24 +87,30 @@ def test_duplicate_anchors_accepted(ba):
 # ---------------------------------------------------------------------------
 
 def _restated_plan(cu, anc, B, R):
-    """Row tiles per zigzag chunk: rows sorted by (limit, main-before-branch,
-    branch index, depth), cut into 128-row tiles; a tile visits the main key
-    tiles [doc start, max limit] in steps of 128."""
+    """Row tiles per document: the document's rows sorted by (limit,
+    main-before-branch, branch index, depth), cut into 128-row tiles; a tile
+    visits the main key tiles [doc start, max limit] in steps of 128 and is
+    owned by the zigzag rank of the chunk holding its first row."""
     cu = list(cu)
     anc = list(anc)
-    S = cu[-1]
     tiles = 0
     pairs = 0
-    for (di, k, c0, c1, rank) in orc.zigzag_chunks(np.array(cu), R):
-        s = cu[di]
-        rows = [(p, 0, 0, 0) for p in range(c0, c1)]
-        rows += [(a, 1, b, t) for b, a in enumerate(anc) if c0 <= a < c1 for t in range(B)]
+    rank_pairs = [0] * R
+    chunks = orc.zigzag_chunks(np.array(cu), R)
+    for di in range(len(cu) - 1):
+        s, e = cu[di], cu[di + 1]
+        rows = [(p, 0, 0, 0) for p in range(s, e)]
+        rows += [(a, 1, b, t) for b, a in enumerate(anc) if s <= a < e for t in range(B)]
         rows.sort()
         for i in range(0, len(rows), 128):
             tile = rows[i:i + 128]
             tiles += 1
-            pairs += -(-(tile[-1][0] - s + 1) // 128)
-    return tiles, pairs
+            n = -(-(tile[-1][0] - s + 1) // 128)
+            pairs += n
+            first = tile[0][0]
+            owner = [c[4] for c in chunks if c[0] == di and c[2] <= first < c[3]][0]
+            rank_pairs[owner] += n
+    return tiles, pairs, rank_pairs
 
 
 @pytest.mark.parametrize("case", [
@@ -118,9 +124,10 @@ def test_planner_matches_restatement(ba, case):
     cu, anc, B, R = case
     a = _attn(ba, cu, anc, B=B, R=R)
     st = a.plan_stats()
-    t, p = _restated_plan(cu, anc, B, R)
+    t, p, rp = _restated_plan(cu, anc, B, R)
     assert st["row_tiles"] == t
     assert st["tile_pairs"] == p
+    assert a.rank_work() == rp
     assert st["visible_pairs"] == orc.visible_pair_count(np.array(cu), np.array(anc), B, 0)
 
 
@@ -133,7 +140,21 @@ def test_planner_on_workload_layouts(ba, idx):
     st = a.plan_stats()
     assert st["visible_pairs"] == orc.visible_pair_count(cu.numpy(), anc.numpy(), cfg.B, cfg.mode)
     if idx <= 2:
-        t, p = _restated_plan(cu.tolist(), anc.tolist(), cfg.B, cfg.R)
+        t, p, rp = _restated_plan(cu.tolist(), anc.tolist(), cfg.B, cfg.R)
         assert (st["row_tiles"], st["tile_pairs"]) == (t, p)
+        assert a.rank_work() == rp
     # every visible pair lies in a visited tile pair
     assert st["tile_pairs"] * 128 * 128 >= st["visible_pairs"] - cfg.n_anchors * cfg.B * cfg.B
+
+
+@pytest.mark.parametrize("R", [2, 4, 8])
+def test_zigzag_split_balances_causal_work(ba, R):
+    """Rank r owns chunks r and 2R-1-r, so every rank gets the same share of
+    the triangular causal work (up to tile rounding): the load-balancing the
+    pages attribute to the zigzag split.  A contiguous split would give the
+    last rank about 2R-1 times the first rank's work."""
+    L = 65536
+    a = _attn(ba, [0, L, 2 * L], list(range(0, 2 * L, 3)), B=3, R=R)
+    w = a.rank_work()
+    assert len(w) == R and sum(w) == a.plan_stats()["tile_pairs"]
+    assert max(w) / min(w) < 1.05, w
