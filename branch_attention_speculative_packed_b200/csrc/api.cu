@@ -135,7 +135,8 @@ ba_status stage_plan(const ba_problem* p, const Plan& plan, const WorkspaceLayou
                       plan.chunks_dev.size() * sizeof(ChunkDev), cudaMemcpyHostToDevice,
                       st) != cudaSuccess ||
       cudaMemsetAsync(ws + w.rows_off, 0xFF, size_t(w.n_slots) * sizeof(int32_t), st) !=
-          cudaSuccess)
+          cudaSuccess ||
+      cudaMemsetAsync(ws + w.counters_off, 0, 4 * sizeof(uint32_t), st) != cudaSuccess)
     return BA_ERR_CUDA;
   ProfScope prof("plan_rows", st);
   if (launch_plan_rows(p->cu_seqlens_d, p->ndoc, p->anchors_d, p->S, p->Nb, plan.B,
@@ -212,6 +213,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   a.lse = lse;
   a.lse_ld = rows;
   a.err = di.err;
+  a.counter = reinterpret_cast<uint32_t*>(ws + w.counters_off);
   a.wait_limit = kWaitLimitCycles;
   ProfScope prof(fused ? "fused_fwd" : "main_fwd", st);
   if (launch_fwd(maps, a, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
@@ -418,6 +420,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   qa.dq = static_cast<__nv_bfloat16*>(dq);
   qa.dqb = static_cast<__nv_bfloat16*>(nb ? dqb : dq);
   qa.err = di.err;
+  qa.counter = reinterpret_cast<uint32_t*>(ws + w.counters_off) + 1;
   qa.wait_limit = kWaitLimitCycles;
   {
     ProfScope prof("bwd_dq", st);
@@ -444,6 +447,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   ka.dk = static_cast<__nv_bfloat16*>(dk);
   ka.dv = static_cast<__nv_bfloat16*>(dv);
   ka.err = di.err;
+  ka.counter = reinterpret_cast<uint32_t*>(ws + w.counters_off) + 2;
   ka.wait_limit = kWaitLimitCycles;
   {
     ProfScope prof("bwd_dkdv", st);

@@ -45,10 +45,10 @@ struct Smem {
   static constexpr uint32_t kDST = kPT + 128u * kHalf * 2u;
   static constexpr uint32_t kBar = kDST + 128u * kHalf * 2u;
   // kv_full, kv_empty, st_full[3], st_empty[3], sd_full[2], sd_empty[2], pd_full, pd_free,
-  // acc_full, acc_free, drain
-  static constexpr uint32_t kNumBars = 19;
-  static constexpr uint32_t kMisc = kBar + kNumBars * 8u;
-  static constexpr uint32_t kTotal = kMisc + 16u;
+  // acc_full, acc_free, drain, item_full[4], item_empty[4]
+  static constexpr uint32_t kNumBars = 25;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base, abort, item slots[4]
+  static constexpr uint32_t kTotal = kMisc + 32u;
   static constexpr uint32_t kAlloc = kTotal + 1024u;
   // offsets inside a stage
   static constexpr uint32_t kSQ = 0, kSDO = kHalfBytes, kSL = 2u * kHalfBytes;
@@ -86,6 +86,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_acc_full = b0 + 112, bar_acc_free = b0 + 120, bar_drain = b0 + 128;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  ptx::ItemRing ring;
+  ring.slot = reinterpret_cast<volatile int*>(smem + L::kMisc + 16);
+  ring.full = bar_drain + 8;
+  ring.empty = ring.full + 8 * ptx::kItemSlots;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_kv_full, 1);
@@ -103,6 +107,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bar_acc_full, 1);
     ptx::mbar_init(bar_acc_free, 128);
     ptx::mbar_init(bar_drain, 1);
+    for (uint32_t i = 0; i < ptx::kItemSlots; ++i) {
+      ptx::mbar_init(ring.full + 8 * i, 1);
+      ptx::mbar_init(ring.empty + 8 * i, 129);  // MMA issuer + 128 gradient threads
+    }
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -129,7 +137,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kv_phase = 0, st = 0, st_phase = 0;
       uint32_t pend_mask = 0, pend_par = 0, kv_fills = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      for (uint32_t rn = 0; ok; ++rn) {
+        const int item = static_cast<int>(atomicAdd(a.counter, 1u));
+        if (!ptx::ring_put(ring, rn, item, abort_flag, a.err, lim, ptx::wait_site(3, 0, 13))) { ok = false; break; }
+        if (item >= a.n_items) break;
         const int code = a.order[item];
         const KvItem it = a.items[code / a.Hkv];
         const int g = code % a.Hkv;
@@ -184,7 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       const uint32_t sK = sbase + L::kK, sV = sbase + L::kV;
       const uint32_t sPT = sbase + L::kPT, sDST = sbase + L::kDST;
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      for (uint32_t rn = 0; ok; ++rn) {
+        int item = 0;
+        if (!ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(3, 1, 14))) { ok = false; break; }
+        if (item >= a.n_items) break;
         const KvItem it = a.items[a.order[item] / a.Hkv];
         if (!ptx::mbar_wait(bar_kv_full, kv_phase, abort_flag, a.err, lim, ptx::wait_site(3, 1, 3))) { ok = false; break; }
         kv_phase ^= 1u;
@@ -270,7 +284,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = a.scale_log2;
     uint32_t st = 0, st_phase = 0, sd_cnt = 0, pd_cnt = 0, acc_cnt = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+    for (uint32_t rn = 0; ok; ++rn) {
+      int item = 0;
+      if (!__all_sync(0xffffffffu, ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(3, 2, 15)))) {
+        ok = false;
+        break;
+      }
+      if (item >= a.n_items) break;
       const int code = a.order[item];
       const KvItem it = a.items[code / a.Hkv];
       const int g = code % a.Hkv;

@@ -39,10 +39,10 @@ struct Smem {
   static constexpr uint32_t kDS = kK0 + kStages * kStageBytes;
   static constexpr uint32_t kBar = kDS + 128u * 128u * 2u;
   // q_full, q_empty, kv_full[2], kv_empty[2], s_full[2], s_empty[2], dp_full, dp_empty,
-  // ds_full, ds_free, drain
-  static constexpr uint32_t kNumBars = 15;
-  static constexpr uint32_t kMisc = kBar + kNumBars * 8u;
-  static constexpr uint32_t kTotal = kMisc + 16u;
+  // ds_full, ds_free, drain, item_full[4], item_empty[4]
+  static constexpr uint32_t kNumBars = 23;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base, abort, item slots[4]
+  static constexpr uint32_t kTotal = kMisc + 32u;
   static constexpr uint32_t kAlloc = kTotal + 1024u;
 };
 
@@ -72,6 +72,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_ds_full = b0 + 96, bar_ds_free = b0 + 104, bar_drain = b0 + 112;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  ptx::ItemRing ring;
+  ring.slot = reinterpret_cast<volatile int*>(smem + L::kMisc + 16);
+  ring.full = bar_drain + 8;
+  ring.empty = ring.full + 8 * ptx::kItemSlots;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_q_full, 1);
@@ -89,6 +93,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bar_ds_full, 128);
     ptx::mbar_init(bar_ds_free, 1);
     ptx::mbar_init(bar_drain, 1);
+    for (uint32_t i = 0; i < ptx::kItemSlots; ++i) {
+      ptx::mbar_init(ring.full + 8 * i, 1);
+      ptx::mbar_init(ring.empty + 8 * i, 129);  // MMA issuer + 128 gradient threads
+    }
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -117,7 +125,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kv_stage = 0, kv_phase = 0, q_phase = 0;
       uint32_t pend_mask = 0, pend_par = 0, q_fills = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      for (uint32_t rn = 0; ok; ++rn) {
+        const int item = static_cast<int>(atomicAdd(a.counter, 1u));
+        if (!ptx::ring_put(ring, rn, item, abort_flag, a.err, lim, ptx::wait_site(2, 0, 12))) { ok = false; break; }
+        if (item >= a.n_items) break;
         const TileDesc td = a.tiles[a.order[item / Hq]];
         const int h = item % Hq;
         const int g = h / a.G;
@@ -187,7 +198,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::umma_commit(bar_kv_empty(stage));
         return true;
       };
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      for (uint32_t rn = 0; ok; ++rn) {
+        int item = 0;
+        if (!ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(2, 1, 13))) { ok = false; break; }
+        if (item >= a.n_items) break;
         const TileDesc td = a.tiles[a.order[item / Hq]];
         const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
@@ -243,7 +257,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = a.scale_log2;
     uint32_t s_cnt = 0, dp_cnt = 0, ds_cnt = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+    for (uint32_t rn = 0; ok; ++rn) {
+      int item = 0;
+      if (!__all_sync(0xffffffffu, ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(2, 2, 14)))) {
+        ok = false;
+        break;
+      }
+      if (item >= a.n_items) break;
       const TileDesc td = a.tiles[a.order[item / Hq]];
       const int h = item % Hq;
       const int nkv = ceil_div(td.kv_end - td.doc_start, 128);

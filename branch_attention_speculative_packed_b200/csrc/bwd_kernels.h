@@ -52,6 +52,7 @@ struct DqArgs {
   __nv_bfloat16* dq;   // [S, Hq, d]
   __nv_bfloat16* dqb;  // [Nb*B, Hq, d]
   uint32_t* err;
+  uint32_t* counter;   // work-item counter, zero at launch
   long long wait_limit;
 };
 struct DqMaps {
@@ -75,6 +76,7 @@ struct DkdvArgs {
   float scale_log2, scale;
   __nv_bfloat16 *dk, *dv;  // [S, Hkv, d]
   uint32_t* err;
+  uint32_t* counter;       // work-item counter, zero at launch
   long long wait_limit;
 };
 struct DkdvMaps {

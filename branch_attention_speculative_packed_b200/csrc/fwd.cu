@@ -14,18 +14,20 @@
 // Roles (192 threads):
 //   warp 0      TMA producer: gathers the 128 query rows of the tile (one
 //               1-row box per row and 64 columns) and streams K/V key tiles
-//               through a 2-stage ring.
+//               through a 3-stage ring.
 //   warp 1      TMEM allocator and single-thread MMA issuer:
-//               S[sb] = Q K^T into one of two TMEM buffers, then O += P V.
+//               S[sb] = Q K^T into one of two TMEM buffers, then O += P V
+//               with P read from TMEM (A operand in tensor memory).
 //   warps 2-5   softmax / epilogue, one query row per thread: load S from
 //               TMEM, mask by the row's key range, update the running max
 //               (lazily: O in TMEM is rescaled only when the max grows by
-//               more than 2^8), write P (bf16) to shared memory for the next
-//               MMA, and finally normalise O and write O and LSE.
+//               more than 2^8), write P (bf16) into one of two TMEM buffers
+//               for the P.V MMA, and finally normalise O and write O and LSE.
 //
-// Shared memory (D = head dim): Q [128 x D] | 2 x (K [128 x D], V [128 x D])
-// | P [128 x 128], all bf16 in the 128-byte-swizzled layout TMA writes.
-// TMEM: S buffers at columns 0 and 128, O at column 256.
+// Shared memory (D = head dim): Q [128 x D] | 3 x (K [128 x D], V [128 x D]),
+// bf16 in the 128-byte-swizzled layout TMA writes.
+// TMEM: S buffers at columns 0 and 128, O at 256, P buffers at 384 and 448
+// (128 rows x 128 bf16 keys = 64 columns each).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -36,9 +38,9 @@ namespace ba {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256;
+constexpr uint32_t kColS0 = 0, kColO = 256, kColP = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
@@ -47,18 +49,18 @@ struct Smem {
   static constexpr uint32_t kTileBytes = 128u * D * 2u;  // one 128-row bf16 tile
   static constexpr uint32_t kK0 = kQ + kTileBytes;
   static constexpr uint32_t kStageBytes = 2u * kTileBytes;  // K + V
-  static constexpr uint32_t kP = kK0 + kStages * kStageBytes;
-  static constexpr uint32_t kBar = kP + 128u * 128u * 2u;
-  // barriers: q_full, q_empty, kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, o_done, drain
-  static constexpr uint32_t kNumBars = 13;
-  static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base (4 B), abort (4 B)
-  static constexpr uint32_t kTotal = kMisc + 16u;
+  static constexpr uint32_t kBar = kK0 + kStages * kStageBytes;
+  // barriers: q_full, q_empty, kv_full[3], kv_empty[3], s_full[2], s_empty[2], p_full[2],
+  // o_done[2], drain, item_full[4], item_empty[4]
+  static constexpr uint32_t kNumBars = 25;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base, abort, item slots[4]
+  static constexpr uint32_t kTotal = kMisc + 32u;
   static constexpr uint32_t kAlloc = kTotal + 1024u;  // slack to align the base to 1024
 };
 
 struct Bars {
-  uint32_t q_full, q_empty, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full,
-      o_done, drain;
+  uint32_t q_full, q_empty, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full[2],
+      o_done[2], drain;
 };
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -86,12 +88,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStages; ++i) { bar.kv_empty[i] = b; b += 8; }
     for (int i = 0; i < 2; ++i) { bar.s_full[i] = b; b += 8; }
     for (int i = 0; i < 2; ++i) { bar.s_empty[i] = b; b += 8; }
-    bar.p_full = b; b += 8;
-    bar.o_done = b; b += 8;
+    for (int i = 0; i < 2; ++i) { bar.p_full[i] = b; b += 8; }
+    for (int i = 0; i < 2; ++i) { bar.o_done[i] = b; b += 8; }
     bar.drain = b;
   }
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  ptx::ItemRing ring;
+  ring.slot = reinterpret_cast<volatile int*>(smem + L::kMisc + 16);
+  ring.full = bar.drain + 8;
+  ring.empty = ring.full + 8 * ptx::kItemSlots;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar.q_full, 1);
@@ -104,9 +110,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(bar.s_full[i], 1);
       ptx::mbar_init(bar.s_empty[i], 128);
     }
-    ptx::mbar_init(bar.p_full, 128);
-    ptx::mbar_init(bar.o_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar.p_full[i], 128);
+      ptx::mbar_init(bar.o_done[i], 1);
+    }
     ptx::mbar_init(bar.drain, 1);
+    for (uint32_t i = 0; i < ptx::kItemSlots; ++i) {
+      ptx::mbar_init(ring.full + 8 * i, 1);
+      ptx::mbar_init(ring.empty + 8 * i, 129);  // MMA issuer + 128 softmax threads
+    }
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -137,7 +149,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (for the abort drain); same for the query tile.
     uint32_t pend_mask = 0, pend_par = 0, q_fills = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+    for (uint32_t rn = 0; ok; ++rn) {
+      int item = 0, put = 1;
+      if (lane == 0) {
+        item = static_cast<int>(atomicAdd(a.counter, 1u));
+        put = ptx::ring_put(ring, rn, item, abort_flag, a.err, lim, ptx::wait_site(1, 0, 12));
+      }
+      item = __shfl_sync(0xffffffffu, item, 0);
+      if (!__shfl_sync(0xffffffffu, put, 0)) { ok = false; break; }
+      if (item >= a.n_items) break;
       const TileDesc td = a.tiles[a.order[item / Hq]];
       const int h = item % Hq;
       const int g = h / a.G;
@@ -210,26 +230,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdPV = ptx::idesc_bf16_f32(128, D, false, true);
-      uint32_t kv_stage = 0, kv_phase = 0, q_phase = 0, p_phase = 0, s_cnt = 0;
+      uint32_t kv_stage = 0, kv_phase = 0, q_phase = 0, s_cnt = 0, pv_cnt = 0;
       bool ok = true;
       const uint32_t sQ = sbase + L::kQ;
-      const uint32_t sP = sbase + L::kP;
+      // O += P V for key tile jj: P from TMEM buffer pv_cnt % 2, V from the stage.
       auto issue_pv = [&](int jj, uint32_t stage) -> bool {
-        if (!ptx::mbar_wait(bar.p_full, p_phase, abort_flag, a.err, lim, ptx::wait_site(1, 1, 3))) return false;
-        p_phase ^= 1u;
+        const uint32_t pb = pv_cnt & 1u;
+        if (!ptx::mbar_wait(bar.p_full[pb], (pv_cnt >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 1, 3))) return false;
         ptx::tc_fence_after();
         const uint32_t sv = sbase + L::kK0 + stage * L::kStageBytes + L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = ptx::sdesc_sw128(sP + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
           const uint64_t bd = ptx::sdesc_sw128(sv + kk * 2048u, 16384u, 1024u);
-          ptx::umma_ss(tmem + kColO, ad, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
+          ptx::umma_ts(tmem + kColO, tmem + kColP + pb * 64u + kk * 8u, bd, kIdPV,
+                       (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        ptx::umma_commit(bar.o_done);
+        ptx::umma_commit(bar.o_done[pb]);
         ptx::umma_commit(bar.kv_empty[stage]);
+        ++pv_cnt;
         return true;
       };
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      for (uint32_t rn = 0; ok; ++rn) {
+        int item = 0;
+        if (!ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(1, 1, 13))) { ok = false; break; }
+        if (item >= a.n_items) break;
         const TileDesc td = a.tiles[a.order[item / Hq]];
         const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
@@ -272,11 +296,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t sP = sbase + L::kP;
     const float sl2 = a.scale_log2;
-    uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t s_cnt = 0, pv_cnt = 0;  // S tiles consumed, P tiles produced
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+    for (uint32_t rn = 0; ok; ++rn) {
+      int item = 0;
+      if (!__all_sync(0xffffffffu, ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(1, 2, 14)))) {
+        ok = false;
+        break;
+      }
+      if (item >= a.n_items) break;
       const TileDesc td = a.tiles[a.order[item / Hq]];
       const int h = item % Hq;
       const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
@@ -361,51 +390,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             sr[c][i] = __float_as_uint(p);
           }
         l = l * alpha + rs;
-        if (j > 0) {
-          // P buffer and O are free once the previous P.V finished.
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done, o_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 8)))) {
-            ok = false;
-            break;
-          }
-          ++o_cnt;
-          ptx::tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
+        const uint32_t pb = pv_cnt & 1u;
+        // P buffer pb is free once the P.V that last read it (two tiles ago) finished.
+        bool w = true;
+        if (pv_cnt >= 2)
+          w = ptx::mbar_wait(bar.o_done[pb], ((pv_cnt >> 1) - 1u) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 9));
+        // Rescaling O needs the previous P.V (the other buffer) to have finished.
+        const bool any_rescale = __any_sync(0xffffffffu, rescale);
+        if (any_rescale && j > 0)
+          w = w && ptx::mbar_wait(bar.o_done[pb ^ 1u], ((pv_cnt - 1u) >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 10));
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        ptx::tc_fence_after();
+        if (any_rescale && j > 0) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              ptx::tmem_ld32(tl + kColO + c * 32u, ov);
-              ptx::tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            ptx::tmem_ld32(tl + kColO + c * 32u, ov);
+            ptx::tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-              ptx::tmem_st32(tl + kColO + c * 32u, ov);
-            }
-            ptx::tmem_wait_st();
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            ptx::tmem_st32(tl + kColO + c * 32u, ov);
           }
         }
-        // P (bf16) -> shared memory, 128-byte-swizzled K-major rows.
+        // P (bf16, two keys per 32-bit column) -> TMEM buffer pb
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          const int c = ch >> 2, i0 = (ch & 3) * 8;
-          const uint32_t w0 = ptx::pack_bf16x2(__uint_as_float(sr[c][i0 + 0]), __uint_as_float(sr[c][i0 + 1]));
-          const uint32_t w1 = ptx::pack_bf16x2(__uint_as_float(sr[c][i0 + 2]), __uint_as_float(sr[c][i0 + 3]));
-          const uint32_t w2 = ptx::pack_bf16x2(__uint_as_float(sr[c][i0 + 4]), __uint_as_float(sr[c][i0 + 5]));
-          const uint32_t w3 = ptx::pack_bf16x2(__uint_as_float(sr[c][i0 + 6]), __uint_as_float(sr[c][i0 + 7]));
-          const uint32_t addr = sP + (ch >> 3) * 16384u + row * 128u + ((((ch & 7) ^ (row & 7))) << 4);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
-                       "r"(w2), "r"(w3)
-                       : "memory");
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t pw[32];
+#pragma unroll
+          for (int wi = 0; wi < 32; ++wi) {
+            const int key = (h2 * 32 + wi) * 2;
+            pw[wi] = ptx::pack_bf16x2(__uint_as_float(sr[key >> 5][key & 31]),
+                                      __uint_as_float(sr[key >> 5][(key & 31) + 1]));
+          }
+          ptx::tmem_st32(tl + kColP + pb * 64u + h2 * 32u, pw);
         }
-        ptx::fence_proxy_async_smem();
+        ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(bar.p_full);
+        ptx::mbar_arrive(bar.p_full[pb]);
+        ++pv_cnt;
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done, o_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 9)))) {
-        ok = false;
-        break;
+      {  // the item's last P.V (and, in order, every earlier one) finished
+        const uint32_t last = pv_cnt - 1u;
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done[last & 1u], (last >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 11)))) {
+          ok = false;
+          break;
+        }
       }
-      ++o_cnt;
       ptx::tc_fence_after();
       const float inv_l = 1.f / l;
 #pragma unroll

@@ -28,6 +28,7 @@ struct FwdArgs {
   float* lse;                // element (h, r) at lse[h * lse_ld + r]
   int64_t lse_ld;
   uint32_t* err;             // device error word
+  uint32_t* counter;         // work-item counter, zero at launch
   long long wait_limit;      // cycles per bounded wait
 };
 

@@ -249,6 +249,8 @@ WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int whic
   const size_t nt = plan.tiles.size();
   w.n_slots = int64_t(nt) * kRowsPerTile;
   size_t off = 0;
+  w.counters_off = off;
+  off = align_up(off + 4 * sizeof(uint32_t), 256);
   w.tiles_off = off;
   off = align_up(off + nt * sizeof(TileDesc), 256);
   w.order_off = off;

@@ -58,6 +58,7 @@ void build_kv_plan(const ba_problem* p, Plan* plan);
 
 // Workspace layout shared by the forward and backward paths.
 struct WorkspaceLayout {
+  size_t counters_off = 0;  // uint32 work-item counters (forward, dQ pass, dK/dV pass)
   size_t tiles_off = 0, order_off = 0, chunks_off = 0, rows_off = 0;
   // backward only
   size_t kv_items_off = 0, kv_order_off = 0;

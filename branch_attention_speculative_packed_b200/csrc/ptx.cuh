@@ -66,6 +66,36 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// ---------------------------------------------------------------- work items
+// Dynamic scheduling inside a persistent CTA: the producer warp claims the
+// next work-item index from a global counter and publishes it in a small ring
+// of shared-memory slots; every consumer thread (the MMA issuer and the
+// softmax / gradient threads) reads it from there.  Each slot has a "full"
+// barrier (1 arrival: the producer) and an "empty" barrier (one arrival per
+// consumer thread).  An index >= the item count tells everyone to stop.
+constexpr uint32_t kItemSlots = 4;
+struct ItemRing {
+  volatile int* slot;  // int[kItemSlots] in shared memory
+  uint32_t full;       // kItemSlots mbarriers, 8 bytes apart
+  uint32_t empty;      // kItemSlots mbarriers, 8 bytes apart
+};
+__device__ __forceinline__ bool ring_put(const ItemRing& r, uint32_t n, int item, volatile int* abort,
+                                         uint32_t* err, long long lim, uint32_t site) {
+  const uint32_t s = n % kItemSlots;
+  if (!mbar_wait(r.empty + 8u * s, ((n / kItemSlots) & 1u) ^ 1u, abort, err, lim, site)) return false;
+  r.slot[s] = item;
+  mbar_arrive(r.full + 8u * s);
+  return true;
+}
+__device__ __forceinline__ bool ring_get(const ItemRing& r, uint32_t n, int* item, volatile int* abort,
+                                         uint32_t* err, long long lim, uint32_t site) {
+  const uint32_t s = n % kItemSlots;
+  if (!mbar_wait(r.full + 8u * s, (n / kItemSlots) & 1u, abort, err, lim, site)) return false;
+  *item = r.slot[s];
+  mbar_arrive(r.empty + 8u * s);
+  return true;
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -177,6 +207,17 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]; A (M x K, K-major) lives in TMEM: lane m holds
+// row m, two 16-bit K elements per 32-bit column (lower half = lower K index).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 // Arrive on `bar` once all previously issued tcgen05 ops of this thread complete.
