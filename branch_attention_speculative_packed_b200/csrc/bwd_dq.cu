@@ -305,15 +305,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++ds_cnt;
         }
+        // S in chunks of 32 columns; the load of chunk c+1 overlaps the math of chunk c.
+        uint32_t sbuf[2][32];
+        ptx::tmem_ld32(tl + kColS0 + sb * 128u, sbuf[0]);
+        ptx::tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t sr[32];
-          ptx::tmem_ld32(tl + kColS0 + sb * 128u + c * 32u, sr);
-          ptx::tmem_wait_ld();
-          if (c == 3) {
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(bar_s_empty(sb));
-          }
+          if (c < 3) ptx::tmem_ld32(tl + kColS0 + sb * 128u + (c + 1) * 32u, sbuf[(c + 1) & 1]);
+          const uint32_t* sr = sbuf[c & 1];
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
@@ -335,6 +334,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[q4 * 4 + 0]),
                          "r"(pk[q4 * 4 + 1]), "r"(pk[q4 * 4 + 2]), "r"(pk[q4 * 4 + 3])
                          : "memory");
+          }
+          ptx::tmem_wait_ld();
+          if (c == 2) {  // all four chunks of S are in registers now
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar_s_empty(sb));
           }
         }
         ++s_cnt;

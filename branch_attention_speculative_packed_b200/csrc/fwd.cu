@@ -352,12 +352,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         lo = max(lo, 0);
         hi = min(hi, 128);
-        float mx = -INFINITY;
+        // Row max with 8 independent accumulators (a single running max would
+        // be a 128-long dependency chain).
+        float mx8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
         if (lo == 0 && hi == 128) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[c][i]));
+            for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[c][i]));
         } else {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -366,9 +370,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int col = c * 32 + i;
               const bool vis = col >= lo && col < hi;
               if (!vis) sr[c][i] = __float_as_uint(-INFINITY);
-              mx = fmaxf(mx, __uint_as_float(sr[c][i]));
+              mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[c][i]));
             }
         }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float mxs = mx * sl2;
         float alpha = 1.f;
         bool rescale = false;
@@ -380,15 +386,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           rescale = true;
         }
         const float neg_m = -m_used;
-        float rs = 0.f;
+        float rs8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float p = ptx::ex2(fmaf(__uint_as_float(sr[c][i]), sl2, neg_m));
-            rs += p;
+            rs8[i & 7] += p;
             sr[c][i] = __float_as_uint(p);
           }
+        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         l = l * alpha + rs;
         const uint32_t pb = pv_cnt & 1u;
         // P buffer pb is free once the P.V that last read it (two tiles ago) finished.
