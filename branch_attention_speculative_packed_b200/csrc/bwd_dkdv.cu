@@ -326,25 +326,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float* Ls = reinterpret_cast<const float*>(sb + L::kSL);
             const float* Ds = reinterpret_cast<const float*>(sb + L::kSD);
             const SlotMeta* Ms = reinterpret_cast<const SlotMeta*>(sb + L::kSM);
-            // P^T and dS^T of this key row over the 64 query rows.  The row tile
-            // sees the whole key tile when its smallest limit reaches the last key.
-            const bool full = td.min_limit >= it.key0 + 127;
+            // P^T and dS^T of this key row over the 64 query rows
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
-              for (int i4 = 0; i4 < 32; i4 += 4) {
-                const int col = c * 32 + i4;
-                const float4 l4 = *reinterpret_cast<const float4*>(Ls + col);
-                const float4 d4 = *reinterpret_cast<const float4*>(Ds + col);
-                const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const bool vis = full || kp <= Ms[col + e].limit;
-                  const float p = vis ? ptx::ex2(fmaf(__uint_as_float(sv[c][i4 + e]), sl2, -lv[e])) : 0.f;
-                  sv[c][i4 + e] = __float_as_uint(p);
-                  pv[c][i4 + e] = __float_as_uint(p * (__uint_as_float(pv[c][i4 + e]) - dv4[e]));
-                }
+              for (int i = 0; i < 32; ++i) {
+                const int col = c * 32 + i;
+                const bool vis = kp <= Ms[col].limit;
+                const float p = vis ? ptx::ex2(fmaf(__uint_as_float(sv[c][i]), sl2, -Ls[col])) : 0.f;
+                sv[c][i] = __float_as_uint(p);
+                pv[c][i] = __float_as_uint(p * (__uint_as_float(pv[c][i]) - Ds[col]));
               }
             if (pd_cnt > 0) {
               // the previous sub-tile's gradient MMAs have read P^T / dS^T

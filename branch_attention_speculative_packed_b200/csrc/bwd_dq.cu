@@ -298,18 +298,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         lo = max(lo, 0);
         hi = min(hi, 128);
-        // dS of the 128 columns into packed registers, so the math overlaps the
-        // previous tile's dQ MMA (which still reads the shared dS buffer).
-        uint32_t pk[64];
+        if (j > 0) {
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_ds_free, ds_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 10)))) {
+            ok = false;
+            break;
+          }
+          ++ds_cnt;
+        }
+        // S in chunks of 32 columns; the load of chunk c+1 overlaps the math of chunk c.
+        uint32_t sbuf[2][32];
+        ptx::tmem_ld32(tl + kColS0 + sb * 128u, sbuf[0]);
+        ptx::tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t sr[32];
-          ptx::tmem_ld32(tl + kColS0 + sb * 128u + c * 32u, sr);
-          ptx::tmem_wait_ld();
-          if (c == 3) {  // all of S is in registers now
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(bar_s_empty(sb));
-          }
+          if (c < 3) ptx::tmem_ld32(tl + kColS0 + sb * 128u + (c + 1) * 32u, sbuf[(c + 1) & 1]);
+          const uint32_t* sr = sbuf[c & 1];
+          uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             float v2[2];
@@ -321,22 +325,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   : 0.f;
               v2[e] = p * (__uint_as_float(dp[c][i + e]) - dval);
             }
-            pk[c * 16 + (i >> 1)] = ptx::pack_bf16x2(v2[0], v2[1]);
+            pk[i >> 1] = ptx::pack_bf16x2(v2[0], v2[1]);
           }
-        }
-        if (j > 0) {  // the dS buffer is free once the previous tile's dQ MMA finished
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_ds_free, ds_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 10)))) {
-            ok = false;
-            break;
-          }
-          ++ds_cnt;
-        }
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          const uint32_t addr = sDS + (ch >> 3) * 16384u + row * 128u + (((ch & 7) ^ (row & 7)) << 4);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[ch * 4 + 0]),
-                       "r"(pk[ch * 4 + 1]), "r"(pk[ch * 4 + 2]), "r"(pk[ch * 4 + 3])
-                       : "memory");
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int ch = c * 4 + q4;
+            const uint32_t addr = sDS + (ch >> 3) * 16384u + row * 128u + (((ch & 7) ^ (row & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[q4 * 4 + 0]),
+                         "r"(pk[q4 * 4 + 1]), "r"(pk[q4 * 4 + 2]), "r"(pk[q4 * 4 + 3])
+                         : "memory");
+          }
+          ptx::tmem_wait_ld();
+          if (c == 2) {  // all four chunks of S are in registers now
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar_s_empty(sb));
+          }
         }
         ++s_cnt;
         ptx::fence_proxy_async_smem();
