@@ -1,20 +1,27 @@
 // dQ pass of the backward on sm_100a (query-stationary, tcgen05 + TMEM).
 //
-// One persistent CTA per SM walks (row tile, query head) items, longest first,
-// like the forward.  Per key tile j of the item (main keys, then the
+// One persistent CTA per SM takes (row tile, query head) items, longest first,
+// from a global counter.  Per key tile j of the item (main keys, then the
 // branch-local keys of the tile's branches):
-//   S  = Q K_j^T      -> TMEM (two buffers)
-//   dP = dO V_j^T     -> TMEM
+//   S_j  = Q K_j^T     -> TMEM buffer j % 2
+//   dP_j = dO V_j^T    -> TMEM
 //   threads: P = exp2(S * scale*log2e - L*log2e) under the row's key range,
-//            dS = P * (dP - D)  -> shared memory (bf16)
-//   dQ += dS K_j      -> TMEM accumulator
+//            dS = P * (dP - D), written as bf16 into the first 64 columns of
+//            S_j's own TMEM buffer
+//   dQ  += dS_j K_j    (A operand read from TMEM) -> TMEM accumulator
 // and finally dQ * scale is written as bf16 to the row's place in dq / dqb.
-// Q and dO come from the pre-pass's slot-ordered copies, so each is one TMA
-// box per 64 columns; L and D are the pre-pass's per-slot values.
+// Because dS_j lives in S_j's buffer, the two S buffers double-buffer dS too;
+// the in-order tensor pipe runs dQ_j (reading dS_j) before S_{j+2}, which
+// overwrites that buffer.
+//
+// Q and dO come from the pre-pass's slot-ordered copies (one TMA box per 64
+// columns); L and D are the pre-pass's per-slot values.  K and V travel in
+// separate rings: V_j is released as soon as dP_j has run, K_j only after
+// dQ_j, so K gets the deeper ring.
 //
 // Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-5
-// one query row per thread.  Shared memory (D = head dim): Q | dO |
-// 2 x (K, V) | dS.  TMEM: S at columns 0 / 128, dP at 256, dQ at 384.
+// one query row per thread.  Shared memory (D = head dim): Q | dO | 3 x K |
+// 2 x V.  TMEM: S/dS buffers at columns 0 and 128, dP at 256, dQ at 384.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -25,7 +32,7 @@ namespace ba {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
+constexpr uint32_t kKStages = 3, kVStages = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColDP = 256, kColDQ = 384;
 
@@ -35,12 +42,11 @@ struct Smem {
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kDO = kQ + kTileBytes;
   static constexpr uint32_t kK0 = kDO + kTileBytes;
-  static constexpr uint32_t kStageBytes = 2u * kTileBytes;
-  static constexpr uint32_t kDS = kK0 + kStages * kStageBytes;
-  static constexpr uint32_t kBar = kDS + 128u * 128u * 2u;
-  // q_full, q_empty, kv_full[2], kv_empty[2], s_full[2], s_empty[2], dp_full, dp_empty,
-  // ds_full, ds_free, drain, item_full[4], item_empty[4]
-  static constexpr uint32_t kNumBars = 23;
+  static constexpr uint32_t kV0 = kK0 + kKStages * kTileBytes;
+  static constexpr uint32_t kBar = kV0 + kVStages * kTileBytes;
+  // q_full, q_empty, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], dp_full,
+  // dp_empty, ds_full[2], dq_done, drain, item_full[4], item_empty[4]
+  static constexpr uint32_t kNumBars = 28;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base, abort, item slots[4]
   static constexpr uint32_t kTotal = kMisc + 32u;
   static constexpr uint32_t kAlloc = kTotal + 1024u;
@@ -64,12 +70,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t b0 = sbase + L::kBar;
   const uint32_t bar_q_full = b0, bar_q_empty = b0 + 8;
-  auto bar_kv_full = [&](uint32_t s) { return b0 + 16 + 8 * s; };
-  auto bar_kv_empty = [&](uint32_t s) { return b0 + 32 + 8 * s; };
-  auto bar_s_full = [&](uint32_t s) { return b0 + 48 + 8 * s; };
-  auto bar_s_empty = [&](uint32_t s) { return b0 + 64 + 8 * s; };
-  const uint32_t bar_dp_full = b0 + 80, bar_dp_empty = b0 + 88;
-  const uint32_t bar_ds_full = b0 + 96, bar_ds_free = b0 + 104, bar_drain = b0 + 112;
+  auto bar_k_full = [&](uint32_t s) { return b0 + 16 + 8 * s; };   // 3
+  auto bar_k_empty = [&](uint32_t s) { return b0 + 40 + 8 * s; };  // 3
+  auto bar_v_full = [&](uint32_t s) { return b0 + 64 + 8 * s; };   // 2
+  auto bar_v_empty = [&](uint32_t s) { return b0 + 80 + 8 * s; };  // 2
+  auto bar_s_full = [&](uint32_t s) { return b0 + 96 + 8 * s; };   // 2
+  const uint32_t bar_dp_full = b0 + 112, bar_dp_empty = b0 + 120;
+  auto bar_ds_full = [&](uint32_t s) { return b0 + 128 + 8 * s; };  // 2
+  const uint32_t bar_dq_done = b0 + 144, bar_drain = b0 + 152;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   ptx::ItemRing ring;
@@ -80,18 +88,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_q_full, 1);
     ptx::mbar_init(bar_q_empty, 1);
-    for (uint32_t i = 0; i < kStages; ++i) {
-      ptx::mbar_init(bar_kv_full(i), 1);
-      ptx::mbar_init(bar_kv_empty(i), 1);
+    for (uint32_t i = 0; i < kKStages; ++i) {
+      ptx::mbar_init(bar_k_full(i), 1);
+      ptx::mbar_init(bar_k_empty(i), 1);
+    }
+    for (uint32_t i = 0; i < kVStages; ++i) {
+      ptx::mbar_init(bar_v_full(i), 1);
+      ptx::mbar_init(bar_v_empty(i), 1);
     }
     for (uint32_t i = 0; i < 2; ++i) {
       ptx::mbar_init(bar_s_full(i), 1);
-      ptx::mbar_init(bar_s_empty(i), 128);
+      ptx::mbar_init(bar_ds_full(i), 128);
     }
     ptx::mbar_init(bar_dp_full, 1);
     ptx::mbar_init(bar_dp_empty, 128);
-    ptx::mbar_init(bar_ds_full, 128);
-    ptx::mbar_init(bar_ds_free, 1);
+    ptx::mbar_init(bar_dq_done, 1);
     ptx::mbar_init(bar_drain, 1);
     for (uint32_t i = 0; i < ptx::kItemSlots; ++i) {
       ptx::mbar_init(ring.full + 8 * i, 1);
@@ -122,8 +133,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t kv_stage = 0, kv_phase = 0, q_phase = 0;
-      uint32_t pend_mask = 0, pend_par = 0, q_fills = 0;
+      uint32_t ks = 0, kph = 0, vs = 0, vph = 0, q_phase = 0;
+      // parity of each stage's last fill and whether it may still be in flight (abort drain)
+      uint32_t kpend = 0, kpar = 0, vpend = 0, vpar = 0, q_fills = 0;
       bool ok = true;
       for (uint32_t rn = 0; ok; ++rn) {
         const int item = static_cast<int>(atomicAdd(a.counter, 1u));
@@ -144,8 +156,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
         for (int j = 0; j < nkv + nbr; ++j) {
-          if (!ptx::mbar_wait(bar_kv_empty(kv_stage), kv_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 0, 2))) { ok = false; break; }
-          ptx::mbar_expect_tx(bar_kv_full(kv_stage), 2u * L::kTileBytes);
           const void* mk = &tmK;
           const void* mv = &tmV;
           int y;
@@ -156,22 +166,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             mk = &tmKb;
             mv = &tmVb;
           }
-          const uint32_t sk = sbase + L::kK0 + kv_stage * L::kStageBytes;
+          if (!ptx::mbar_wait(bar_k_empty(ks), kph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 0, 2))) { ok = false; break; }
+          ptx::mbar_expect_tx(bar_k_full(ks), L::kTileBytes);
 #pragma unroll
-          for (int cb = 0; cb < D / 64; ++cb) {
-            ptx::tma_load_2d(sk + cb * 16384u, mk, bar_kv_full(kv_stage), g * D + cb * 64, y);
-            ptx::tma_load_2d(sk + L::kTileBytes + cb * 16384u, mv, bar_kv_full(kv_stage), g * D + cb * 64, y);
-          }
-          pend_mask |= 1u << kv_stage;
-          pend_par = (pend_par & ~(1u << kv_stage)) | (kv_phase << kv_stage);
-          if (++kv_stage == kStages) { kv_stage = 0; kv_phase ^= 1u; }
+          for (int cb = 0; cb < D / 64; ++cb)
+            ptx::tma_load_2d(sbase + L::kK0 + ks * L::kTileBytes + cb * 16384u, mk, bar_k_full(ks), g * D + cb * 64, y);
+          kpend |= 1u << ks;
+          kpar = (kpar & ~(1u << ks)) | (kph << ks);
+          if (++ks == kKStages) { ks = 0; kph ^= 1u; }
+          if (!ptx::mbar_wait(bar_v_empty(vs), vph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 0, 3))) { ok = false; break; }
+          ptx::mbar_expect_tx(bar_v_full(vs), L::kTileBytes);
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb)
+            ptx::tma_load_2d(sbase + L::kV0 + vs * L::kTileBytes + cb * 16384u, mv, bar_v_full(vs), g * D + cb * 64, y);
+          vpend |= 1u << vs;
+          vpar = (vpar & ~(1u << vs)) | (vph << vs);
+          if (++vs == kVStages) { vs = 0; vph ^= 1u; }
         }
       }
       if (*abort_flag) {
         volatile int never = 0;
-        for (int i = 0; i < kStages; ++i)
-          if (pend_mask & (1u << i))
-            ptx::mbar_wait(bar_kv_full(i), (pend_par >> i) & 1u, &never, a.err, lim / 8);
+        for (uint32_t i = 0; i < kKStages; ++i)
+          if (kpend & (1u << i)) ptx::mbar_wait(bar_k_full(i), (kpar >> i) & 1u, &never, a.err, lim / 8);
+        for (uint32_t i = 0; i < kVStages; ++i)
+          if (vpend & (1u << i)) ptx::mbar_wait(bar_v_full(i), (vpar >> i) & 1u, &never, a.err, lim / 8);
         if (q_fills) ptx::mbar_wait(bar_q_full, (q_fills - 1) & 1u, &never, a.err, lim / 8);
       }
     }
@@ -180,22 +198,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdDQ = ptx::idesc_bf16_f32(128, D, false, true);
-      uint32_t kv_stage = 0, kv_phase = 0, q_phase = 0, dp_phase = 0, ds_phase = 0, s_cnt = 0;
+      uint32_t ks = 0, kph = 0, vs = 0, vph = 0, q_phase = 0, dp_phase = 0;
+      uint32_t s_cnt = 0, ds_cnt = 0;  // S tiles issued, dQ MMAs issued
       bool ok = true;
-      const uint32_t sQ = sbase + L::kQ, sDO = sbase + L::kDO, sDS = sbase + L::kDS;
-      auto issue_dq = [&](int jj, uint32_t stage) -> bool {
-        if (!ptx::mbar_wait(bar_ds_full, ds_phase, abort_flag, a.err, lim, ptx::wait_site(2, 1, 3))) return false;
-        ds_phase ^= 1u;
+      const uint32_t sQ = sbase + L::kQ, sDO = sbase + L::kDO;
+      // dQ += dS K for the tile whose S went to buffer ds_cnt % 2 and whose K
+      // sits in K stage `kstage`.
+      auto issue_dq = [&](int jj, uint32_t kstage) -> bool {
+        const uint32_t b = ds_cnt & 1u;
+        if (!ptx::mbar_wait(bar_ds_full(b), (ds_cnt >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 1, 3))) return false;
         ptx::tc_fence_after();
-        const uint32_t sk = sbase + L::kK0 + stage * L::kStageBytes;
+        const uint32_t sk = sbase + L::kK0 + kstage * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = ptx::sdesc_sw128(sDS + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
           const uint64_t bd = ptx::sdesc_sw128(sk + kk * 2048u, 16384u, 1024u);
-          ptx::umma_ss(tmem + kColDQ, ad, bd, kIdDQ, (jj > 0 || kk > 0) ? 1u : 0u);
+          ptx::umma_ts(tmem + kColDQ, tmem + kColS0 + b * 128u + kk * 8u, bd, kIdDQ,
+                       (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        ptx::umma_commit(bar_ds_free);
-        ptx::umma_commit(bar_kv_empty(stage));
+        ptx::umma_commit(bar_k_empty(kstage));
+        ++ds_cnt;
         return true;
       };
       for (uint32_t rn = 0; ok; ++rn) {
@@ -209,15 +230,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ptx::mbar_wait(bar_q_full, q_phase, abort_flag, a.err, lim, ptx::wait_site(2, 1, 4))) { ok = false; break; }
         q_phase ^= 1u;
         ptx::tc_fence_after();
-        uint32_t prev_stage = 0;
+        uint32_t prev_ks = 0;
         for (int j = 0; j < n; ++j) {
-          if (!ptx::mbar_wait(bar_kv_full(kv_stage), kv_phase, abort_flag, a.err, lim, ptx::wait_site(2, 1, 5))) { ok = false; break; }
-          const uint32_t sb = s_cnt & 1u;
-          const uint32_t sph = (s_cnt >> 1) & 1u;
-          if (!ptx::mbar_wait(bar_s_empty(sb), sph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 1, 6))) { ok = false; break; }
+          // S_j = Q K_j^T.  Its buffer last held S/dS of tile j-2, whose dQ MMA
+          // was issued before this point, so the in-order pipe keeps them apart.
+          if (!ptx::mbar_wait(bar_k_full(ks), kph, abort_flag, a.err, lim, ptx::wait_site(2, 1, 5))) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t sk = sbase + L::kK0 + kv_stage * L::kStageBytes;
-          const uint32_t sv = sk + L::kTileBytes;
+          const uint32_t sb = s_cnt & 1u;
+          const uint32_t sk = sbase + L::kK0 + ks * L::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
@@ -226,9 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ptx::umma_commit(bar_s_full(sb));
           ++s_cnt;
+          // dP_j = dO V_j^T once the threads hold dP_{j-1} in registers
+          if (!ptx::mbar_wait(bar_v_full(vs), vph, abort_flag, a.err, lim, ptx::wait_site(2, 1, 6))) { ok = false; break; }
           if (!ptx::mbar_wait(bar_dp_empty, dp_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 1, 7))) { ok = false; break; }
           dp_phase ^= 1u;
           ptx::tc_fence_after();
+          const uint32_t sv = sbase + L::kV0 + vs * L::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
@@ -236,13 +259,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                          ptx::sdesc_sw128(sv + off, 16u, 1024u), kIdS, kk > 0 ? 1u : 0u);
           }
           ptx::umma_commit(bar_dp_full);
+          ptx::umma_commit(bar_v_empty(vs));
+          if (++vs == kVStages) { vs = 0; vph ^= 1u; }
           if (j == n - 1) ptx::umma_commit(bar_q_empty);
-          if (j > 0 && !issue_dq(j - 1, prev_stage)) { ok = false; break; }
-          prev_stage = kv_stage;
-          if (++kv_stage == kStages) { kv_stage = 0; kv_phase ^= 1u; }
+          if (j > 0 && !issue_dq(j - 1, prev_ks)) { ok = false; break; }
+          prev_ks = ks;
+          if (++ks == kKStages) { ks = 0; kph ^= 1u; }
         }
         if (!ok) break;
-        if (!issue_dq(n - 1, prev_stage)) { ok = false; break; }
+        if (!issue_dq(n - 1, prev_ks)) { ok = false; break; }
+        ptx::umma_commit(bar_dq_done);
       }
       ptx::umma_commit(bar_drain);
       volatile int never = 0;
@@ -253,9 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t sDS = sbase + L::kDS;
     const float sl2 = a.scale_log2;
-    uint32_t s_cnt = 0, dp_cnt = 0, ds_cnt = 0;
+    uint32_t s_cnt = 0, dp_cnt = 0, items = 0;
     bool ok = true;
     for (uint32_t rn = 0; ok; ++rn) {
       int item = 0;
@@ -275,8 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float dval = a.ds[int64_t(h) * a.n_slots + slot];
       for (int j = 0; j < n; ++j) {
         const uint32_t sb = s_cnt & 1u;
-        const uint32_t sph = (s_cnt >> 1) & 1u;
-        bool w = ptx::mbar_wait(bar_s_full(sb), sph, abort_flag, a.err, lim, ptx::wait_site(2, 2, 8));
+        bool w = ptx::mbar_wait(bar_s_full(sb), (s_cnt >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 8));
         w = w && ptx::mbar_wait(bar_dp_full, dp_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 9));
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         ++dp_cnt;
@@ -298,61 +322,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         lo = max(lo, 0);
         hi = min(hi, 128);
-        if (j > 0) {
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_ds_free, ds_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 10)))) {
-            ok = false;
-            break;
-          }
-          ++ds_cnt;
-        }
-        // S in chunks of 32 columns; the load of chunk c+1 overlaps the math of chunk c.
-        uint32_t sbuf[2][32];
-        ptx::tmem_ld32(tl + kColS0 + sb * 128u, sbuf[0]);
-        ptx::tmem_wait_ld();
+        // dS in two halves of 64 keys: the S columns of a half are all read
+        // before its 32 packed dS columns overwrite the front of the buffer.
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < 3) ptx::tmem_ld32(tl + kColS0 + sb * 128u + (c + 1) * 32u, sbuf[(c + 1) & 1]);
-          const uint32_t* sr = sbuf[c & 1];
-          uint32_t pk[16];
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float v2[2];
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = hf * 2 + cc;
+            uint32_t sr[32];
+            ptx::tmem_ld32(tl + kColS0 + sb * 128u + c * 32u, sr);
+            ptx::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int col = c * 32 + i + e;
-              const float p = (col >= lo && col < hi)
-                                  ? ptx::ex2(fmaf(__uint_as_float(sr[i + e]), sl2, neg_l2))
-                                  : 0.f;
-              v2[e] = p * (__uint_as_float(dp[c][i + e]) - dval);
+            for (int i = 0; i < 32; i += 2) {
+              float v2[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int col = c * 32 + i + e;
+                const float p = (col >= lo && col < hi)
+                                    ? ptx::ex2(fmaf(__uint_as_float(sr[i + e]), sl2, neg_l2))
+                                    : 0.f;
+                v2[e] = p * (__uint_as_float(dp[c][i + e]) - dval);
+              }
+              pk[cc * 16 + (i >> 1)] = ptx::pack_bf16x2(v2[0], v2[1]);
             }
-            pk[i >> 1] = ptx::pack_bf16x2(v2[0], v2[1]);
           }
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int ch = c * 4 + q4;
-            const uint32_t addr = sDS + (ch >> 3) * 16384u + row * 128u + (((ch & 7) ^ (row & 7)) << 4);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[q4 * 4 + 0]),
-                         "r"(pk[q4 * 4 + 1]), "r"(pk[q4 * 4 + 2]), "r"(pk[q4 * 4 + 3])
-                         : "memory");
-          }
-          ptx::tmem_wait_ld();
-          if (c == 2) {  // all four chunks of S are in registers now
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(bar_s_empty(sb));
-          }
+          ptx::tmem_st32(tl + kColS0 + sb * 128u + hf * 32u, pk);
         }
-        ++s_cnt;
-        ptx::fence_proxy_async_smem();
+        ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(bar_ds_full);
+        ptx::mbar_arrive(bar_ds_full(sb));
+        ++s_cnt;
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_ds_free, ds_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 11)))) {
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_dq_done, items & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 11)))) {
         ok = false;
         break;
       }
-      ++ds_cnt;
+      ++items;
       ptx::tc_fence_after();
       const int r = m.row;
 #pragma unroll
