@@ -215,13 +215,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ptx::tc_fence_after();
           const uint32_t sb = sbase + L::kStage0 + stg * L::kStageBytes;
+          const uint64_t pd0 = ptx::sdesc_sw128(sPT, 16u, 1024u);
+          const uint64_t sd0 = ptx::sdesc_sw128(sDST, 16u, 1024u);
+          const uint64_t od0 = ptx::sdesc_sw128(sb + L::kSDO, 8192u, 1024u);
+          const uint64_t qd0 = ptx::sdesc_sw128(sb + L::kSQ, 8192u, 1024u);
 #pragma unroll
           for (int kk = 0; kk < kHalf / 16; ++kk) {
             const uint32_t acc = (!first_grad || kk > 0) ? 1u : 0u;
-            ptx::umma_ss(tmem + kColDV, ptx::sdesc_sw128(sPT + kk * 32u, 16u, 1024u),
-                         ptx::sdesc_sw128(sb + L::kSDO + kk * 2048u, 8192u, 1024u), kIdG, acc);
-            ptx::umma_ss(tmem + kColDK, ptx::sdesc_sw128(sDST + kk * 32u, 16u, 1024u),
-                         ptx::sdesc_sw128(sb + L::kSQ + kk * 2048u, 8192u, 1024u), kIdG, acc);
+            ptx::umma_ss(tmem + kColDV, ptx::sdesc_add(pd0, kk * 32u), ptx::sdesc_add(od0, kk * 2048u), kIdG, acc);
+            ptx::umma_ss(tmem + kColDK, ptx::sdesc_add(sd0, kk * 32u), ptx::sdesc_add(qd0, kk * 2048u), kIdG, acc);
           }
           first_grad = false;
           ptx::umma_commit(bar_pd_free);
@@ -239,19 +241,23 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!ptx::mbar_wait(bar_sd_empty(b), bph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 7))) { ok = false; break; }
               ptx::tc_fence_after();
               const uint32_t sb = sbase + L::kStage0 + st * L::kStageBytes;
+              const uint64_t kd0 = ptx::sdesc_sw128(sK, 16u, 1024u);
+              const uint64_t vd0 = ptx::sdesc_sw128(sV, 16u, 1024u);
+              const uint64_t qd0 = ptx::sdesc_sw128(sb + L::kSQ, 16u, 1024u);
+              const uint64_t od0 = ptx::sdesc_sw128(sb + L::kSDO, 16u, 1024u);
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t offA = (kk >> 2) * 16384u + (kk & 3) * 32u;
                 const uint32_t offB = (kk >> 2) * 8192u + (kk & 3) * 32u;
-                ptx::umma_ss(tmem + kColS + b * kHalf, ptx::sdesc_sw128(sK + offA, 16u, 1024u),
-                             ptx::sdesc_sw128(sb + L::kSQ + offB, 16u, 1024u), kIdS, kk > 0 ? 1u : 0u);
+                ptx::umma_ss(tmem + kColS + b * kHalf, ptx::sdesc_add(kd0, offA), ptx::sdesc_add(qd0, offB),
+                             kIdS, kk > 0 ? 1u : 0u);
               }
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t offA = (kk >> 2) * 16384u + (kk & 3) * 32u;
                 const uint32_t offB = (kk >> 2) * 8192u + (kk & 3) * 32u;
-                ptx::umma_ss(tmem + kColDP + b * kHalf, ptx::sdesc_sw128(sV + offA, 16u, 1024u),
-                             ptx::sdesc_sw128(sb + L::kSDO + offB, 16u, 1024u), kIdS, kk > 0 ? 1u : 0u);
+                ptx::umma_ss(tmem + kColDP + b * kHalf, ptx::sdesc_add(vd0, offA), ptx::sdesc_add(od0, offB),
+                             kIdS, kk > 0 ? 1u : 0u);
               }
               ptx::umma_commit(bar_sd_full(b));
               ++sd_cnt;

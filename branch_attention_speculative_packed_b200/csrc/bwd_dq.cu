@@ -209,9 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ptx::mbar_wait(bar_ds_full(b), (ds_cnt >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 1, 3))) return false;
         ptx::tc_fence_after();
         const uint32_t sk = sbase + L::kK0 + kstage * L::kTileBytes;
+        const uint64_t bd0 = ptx::sdesc_sw128(sk, 16384u, 1024u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = ptx::sdesc_sw128(sk + kk * 2048u, 16384u, 1024u);
+          const uint64_t bd = ptx::sdesc_add(bd0, kk * 2048u);
           ptx::umma_ts(tmem + kColDQ, tmem + kColS0 + b * 128u + kk * 8u, bd, kIdDQ,
                        (jj > 0 || kk > 0) ? 1u : 0u);
         }
@@ -238,11 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tc_fence_after();
           const uint32_t sb = s_cnt & 1u;
           const uint32_t sk = sbase + L::kK0 + ks * L::kTileBytes;
+          const uint64_t qd0 = ptx::sdesc_sw128(sQ, 16u, 1024u);
+          const uint64_t kd0 = ptx::sdesc_sw128(sk, 16u, 1024u);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-            ptx::umma_ss(tmem + kColS0 + sb * 128u, ptx::sdesc_sw128(sQ + off, 16u, 1024u),
-                         ptx::sdesc_sw128(sk + off, 16u, 1024u), kIdS, kk > 0 ? 1u : 0u);
+            ptx::umma_ss(tmem + kColS0 + sb * 128u, ptx::sdesc_add(qd0, off), ptx::sdesc_add(kd0, off),
+                         kIdS, kk > 0 ? 1u : 0u);
           }
           ptx::umma_commit(bar_s_full(sb));
           ++s_cnt;
@@ -252,11 +255,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           dp_phase ^= 1u;
           ptx::tc_fence_after();
           const uint32_t sv = sbase + L::kV0 + vs * L::kTileBytes;
+          const uint64_t od0 = ptx::sdesc_sw128(sDO, 16u, 1024u);
+          const uint64_t vd0 = ptx::sdesc_sw128(sv, 16u, 1024u);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-            ptx::umma_ss(tmem + kColDP, ptx::sdesc_sw128(sDO + off, 16u, 1024u),
-                         ptx::sdesc_sw128(sv + off, 16u, 1024u), kIdS, kk > 0 ? 1u : 0u);
+            ptx::umma_ss(tmem + kColDP, ptx::sdesc_add(od0, off), ptx::sdesc_add(vd0, off), kIdS,
+                         kk > 0 ? 1u : 0u);
           }
           ptx::umma_commit(bar_dp_full);
           ptx::umma_commit(bar_v_empty(vs));

@@ -239,9 +239,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ptx::mbar_wait(bar.p_full[pb], (pv_cnt >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 1, 3))) return false;
         ptx::tc_fence_after();
         const uint32_t sv = sbase + L::kK0 + stage * L::kStageBytes + L::kTileBytes;
+        const uint64_t bd0 = ptx::sdesc_sw128(sv, 16384u, 1024u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = ptx::sdesc_sw128(sv + kk * 2048u, 16384u, 1024u);
+          const uint64_t bd = ptx::sdesc_add(bd0, kk * 2048u);
           ptx::umma_ts(tmem + kColO, tmem + kColP + pb * 64u + kk * 8u, bd, kIdPV,
                        (jj > 0 || kk > 0) ? 1u : 0u);
         }
@@ -269,11 +270,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ptx::mbar_wait(bar.s_empty[sb], sph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(1, 1, 6))) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t sk = sbase + L::kK0 + kv_stage * L::kStageBytes;
+          const uint64_t ad0 = ptx::sdesc_sw128(sQ, 16u, 1024u);
+          const uint64_t bd0 = ptx::sdesc_sw128(sk, 16u, 1024u);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-            const uint64_t ad = ptx::sdesc_sw128(sQ + off, 16u, 1024u);
-            const uint64_t bd = ptx::sdesc_sw128(sk + off, 16u, 1024u);
+            const uint64_t ad = ptx::sdesc_add(ad0, off);
+            const uint64_t bd = ptx::sdesc_add(bd0, off);
             ptx::umma_ss(tmem + kColS0 + sb * 128u, ad, bd, kIdS, kk > 0 ? 1u : 0u);
           }
           ptx::umma_commit(bar.s_full[sb]);
