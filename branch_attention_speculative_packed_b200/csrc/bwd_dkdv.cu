@@ -7,16 +7,20 @@
 //   S^T  = K Q^T      [128 keys x 64 rows]  -> TMEM (two buffers)
 //   dP^T = V dO^T     [128 x 64]            -> TMEM (two buffers)
 //   threads (one key per thread): P^T = exp2(S^T*scale*log2e - L*log2e) where
-//       key <= the row's limit, dS^T = P^T (dP^T - D)  -> shared memory (bf16)
-//   dV += P^T dO,  dK += dS^T Q             -> TMEM accumulators
+//       key <= the row's limit, dS^T = P^T (dP^T - D), written as bf16 into
+//       the first 32 columns of S^T's and dP^T's own TMEM buffers
+//   dV += P^T dO,  dK += dS^T Q             (A operand read from TMEM)
 // and finally dK * scale and dV are written as bf16 for the keys this item
 // owns (a key tile may run past its document's end; those keys belong to the
 // next document's items and are not written here).
 //
+// The tensor pipe runs the gradient MMAs of sub-tile i (reading P^T_i and
+// dS^T_i) before the S^T / dP^T MMAs of sub-tile i + 2, which overwrite those
+// buffers, so the two S^T / dP^T buffers double-buffer P^T / dS^T as well.
+//
 // Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-5
 // one key row each.  TMEM: dK 0..127, dV 128..255, S^T 256 / 320, dP^T 384 / 448.
-// Shared memory: K | V | 3 stages of (Q half, dO half, L, D, slot metadata) |
-// P^T | dS^T.
+// Shared memory: K | V | 4 stages of (Q half, dO half, L, D, slot metadata).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -27,7 +31,7 @@ namespace ba {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kHalf = 64;  // query rows per sub-tile
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;
@@ -41,11 +45,9 @@ struct Smem {
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kKVBytes;
   static constexpr uint32_t kStage0 = kV + kKVBytes;
-  static constexpr uint32_t kPT = kStage0 + kStages * kStageBytes;
-  static constexpr uint32_t kDST = kPT + 128u * kHalf * 2u;
-  static constexpr uint32_t kBar = kDST + 128u * kHalf * 2u;
-  // kv_full, kv_empty, st_full[3], st_empty[3], sd_full[2], sd_empty[2], pd_full, pd_free,
-  // acc_full, acc_free, drain, item_full[4], item_empty[4]
+  static constexpr uint32_t kBar = kStage0 + kStages * kStageBytes;
+  // kv_full, kv_empty, st_full[4], st_empty[4], sd_full[2], pd_full[2], acc_full, acc_free,
+  // drain, item_full[4], item_empty[4]
   static constexpr uint32_t kNumBars = 25;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base, abort, item slots[4]
   static constexpr uint32_t kTotal = kMisc + 32u;
@@ -78,11 +80,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t b0 = sbase + L::kBar;
   const uint32_t bar_kv_full = b0, bar_kv_empty = b0 + 8;
-  auto bar_st_full = [&](uint32_t s) { return b0 + 16 + 8 * s; };
-  auto bar_st_empty = [&](uint32_t s) { return b0 + 40 + 8 * s; };
-  auto bar_sd_full = [&](uint32_t s) { return b0 + 64 + 8 * s; };
-  auto bar_sd_empty = [&](uint32_t s) { return b0 + 80 + 8 * s; };
-  const uint32_t bar_pd_full = b0 + 96, bar_pd_free = b0 + 104;
+  auto bar_st_full = [&](uint32_t s) { return b0 + 16 + 8 * s; };   // 4
+  auto bar_st_empty = [&](uint32_t s) { return b0 + 48 + 8 * s; };  // 4
+  auto bar_sd_full = [&](uint32_t s) { return b0 + 80 + 8 * s; };   // 2
+  auto bar_pd_full = [&](uint32_t s) { return b0 + 96 + 8 * s; };   // 2
   const uint32_t bar_acc_full = b0 + 112, bar_acc_free = b0 + 120, bar_drain = b0 + 128;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -100,10 +101,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (uint32_t i = 0; i < 2; ++i) {
       ptx::mbar_init(bar_sd_full(i), 1);
-      ptx::mbar_init(bar_sd_empty(i), 128);
+      ptx::mbar_init(bar_pd_full(i), 128);
     }
-    ptx::mbar_init(bar_pd_full, 128);
-    ptx::mbar_init(bar_pd_free, 1);
     ptx::mbar_init(bar_acc_full, 1);
     ptx::mbar_init(bar_acc_free, 128);
     ptx::mbar_init(bar_drain, 1);
@@ -194,7 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kv_phase = 0, st = 0, st_phase = 0, pd_phase = 0, acc_phase = 0, sd_cnt = 0;
       bool ok = true;
       const uint32_t sK = sbase + L::kK, sV = sbase + L::kV;
-      const uint32_t sPT = sbase + L::kPT, sDST = sbase + L::kDST;
       for (uint32_t rn = 0; ok; ++rn) {
         int item = 0;
         if (!ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(3, 1, 14))) { ok = false; break; }
@@ -204,29 +202,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         kv_phase ^= 1u;
         ptx::tc_fence_after();
         bool first_grad = true;
-        uint32_t prev_st = 0;
+        uint32_t prev_st = 0, prev_b = 0;
         bool have_prev = false;
-        auto issue_grad = [&](uint32_t stg) -> bool {
-          if (!ptx::mbar_wait(bar_pd_full, pd_phase, abort_flag, a.err, lim, ptx::wait_site(3, 1, 4))) return false;
-          pd_phase ^= 1u;
+        auto issue_grad = [&](uint32_t stg, uint32_t pb) -> bool {
+          // pd_phase bit pb: parity of buffer pb's next P^T / dS^T hand-over
+          if (!ptx::mbar_wait(bar_pd_full(pb), (pd_phase >> pb) & 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 4))) return false;
+          pd_phase ^= 1u << pb;
           if (first_grad) {  // the previous item's epilogue has read dK / dV
             if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 5))) return false;
             acc_phase ^= 1u;
           }
           ptx::tc_fence_after();
           const uint32_t sb = sbase + L::kStage0 + stg * L::kStageBytes;
-          const uint64_t pd0 = ptx::sdesc_sw128(sPT, 16u, 1024u);
-          const uint64_t sd0 = ptx::sdesc_sw128(sDST, 16u, 1024u);
           const uint64_t od0 = ptx::sdesc_sw128(sb + L::kSDO, 8192u, 1024u);
           const uint64_t qd0 = ptx::sdesc_sw128(sb + L::kSQ, 8192u, 1024u);
+          const uint32_t pt = tmem + kColS + pb * kHalf, dst = tmem + kColDP + pb * kHalf;
 #pragma unroll
           for (int kk = 0; kk < kHalf / 16; ++kk) {
             const uint32_t acc = (!first_grad || kk > 0) ? 1u : 0u;
-            ptx::umma_ss(tmem + kColDV, ptx::sdesc_add(pd0, kk * 32u), ptx::sdesc_add(od0, kk * 2048u), kIdG, acc);
-            ptx::umma_ss(tmem + kColDK, ptx::sdesc_add(sd0, kk * 32u), ptx::sdesc_add(qd0, kk * 2048u), kIdG, acc);
+            ptx::umma_ts(tmem + kColDV, pt + kk * 8u, ptx::sdesc_add(od0, kk * 2048u), kIdG, acc);
+            ptx::umma_ts(tmem + kColDK, dst + kk * 8u, ptx::sdesc_add(qd0, kk * 2048u), kIdG, acc);
           }
           first_grad = false;
-          ptx::umma_commit(bar_pd_free);
           ptx::umma_commit(bar_st_empty(stg));
           return true;
         };
@@ -236,9 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int hh = 0; hh < G && ok; ++hh) {
             for (int half = 0; half < nh; ++half) {
               if (!ptx::mbar_wait(bar_st_full(st), st_phase, abort_flag, a.err, lim, ptx::wait_site(3, 1, 6))) { ok = false; break; }
+              // buffer b last held sub-tile sd_cnt - 2, whose gradient MMAs were issued above
               const uint32_t b = sd_cnt & 1u;
-              const uint32_t bph = (sd_cnt >> 1) & 1u;
-              if (!ptx::mbar_wait(bar_sd_empty(b), bph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 7))) { ok = false; break; }
               ptx::tc_fence_after();
               const uint32_t sb = sbase + L::kStage0 + st * L::kStageBytes;
               const uint64_t kd0 = ptx::sdesc_sw128(sK, 16u, 1024u);
@@ -261,15 +257,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               ptx::umma_commit(bar_sd_full(b));
               ++sd_cnt;
-              if (have_prev && !issue_grad(prev_st)) { ok = false; break; }
+              if (have_prev && !issue_grad(prev_st, prev_b)) { ok = false; break; }
               prev_st = st;
+              prev_b = b;
               have_prev = true;
               if (++st == kStages) { st = 0; st_phase ^= 1u; }
             }
           }
         }
         if (!ok) break;
-        if (have_prev && !issue_grad(prev_st)) { ok = false; break; }
+        if (have_prev && !issue_grad(prev_st, prev_b)) { ok = false; break; }
         if (first_grad) {  // no gradient MMA in this item: still pair the epilogue handshake
           if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 8))) { ok = false; break; }
           acc_phase ^= 1u;
@@ -286,9 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key row within the tile
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t sPT = sbase + L::kPT, sDST = sbase + L::kDST;
     const float sl2 = a.scale_log2;
-    uint32_t st = 0, st_phase = 0, sd_cnt = 0, pd_cnt = 0, acc_cnt = 0;
+    uint32_t st = 0, st_phase = 0, sd_cnt = 0, acc_cnt = 0;
     bool ok = true;
     for (uint32_t rn = 0; ok; ++rn) {
       int item = 0;
@@ -321,8 +317,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_ld32(tl + kColDP + b * kHalf, pv[0]);
             ptx::tmem_ld32(tl + kColDP + b * kHalf + 32u, pv[1]);
             ptx::tmem_wait_ld();
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(bar_sd_empty(b));
             // the stage's L, D and metadata landed (TMA completion, seen by this thread)
             if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_st_full(st), st_phase, abort_flag, a.err, lim, ptx::wait_site(3, 2, 12)))) {
               ok = false;
@@ -343,34 +337,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sv[c][i] = __float_as_uint(p);
                 pv[c][i] = __float_as_uint(p * (__uint_as_float(pv[c][i]) - Ds[col]));
               }
-            if (pd_cnt > 0) {
-              // the previous sub-tile's gradient MMAs have read P^T / dS^T
-              if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_pd_free, (pd_cnt - 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(3, 2, 10)))) {
-                ok = false;
-                break;
-              }
-            }
+            // bf16 pairs (lower row in the low half) over S^T's / dP^T's first 32 columns
+            uint32_t pk[32], dk[32];
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const int c = ch >> 2, i0 = (ch & 3) * 8;
-              const uint32_t off = row * 128u + (((ch ^ (row & 7))) << 4);
-              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPT + off),
-                           "r"(ptx::pack_bf16x2(__uint_as_float(sv[c][i0 + 0]), __uint_as_float(sv[c][i0 + 1]))),
-                           "r"(ptx::pack_bf16x2(__uint_as_float(sv[c][i0 + 2]), __uint_as_float(sv[c][i0 + 3]))),
-                           "r"(ptx::pack_bf16x2(__uint_as_float(sv[c][i0 + 4]), __uint_as_float(sv[c][i0 + 5]))),
-                           "r"(ptx::pack_bf16x2(__uint_as_float(sv[c][i0 + 6]), __uint_as_float(sv[c][i0 + 7])))
-                           : "memory");
-              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sDST + off),
-                           "r"(ptx::pack_bf16x2(__uint_as_float(pv[c][i0 + 0]), __uint_as_float(pv[c][i0 + 1]))),
-                           "r"(ptx::pack_bf16x2(__uint_as_float(pv[c][i0 + 2]), __uint_as_float(pv[c][i0 + 3]))),
-                           "r"(ptx::pack_bf16x2(__uint_as_float(pv[c][i0 + 4]), __uint_as_float(pv[c][i0 + 5]))),
-                           "r"(ptx::pack_bf16x2(__uint_as_float(pv[c][i0 + 6]), __uint_as_float(pv[c][i0 + 7])))
-                           : "memory");
+            for (int j = 0; j < 32; ++j) {
+              const int c = j >> 4, i = (j & 15) * 2;
+              pk[j] = ptx::pack_bf16x2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
+              dk[j] = ptx::pack_bf16x2(__uint_as_float(pv[c][i]), __uint_as_float(pv[c][i + 1]));
             }
-            ptx::fence_proxy_async_smem();
+            ptx::tmem_st32(tl + kColS + b * kHalf, pk);
+            ptx::tmem_st32(tl + kColDP + b * kHalf, dk);
+            ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            ptx::mbar_arrive(bar_pd_full);
-            ++pd_cnt;
+            ptx::mbar_arrive(bar_pd_full(b));
             any = true;
             if (++st == kStages) { st = 0; st_phase ^= 1u; }
           }
