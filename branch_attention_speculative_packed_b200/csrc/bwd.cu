@@ -68,11 +68,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepArgs a) {
     if (sub == 0) {
       const int64_t hs = int64_t(h) * a.n_slots + slot;
       if (r >= 0) {
-        a.ls[hs] = a.lse[int64_t(h) * a.rows + r] * 1.4426950408889634f;
+        a.ls[hs] = -a.lse[int64_t(h) * a.rows + r] * 1.4426950408889634f;
         a.ds[hs] = dsum;
         a.drow[int64_t(h) * a.rows + r] = dsum;
       } else {
-        a.ls[hs] = INFINITY;  // padding: P = exp2(s - inf) = 0
+        a.ls[hs] = -INFINITY;  // padding: P = exp2(s - inf) = 0
         a.ds[hs] = 0.f;
       }
       if (h == 0) {

@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const KvItem it = a.items[code / a.Hkv];
       const int g = code % a.Hkv;
       const int kp = it.key0 + row;  // this thread's key position
+      const int warp_last_key = it.key0 + quarter * 32 + 31;
       bool any = false;
       for (int ti = 0; ti < it.t_count && ok; ++ti) {
         const TileDesc td = a.tiles[it.t_first + it.t_count - 1 - ti];
@@ -323,20 +324,51 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             const uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
-            const float* Ls = reinterpret_cast<const float*>(sb + L::kSL);
-            const float* Ds = reinterpret_cast<const float*>(sb + L::kSD);
+            const float4* L4 = reinterpret_cast<const float4*>(sb + L::kSL);  // -L * log2(e)
+            const float4* D4 = reinterpret_cast<const float4*>(sb + L::kSD);
             const SlotMeta* Ms = reinterpret_cast<const SlotMeta*>(sb + L::kSM);
-            // P^T and dS^T of this key row over the 64 query rows
+            // exponent arguments S^T * scale*log2(e) - L*log2(e), two rows per instruction
+            const float2 c2 = make_float2(sl2, sl2);
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+            for (int q = 0; q < 16; ++q) {
+              const float4 l = L4[q];
+              const int c = q >> 3, i = (q & 7) * 4;
+              const float2 x0 = ptx::fma2(make_float2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])), c2,
+                                          make_float2(l.x, l.y));
+              const float2 x1 = ptx::fma2(make_float2(__uint_as_float(sv[c][i + 2]), __uint_as_float(sv[c][i + 3])), c2,
+                                          make_float2(l.z, l.w));
+              sv[c][i] = __float_as_uint(x0.x);
+              sv[c][i + 1] = __float_as_uint(x0.y);
+              sv[c][i + 2] = __float_as_uint(x1.x);
+              sv[c][i + 3] = __float_as_uint(x1.y);
+            }
+            // The half's rows are sorted by limit (padding, limit -1, only at a tile's end), so
+            // when the warp's last key is visible to the first row, every pair is visible.
+            if (!(warp_last_key <= Ms[0].limit)) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int col = c * 32 + i;
-                const bool vis = kp <= Ms[col].limit;
-                const float p = vis ? ptx::ex2(fmaf(__uint_as_float(sv[c][i]), sl2, -Ls[col])) : 0.f;
-                sv[c][i] = __float_as_uint(p);
-                pv[c][i] = __float_as_uint(p * (__uint_as_float(pv[c][i]) - Ds[col]));
-              }
+              for (int col = 0; col < 64; ++col)
+                if (kp > Ms[col].limit) sv[col >> 5][col & 31] = __float_as_uint(-INFINITY);
+            }
+            // P^T and dS^T = P^T (dP^T - D) of this key row over the 64 query rows
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const float4 dd = D4[q];
+              const int c = q >> 3, i = (q & 7) * 4;
+              const float2 p0 = make_float2(ptx::ex2(__uint_as_float(sv[c][i])), ptx::ex2(__uint_as_float(sv[c][i + 1])));
+              const float2 p1 = make_float2(ptx::ex2(__uint_as_float(sv[c][i + 2])), ptx::ex2(__uint_as_float(sv[c][i + 3])));
+              const float2 g0 = ptx::mul2(p0, ptx::sub2(make_float2(__uint_as_float(pv[c][i]), __uint_as_float(pv[c][i + 1])),
+                                                       make_float2(dd.x, dd.y)));
+              const float2 g1 = ptx::mul2(p1, ptx::sub2(make_float2(__uint_as_float(pv[c][i + 2]), __uint_as_float(pv[c][i + 3])),
+                                                       make_float2(dd.z, dd.w)));
+              sv[c][i] = __float_as_uint(p0.x);
+              sv[c][i + 1] = __float_as_uint(p0.y);
+              sv[c][i + 2] = __float_as_uint(p1.x);
+              sv[c][i + 3] = __float_as_uint(p1.y);
+              pv[c][i] = __float_as_uint(g0.x);
+              pv[c][i + 1] = __float_as_uint(g0.y);
+              pv[c][i + 2] = __float_as_uint(g1.x);
+              pv[c][i + 3] = __float_as_uint(g1.y);
+            }
             // bf16 pairs (lower row in the low half) over S^T's / dP^T's first 32 columns
             uint32_t pk[32], dk[32];
 #pragma unroll

@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = nkv + nbr;
       const int64_t slot = int64_t(td.row_base) + row;
       const SlotMeta m = a.meta[slot];
-      const float neg_l2 = -a.ls[int64_t(h) * a.n_slots + slot];
+      const float neg_l2 = a.ls[int64_t(h) * a.n_slots + slot];
       const float dval = a.ds[int64_t(h) * a.n_slots + slot];
       for (int j = 0; j < n; ++j) {
         const uint32_t sb = s_cnt & 1u;

@@ -19,7 +19,7 @@ struct PrepArgs {
   int64_t rows, n_slots;
   __nv_bfloat16* qg;         // [n_slots, Hq, d]
   __nv_bfloat16* dog;        // [n_slots, Hq, d]
-  float* ls;                 // [Hq, n_slots], log2-scaled LSE (+inf for padding)
+  float* ls;                 // [Hq, n_slots], -LSE * log2(e) (-inf for padding)
   float* ds;                 // [Hq, n_slots]
   float* drow;               // [Hq, rows]
   SlotMeta* meta;            // [n_slots]
@@ -42,7 +42,7 @@ struct DqArgs {
   const TileDesc* tiles;
   const int32_t* order;
   const SlotMeta* meta;
-  const float* ls;  // [Hq, n_slots]
+  const float* ls;  // [Hq, n_slots], -LSE * log2(e)
   const float* ds;  // [Hq, n_slots]
   int S, Hq, G, d;
   int64_t n_slots;
@@ -68,8 +68,8 @@ struct DkdvArgs {
   const int32_t* order;
   const TileDesc* tiles;
   const SlotMeta* meta;
-  const float* ls;
-  const float* ds;
+  const float* ls;  // [Hq, n_slots], -LSE * log2(e)
+  const float* ds;  // [Hq, n_slots]
   int Hq, Hkv, G, d;
   int64_t n_slots;
   int n_items;  // n_kv * Hkv
