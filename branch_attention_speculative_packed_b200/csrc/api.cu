@@ -179,9 +179,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   const void* kb = p->Nb > 0 ? p->kb : p->k;
   const void* vb = p->Nb > 0 ? p->vb : p->v;
   const int64_t nb_rows_map = p->Nb > 0 ? nbr_rows : p->S;
-  if (encode_2d(&maps.q, p->q, p->S, int64_t(p->Hq) * p->d, 1) != BA_OK ||
-      encode_2d(&maps.qb, qb, nb_rows_map, int64_t(p->Hq) * p->d, 1) != BA_OK ||
-      encode_2d(&maps.k, p->k, p->S, int64_t(p->Hkv) * p->d, 128) != BA_OK ||
+  if (encode_2d(&maps.k, p->k, p->S, int64_t(p->Hkv) * p->d, 128) != BA_OK ||
       encode_2d(&maps.v, p->v, p->S, int64_t(p->Hkv) * p->d, 128) != BA_OK ||
       encode_2d(&maps.kb, kb, nb_rows_map, int64_t(p->Hkv) * p->d, 128) != BA_OK ||
       encode_2d(&maps.vb, vb, nb_rows_map, int64_t(p->Hkv) * p->d, 128) != BA_OK)
@@ -190,6 +188,8 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   uint8_t* ws = static_cast<uint8_t*>(p->workspace);
   FwdArgs a;
   std::memset(&a, 0, sizeof(a));
+  a.q = static_cast<const __nv_bfloat16*>(p->q);
+  a.qb = static_cast<const __nv_bfloat16*>(qb);
   a.anchors = p->anchors_d;
   a.row_table = reinterpret_cast<const int32_t*>(ws + w.rows_off);
   a.tiles = reinterpret_cast<const TileDesc*>(ws + w.tiles_off);

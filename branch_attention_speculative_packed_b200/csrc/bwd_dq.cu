@@ -137,11 +137,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // parity of each stage's last fill and whether it may still be in flight (abort drain)
       uint32_t kpend = 0, kpar = 0, vpend = 0, vpar = 0, q_fills = 0;
       bool ok = true;
-      for (uint32_t rn = 0; ok; ++rn) {
-        const int item = static_cast<int>(atomicAdd(a.counter, 1u));
-        if (!ptx::ring_put(ring, rn, item, abort_flag, a.err, lim, ptx::wait_site(2, 0, 12))) { ok = false; break; }
-        if (item >= a.n_items) break;
-        const TileDesc td = a.tiles[a.order[item / Hq]];
+      // The ring runs one item ahead of the loads, so the next item's tile
+      // descriptor is fetched while this item's K/V tiles stream.
+      int item = static_cast<int>(atomicAdd(a.counter, 1u));
+      ok = ptx::ring_put(ring, 0, item, abort_flag, a.err, lim, ptx::wait_site(2, 0, 12));
+      TileDesc td = {};
+      if (ok && item < a.n_items) td = a.tiles[a.order[item / Hq]];
+      for (uint32_t rn = 1; ok && item < a.n_items; ++rn) {
+        const int nxt = static_cast<int>(atomicAdd(a.counter, 1u));
+        if (!ptx::ring_put(ring, rn, nxt, abort_flag, a.err, lim, ptx::wait_site(2, 0, 12))) { ok = false; break; }
+        TileDesc td_next = {};
+        if (nxt < a.n_items) td_next = a.tiles[a.order[nxt / Hq]];
         const int h = item % Hq;
         const int g = h / a.G;
         if (!ptx::mbar_wait(bar_q_empty, q_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 0, 1))) { ok = false; break; }
@@ -183,6 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           vpar = (vpar & ~(1u << vs)) | (vph << vs);
           if (++vs == kVStages) { vs = 0; vph ^= 1u; }
         }
+        item = nxt;
+        td = td_next;
       }
       if (*abort_flag) {
         volatile int never = 0;
@@ -327,6 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         lo = max(lo, 0);
         hi = min(hi, 128);
+        const bool full = lo == 0 && hi == 128;
+        const float2 c2 = make_float2(sl2, sl2), nl2 = make_float2(neg_l2, neg_l2), d2 = make_float2(dval, dval);
         // dS in two halves of 64 keys: the S columns of a half are all read
         // before its 32 packed dS columns overwrite the front of the buffer.
 #pragma unroll
@@ -338,18 +348,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t sr[32];
             ptx::tmem_ld32(tl + kColS0 + sb * 128u + c * 32u, sr);
             ptx::tmem_wait_ld();
+            // exponent arguments S * scale*log2(e) - L*log2(e), two keys per instruction
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-              float v2[2];
+              const float2 x = ptx::fma2(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2, nl2);
+              sr[i] = __float_as_uint(x.x);
+              sr[i + 1] = __float_as_uint(x.y);
+            }
+            if (!full) {
 #pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int col = c * 32 + i + e;
-                const float p = (col >= lo && col < hi)
-                                    ? ptx::ex2(fmaf(__uint_as_float(sr[i + e]), sl2, neg_l2))
-                                    : 0.f;
-                v2[e] = p * (__uint_as_float(dp[c][i + e]) - dval);
+              for (int i = 0; i < 32; ++i) {
+                const int col = c * 32 + i;
+                if (col < lo || col >= hi) sr[i] = __float_as_uint(-INFINITY);
               }
-              pk[cc * 16 + (i >> 1)] = ptx::pack_bf16x2(v2[0], v2[1]);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float2 p = make_float2(ptx::ex2(__uint_as_float(sr[i])), ptx::ex2(__uint_as_float(sr[i + 1])));
+              const float2 g = ptx::mul2(p, ptx::sub2(make_float2(__uint_as_float(dp[c][i]), __uint_as_float(dp[c][i + 1])), d2));
+              pk[cc * 16 + (i >> 1)] = ptx::pack_bf16x2(g.x, g.y);
             }
           }
           ptx::tmem_st32(tl + kColS0 + sb * 128u + hf * 32u, pk);

@@ -12,20 +12,25 @@
 // component, the branch-local component and their merge all happen here.
 //
 // Roles (192 threads):
-//   warp 0      TMA producer: gathers the 128 query rows of the tile (one
-//               1-row box per row and 64 columns) and streams K/V key tiles
-//               through a 3-stage ring.
+//   warp 0      producer: claims work items (one item ahead of the consumers)
+//               and streams the K/V key tiles through a 3-stage TMA ring.
 //   warp 1      TMEM allocator and single-thread MMA issuer:
 //               S[sb] = Q K^T into one of two TMEM buffers, then O += P V
 //               with P read from TMEM (A operand in tensor memory).
-//   warps 2-5   softmax / epilogue, one query row per thread: load S from
+//   warps 2-5   softmax / epilogue, one query row per thread.  Each thread
+//               copies its own query row into shared memory (cp.async): the
+//               next item's rows go in as soon as the current item's last
+//               S MMA, the only reader of Q, has finished, so the copy
+//               overlaps the last softmax step and the epilogue.  Per key
+//               tile: load S from
 //               TMEM, mask by the row's key range, update the running max
 //               (lazily: O in TMEM is rescaled only when the max grows by
 //               more than 2^8), write P (bf16) into one of two TMEM buffers
 //               for the P.V MMA, and finally normalise O and write O and LSE.
 //
 // Shared memory (D = head dim): Q [128 x D] | 3 x (K [128 x D], V [128 x D]),
-// bf16 in the 128-byte-swizzled layout TMA writes.
+// bf16 in the 128-byte-swizzled layout (TMA writes K / V; the threads write Q
+// in the same pattern).
 // TMEM: S buffers at columns 0 and 128, O at 256, P buffers at 384 and 448
 // (128 rows x 128 bf16 keys = 64 columns each).
 #include <cuda.h>
@@ -50,16 +55,16 @@ struct Smem {
   static constexpr uint32_t kK0 = kQ + kTileBytes;
   static constexpr uint32_t kStageBytes = 2u * kTileBytes;  // K + V
   static constexpr uint32_t kBar = kK0 + kStages * kStageBytes;
-  // barriers: q_full, q_empty, kv_full[3], kv_empty[3], s_full[2], s_empty[2], p_full[2],
-  // o_done[2], drain, item_full[4], item_empty[4]
-  static constexpr uint32_t kNumBars = 25;
+  // barriers: q_full, kv_full[3], kv_empty[3], s_full[2], s_empty[2], p_full[2], o_done[2],
+  // drain, item_full[4], item_empty[4]
+  static constexpr uint32_t kNumBars = 24;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base, abort, item slots[4]
   static constexpr uint32_t kTotal = kMisc + 32u;
   static constexpr uint32_t kAlloc = kTotal + 1024u;  // slack to align the base to 1024
 };
 
 struct Bars {
-  uint32_t q_full, q_empty, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full[2],
+  uint32_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full[2],
       o_done[2], drain;
 };
 
@@ -67,8 +72,7 @@ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; 
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQb,
-               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
                const FwdArgs a) {
   using L = Smem<D>;
@@ -83,7 +87,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     uint32_t b = sbase + L::kBar;
     bar.q_full = b; b += 8;
-    bar.q_empty = b; b += 8;
     for (int i = 0; i < kStages; ++i) { bar.kv_full[i] = b; b += 8; }
     for (int i = 0; i < kStages; ++i) { bar.kv_empty[i] = b; b += 8; }
     for (int i = 0; i < 2; ++i) { bar.s_full[i] = b; b += 8; }
@@ -100,8 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   ring.empty = ring.full + 8 * ptx::kItemSlots;
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(bar.q_full, 1);
-    ptx::mbar_init(bar.q_empty, 1);
+    ptx::mbar_init(bar.q_full, 128);  // one arrival per softmax thread (its copied row)
     for (int i = 0; i < kStages; ++i) {
       ptx::mbar_init(bar.kv_full[i], 1);
       ptx::mbar_init(bar.kv_empty[i], 1);
@@ -123,8 +125,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    ptx::prefetch_tmap(&tmQ);
-    ptx::prefetch_tmap(&tmQb);
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
     ptx::prefetch_tmap(&tmKb);
@@ -144,47 +144,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    uint32_t kv_stage = 0, kv_phase = 0, q_phase = 0;
-    // Parity of each stage's last fill and whether it may still be in flight
-    // (for the abort drain); same for the query tile.
-    uint32_t pend_mask = 0, pend_par = 0, q_fills = 0;
-    bool ok = true;
-    for (uint32_t rn = 0; ok; ++rn) {
-      int item = 0, put = 1;
-      if (lane == 0) {
-        item = static_cast<int>(atomicAdd(a.counter, 1u));
-        put = ptx::ring_put(ring, rn, item, abort_flag, a.err, lim, ptx::wait_site(1, 0, 12));
-      }
-      item = __shfl_sync(0xffffffffu, item, 0);
-      if (!__shfl_sync(0xffffffffu, put, 0)) { ok = false; break; }
-      if (item >= a.n_items) break;
-      const TileDesc td = a.tiles[a.order[item / Hq]];
-      const int h = item % Hq;
-      const int g = h / a.G;
-      int waited = 1;
-      if (lane == 0) waited = ptx::mbar_wait(bar.q_empty, q_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(1, 0, 1));
-      waited = __shfl_sync(0xffffffffu, waited, 0);
-      if (!waited) { ok = false; break; }
-      q_phase ^= 1u;
-      if (lane == 0) ptx::mbar_expect_tx(bar.q_full, L::kTileBytes);
-      ++q_fills;
-      __syncwarp();
-      for (int i = lane; i < 128; i += 32) {
-        const int r = a.row_table[td.row_base + i];
-        const void* map = &tmQ;
-        int y = -1;  // out of range: TMA fills zeros for padding rows
-        if (r >= 0 && r < a.S) {
-          y = r;
-        } else if (r >= a.S) {
-          map = &tmQb;
-          y = r - a.S;
-        }
-#pragma unroll
-        for (int cb = 0; cb < D / 64; ++cb)
-          ptx::tma_load_2d(sbase + L::kQ + cb * 16384u + i * 128u, map, bar.q_full, h * D + cb * 64, y);
-      }
-      __syncwarp();
-      if (lane == 0) {
+    if (lane == 0) {
+      uint32_t kv_stage = 0, kv_phase = 0;
+      // Parity of each stage's last fill and whether it may still be in flight (abort drain).
+      uint32_t pend_mask = 0, pend_par = 0;
+      // The ring runs one item ahead of the K/V stream, so the consumers learn
+      // the next item (and copy its query rows) before the current one ends.
+      int cur = static_cast<int>(atomicAdd(a.counter, 1u));
+      bool ok = ptx::ring_put(ring, 0, cur, abort_flag, a.err, lim, ptx::wait_site(1, 0, 12));
+      for (uint32_t rn = 1; ok && cur < a.n_items; ++rn) {
+        const int nxt = static_cast<int>(atomicAdd(a.counter, 1u));
+        if (!ptx::ring_put(ring, rn, nxt, abort_flag, a.err, lim, ptx::wait_site(1, 0, 12))) { ok = false; break; }
+        const TileDesc td = a.tiles[a.order[cur / Hq]];
+        const int g = (cur % Hq) / a.G;
         const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
         for (int j = 0; j < nkv + nbr; ++j) {
@@ -214,16 +186,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           pend_par = (pend_par & ~(1u << kv_stage)) | (kv_phase << kv_stage);
           if (++kv_stage == kStages) { kv_stage = 0; kv_phase ^= 1u; }
         }
+        cur = nxt;
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    }
-    if (lane == 0 && *abort_flag) {
-      // Let our own copies in flight land before the CTA exits (bounded).
-      volatile int never = 0;
-      for (int i = 0; i < kStages; ++i)
-        if (pend_mask & (1u << i))
-          ptx::mbar_wait(bar.kv_full[i], (pend_par >> i) & 1u, &never, a.err, lim / 8);
-      if (q_fills) ptx::mbar_wait(bar.q_full, (q_fills - 1) & 1u, &never, a.err, lim / 8);
+      if (*abort_flag) {
+        // Let our own copies in flight land before the CTA exits (bounded).
+        volatile int never = 0;
+        for (int i = 0; i < kStages; ++i)
+          if (pend_mask & (1u << i))
+            ptx::mbar_wait(bar.kv_full[i], (pend_par >> i) & 1u, &never, a.err, lim / 8);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -281,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ptx::umma_commit(bar.s_full[sb]);
           ++s_cnt;
-          if (j == n - 1) ptx::umma_commit(bar.q_empty);
           if (j > 0 && !issue_pv(j - 1, prev_stage)) { ok = false; break; }
           prev_stage = kv_stage;
           if (++kv_stage == kStages) { kv_stage = 0; kv_phase ^= 1u; }
@@ -301,34 +271,84 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float sl2 = a.scale_log2;
     uint32_t s_cnt = 0, pv_cnt = 0;  // S tiles consumed, P tiles produced
-    bool ok = true;
-    for (uint32_t rn = 0; ok; ++rn) {
+
+    // This thread's row of a work item.
+    struct RowItem {
+      bool valid;
+      int h, n, nkv, doc_start, br_lo, r, limit, blo, bhi;
+    };
+    auto fetch = [&](uint32_t rn, RowItem& it) -> bool {
       int item = 0;
-      if (!__all_sync(0xffffffffu, ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(1, 2, 14)))) {
-        ok = false;
-        break;
-      }
-      if (item >= a.n_items) break;
+      if (!__all_sync(0xffffffffu, ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(1, 2, 14))))
+        return false;
+      it.valid = item < a.n_items;
+      if (!it.valid) return true;
       const TileDesc td = a.tiles[a.order[item / Hq]];
-      const int h = item % Hq;
-      const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
-      const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
-      const int n = nkv + nbr;
-      const int r = a.row_table[td.row_base + row];
-      int limit = td.doc_start;  // padding rows see one key: keeps their math finite
-      int blo = 0, bhi = 0;      // visible branch key rows [blo, bhi)
-      if (r >= 0 && r < a.S) {
-        limit = r;
-      } else if (r >= a.S) {
-        const int b = (r - a.S) / a.B;
-        const int t = (r - a.S) - b * a.B;
-        limit = a.anchors[b];
-        blo = b * a.B;
-        bhi = blo + (a.mode == 1 ? a.B : t + 1);
+      it.h = item % Hq;
+      it.doc_start = td.doc_start;
+      it.br_lo = td.br_lo;
+      it.nkv = ceil_div(td.kv_end - td.doc_start, 128);
+      it.n = it.nkv + ((a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0);
+      it.r = a.row_table[td.row_base + row];
+      it.limit = td.doc_start;  // padding rows see one key: keeps their math finite
+      it.blo = it.bhi = 0;      // visible branch key rows [blo, bhi)
+      if (it.r >= 0 && it.r < a.S) {
+        it.limit = it.r;
+      } else if (it.r >= a.S) {
+        const int b = (it.r - a.S) / a.B;
+        const int t = (it.r - a.S) - b * a.B;
+        it.limit = a.anchors[b];
+        it.blo = b * a.B;
+        it.bhi = it.blo + (a.mode == 1 ? a.B : t + 1);
       }
+      return true;
+    };
+    // Copy this thread's query row (bf16, D values) into row `row` of the
+    // swizzled Q tile; padding rows are zero-filled.
+    auto copy_q = [&](const RowItem& it) {
+      const __nv_bfloat16* src = a.q;
+      uint32_t bytes = 0;
+      if (it.r >= 0 && it.r < a.S) {
+        src = a.q + (int64_t(it.r) * Hq + it.h) * D;
+        bytes = 16;
+      } else if (it.r >= a.S) {
+        src = a.qb + (int64_t(it.r - a.S) * Hq + it.h) * D;
+        bytes = 16;
+      }
+      const uint32_t dst = sbase + L::kQ + static_cast<uint32_t>(row) * 128u;
+#pragma unroll
+      for (int cb = 0; cb < D / 64; ++cb)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          ptx::cp_async16(dst + cb * 16384u + ((static_cast<uint32_t>(c) ^ (row & 7)) << 4),
+                          src + (bytes ? cb * 64 + c * 8 : 0), bytes);
+      ptx::cp_async_commit();
+    };
+    // The copies have landed: make them visible to the tensor core, then tell the MMA issuer.
+    auto publish_q = [&]() {
+      ptx::cp_async_wait_all();
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(bar.q_full);
+    };
+
+    RowItem cur;
+    bool ok = fetch(0, cur);
+    if (ok && cur.valid) {
+      copy_q(cur);
+      publish_q();
+    }
+    for (uint32_t rn = 1; ok && cur.valid; ++rn) {
+      const int h = cur.h, n = cur.n, nkv = cur.nkv, r = cur.r;
+      const int limit = cur.limit, blo = cur.blo, bhi = cur.bhi;
+      RowItem nxt;
+      nxt.valid = false;
       float m_used = -INFINITY;
       float l = 0.f;
       for (int j = 0; j < n; ++j) {
+        if (j == n - 1 && !fetch(rn, nxt)) {
+          ok = false;
+          break;
+        }
         const uint32_t sb = s_cnt & 1u;
         const uint32_t sph = (s_cnt >> 1) & 1u;
         if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.s_full[sb], sph, abort_flag, a.err, lim, ptx::wait_site(1, 2, 7)))) {
@@ -343,41 +363,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar.s_empty[sb]);
         ++s_cnt;
+        // The item's last S MMA has finished: the next item's rows may overwrite Q.
+        if (j == n - 1 && nxt.valid) copy_q(nxt);
         // visible columns [lo, hi) of this key tile
         int lo, hi;
         if (j < nkv) {
           lo = 0;
-          hi = limit - (td.doc_start + 128 * j) + 1;
+          hi = limit - (cur.doc_start + 128 * j) + 1;
         } else {
-          const int kr0 = td.br_lo + 128 * (j - nkv);
+          const int kr0 = cur.br_lo + 128 * (j - nkv);
           lo = blo - kr0;
           hi = bhi - kr0;
         }
         lo = max(lo, 0);
         hi = min(hi, 128);
-        // Row max with 8 independent accumulators (a single running max would
-        // be a 128-long dependency chain).
-        float mx8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-        if (lo == 0 && hi == 128) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[c][i]));
-        } else {
+        if (!(lo == 0 && hi == 128)) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int col = c * 32 + i;
-              const bool vis = col >= lo && col < hi;
-              if (!vis) sr[c][i] = __float_as_uint(-INFINITY);
-              mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(sr[c][i]));
+              if (col < lo || col >= hi) sr[c][i] = __float_as_uint(-INFINITY);
             }
         }
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        // Row max over 8 independent accumulators, two new values per instruction.
+        float mx8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            mx8[(i >> 1) & 7] = ptx::max3(mx8[(i >> 1) & 7], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+        const float mx = fmaxf(ptx::max3(mx8[0], mx8[1], mx8[2]),
+                               fmaxf(ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float mxs = mx * sl2;
         float alpha = 1.f;
         bool rescale = false;
@@ -388,20 +407,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = mxs;
           rescale = true;
         }
-        const float neg_m = -m_used;
-        float rs8[8];
+        // P = exp2(S * scale*log2(e) - m), row sum over 4 paired accumulators
+        const float2 c2 = make_float2(sl2, sl2);
+        const float2 nm2 = make_float2(-m_used, -m_used);
+        float2 rs4[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
+        for (int u = 0; u < 4; ++u) rs4[u] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p = ptx::ex2(fmaf(__uint_as_float(sr[c][i]), sl2, neg_m));
-            rs8[i & 7] += p;
-            sr[c][i] = __float_as_uint(p);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 x = ptx::fma2(make_float2(__uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1])), c2, nm2);
+            const float2 p = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+            rs4[(i >> 1) & 3] = ptx::add2(rs4[(i >> 1) & 3], p);
+            sr[c][i] = __float_as_uint(p.x);
+            sr[c][i + 1] = __float_as_uint(p.y);
           }
-        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-        l = l * alpha + rs;
+        const float2 rsa = ptx::add2(ptx::add2(rs4[0], rs4[1]), ptx::add2(rs4[2], rs4[3]));
+        l = l * alpha + (rsa.x + rsa.y);
         const uint32_t pb = pv_cnt & 1u;
         // P buffer pb is free once the P.V that last read it (two tiles ago) finished.
         bool w = true;
@@ -442,6 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++pv_cnt;
       }
       if (!ok) break;
+      // The next item's S MMAs may start while this item's epilogue runs.
+      if (nxt.valid) publish_q();
       // ---------------------------------------------------------- epilogue
       {  // the item's last P.V (and, in order, every earlier one) finished
         const uint32_t last = pv_cnt - 1u;
@@ -486,7 +511,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (r >= 0) a.lse[int64_t(h) * a.lse_ld + r] = (m_used + __log2f(l)) * 0.69314718055994531f;
       ptx::tc_fence_before();
+      cur = nxt;
     }
+    // Copies this thread issued must land before the CTA's shared memory goes away.
+    ptx::cp_async_wait_all();
   }
 
   ptx::tc_fence_before();
@@ -506,7 +534,7 @@ cudaError_t launch_fwd_d(const FwdMaps& m, const FwdArgs& a, int num_sms, cudaSt
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;
-  fwd_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(m.q, m.qb, m.k, m.v, m.kb, m.vb, a);
+  fwd_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(m.k, m.v, m.kb, m.vb, a);
   return cudaGetLastError();
 }
 

@@ -13,6 +13,8 @@ namespace ba {
 
 // ---------------------------------------------------------------- forward
 struct FwdArgs {
+  const __nv_bfloat16* q;    // [S, Hq, d]
+  const __nv_bfloat16* qb;   // [Nb*B, Hq, d] (q when there are no branches)
   const int32_t* anchors;    // [Nb]
   const int32_t* row_table;  // [ntiles * 128], -1 = padding
   const TileDesc* tiles;     // [ntiles]
@@ -33,7 +35,7 @@ struct FwdArgs {
 };
 
 struct FwdMaps {
-  CUtensorMap q, qb, k, v, kb, vb;
+  CUtensorMap k, v, kb, vb;  // [rows, Hkv*d], box 64 x 128
 };
 
 cudaError_t launch_fwd(const FwdMaps& maps, const FwdArgs& a, int num_sms, cudaStream_t stream);
