@@ -378,6 +378,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   pa.ds = reinterpret_cast<float*>(ws + w.ds_off);
   pa.drow = reinterpret_cast<float*>(ws + w.drow_off);
   pa.meta = reinterpret_cast<SlotMeta*>(ws + w.meta_off);
+  pa.lims = reinterpret_cast<int32_t*>(ws + w.lims_off);
   {
     ProfScope prof("bwd_prep", st);
     if (launch_bwd_prep(pa, p->d, st) != cudaSuccess) return BA_ERR_CUDA;
@@ -394,8 +395,8 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
       encode_2d(&dm.v, p->v, p->S, kcols, 128) != BA_OK ||
       encode_2d(&dm.kb, nb ? p->kb : p->k, nb_rows_map, kcols, 128) != BA_OK ||
       encode_2d(&dm.vb, nb ? p->vb : p->v, nb_rows_map, kcols, 128) != BA_OK ||
-      encode_2d(&km.qg, pa.qg, w.n_slots, qcols, 64) != BA_OK ||
-      encode_2d(&km.dog, pa.dog, w.n_slots, qcols, 64) != BA_OK)
+      encode_2d(&km.qg, pa.qg, w.n_slots, qcols, 128) != BA_OK ||
+      encode_2d(&km.dog, pa.dog, w.n_slots, qcols, 128) != BA_OK)
     return BA_ERR_CUDA;
   km.k = dm.k;
   km.v = dm.v;
@@ -433,7 +434,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   ka.items = reinterpret_cast<const KvItem*>(ws + w.kv_items_off);
   ka.order = reinterpret_cast<const int32_t*>(ws + w.kv_order_off);
   ka.tiles = qa.tiles;
-  ka.meta = pa.meta;
+  ka.lims = pa.lims;
   ka.ls = pa.ls;
   ka.ds = pa.ds;
   ka.Hq = p->Hq;

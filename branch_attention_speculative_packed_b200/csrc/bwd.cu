@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepArgs a) {
           m.bhi = m.blo + (a.mode == 1 ? a.B : t + 1);
         }
         a.meta[slot] = m;
+        a.lims[slot] = m.limit;
       }
     }
   }

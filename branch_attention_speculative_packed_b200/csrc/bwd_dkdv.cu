@@ -1,26 +1,35 @@
 // dK/dV pass of the backward on sm_100a (key-stationary, tcgen05 + TMEM).
 //
-// One persistent CTA per SM walks (main key tile, KV head) items, most work
-// first.  The item's K and V tiles (128 keys) stay in shared memory; the CTA
-// visits every row tile that can see them (a contiguous range of the plan's
-// tiles), for each of the G query heads of the KV head, in halves of 64 rows:
-//   S^T  = K Q^T      [128 keys x 64 rows]  -> TMEM (two buffers)
-//   dP^T = V dO^T     [128 x 64]            -> TMEM (two buffers)
-//   threads (one key per thread): P^T = exp2(S^T*scale*log2e - L*log2e) where
-//       key <= the row's limit, dS^T = P^T (dP^T - D), written as bf16 into
-//       the first 32 columns of S^T's and dP^T's own TMEM buffers
-//   dV += P^T dO,  dK += dS^T Q             (A operand read from TMEM)
+// One persistent CTA per SM takes (main key tile, KV head) items, most work
+// first, from a global counter.  The item's K and V tiles (128 keys) stay in
+// shared memory; the CTA visits every row tile that can see them (a
+// contiguous range of the plan's tiles), for each of the G query heads of the
+// KV head.  Per (row tile, head) sub-tile i of 128 query rows:
+//   S^T_i  = K Q_i^T     [128 keys x 128 rows]  -> TMEM buffer SB
+//   dP^T_i = V dO_i^T                           -> TMEM buffer DB
+//   threads (one key per thread, two warpgroups of 64 rows each):
+//       P^T = exp2(S^T*scale*log2e - L*log2e) where key <= the row's limit,
+//       written as bf16 over the front of each warpgroup's half of SB;
+//       dS^T = P^T (dP^T - D), written as bf16 the same way into DB
+//   dV += P^T dO_i,  dK += dS^T Q_i             (A operand read from TMEM)
 // and finally dK * scale and dV are written as bf16 for the keys this item
 // owns (a key tile may run past its document's end; those keys belong to the
 // next document's items and are not written here).
 //
-// The tensor pipe runs the gradient MMAs of sub-tile i (reading P^T_i and
-// dS^T_i) before the S^T / dP^T MMAs of sub-tile i + 2, which overwrite those
-// buffers, so the two S^T / dP^T buffers double-buffer P^T / dS^T as well.
+// The tensor pipe executes in issue order
+//     S_i, dK_{i-1}, dP_i, dV_i, S_{i+1}, dK_i, ...
+// so S_{i+1} overwrites SB only after dV_i has read P^T_i, and dP_{i+1}
+// overwrites DB only after dK_i has read dS^T_i; while the threads turn S_i
+// into P^T_i the pipe runs dK_{i-1} and dP_i, and while they form dS^T_i it
+// runs dV_i and S_{i+1}.  Every MMA is 128 x 128 x 16 (N = 128 runs the
+// tensor core at full rate; N = 64 costs nearly as much per instruction).
 //
-// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-5
-// one key row each.  TMEM: dK 0..127, dV 128..255, S^T 256 / 320, dP^T 384 / 448.
-// Shared memory: K | V | 4 stages of (Q half, dO half, L, D, slot metadata).
+// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
+// issuer, warps 2-9 one key row each (warps w and w + 4 share TMEM lane
+// quarter w % 4 and split the 128 query rows of a sub-tile).
+// TMEM: dK 0..127, dV 128..255, SB 256..383, DB 384..511.
+// Shared memory: K | V | 2 x (Q tile, L, D, limits) | 2 x dO tile.  Q_i is
+// released after dK_i and dO_i after dV_i.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -30,32 +39,29 @@
 namespace ba {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kStages = 4;
-constexpr int kHalf = 64;  // query rows per sub-tile
+constexpr int kThreads = 320;
+constexpr int kSlots = 2;  // Q and dO ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;
 
 template <int D>
 struct Smem {
-  static constexpr uint32_t kKVBytes = 128u * D * 2u;       // K or V tile
-  static constexpr uint32_t kHalfBytes = kHalf * D * 2u;    // Q or dO half tile
-  static constexpr uint32_t kMetaBytes = kHalf * (4u + 4u + 16u);  // L, D, SlotMeta
-  static constexpr uint32_t kStageBytes = ((2u * kHalfBytes + kMetaBytes) + 1023u) / 1024u * 1024u;
+  static constexpr uint32_t kTile = 128u * D * 2u;  // K, V, Q or dO tile (128 rows)
+  static constexpr uint32_t kMeta = 3u * 128u * 4u;  // L, D, limits of 128 rows
+  static constexpr uint32_t kQSlot = (kTile + kMeta + 1023u) / 1024u * 1024u;
   static constexpr uint32_t kK = 0;
-  static constexpr uint32_t kV = kK + kKVBytes;
-  static constexpr uint32_t kStage0 = kV + kKVBytes;
-  static constexpr uint32_t kBar = kStage0 + kStages * kStageBytes;
-  // kv_full, kv_empty, st_full[4], st_empty[4], sd_full[2], pd_full[2], acc_full, acc_free,
-  // drain, item_full[4], item_empty[4]
+  static constexpr uint32_t kV = kK + kTile;
+  static constexpr uint32_t kQ0 = kV + kTile;
+  static constexpr uint32_t kO0 = kQ0 + kSlots * kQSlot;
+  static constexpr uint32_t kBar = kO0 + kSlots * kTile;
+  // kv_full, kv_empty, q_full[2], q_empty[2], o_full[2], o_empty[2], s_full, p_ready, dp_full,
+  // ds_ready, acc_full, acc_free, drain, item_full[4], item_empty[4]
   static constexpr uint32_t kNumBars = 25;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base, abort, item slots[4]
   static constexpr uint32_t kTotal = kMisc + 32u;
   static constexpr uint32_t kAlloc = kTotal + 1024u;
-  // offsets inside a stage
-  static constexpr uint32_t kSQ = 0, kSDO = kHalfBytes, kSL = 2u * kHalfBytes;
-  static constexpr uint32_t kSD = kSL + kHalf * 4u, kSM = kSD + kHalf * 4u;
-  static constexpr uint32_t kStageTx = 2u * kHalfBytes + kMetaBytes;
+  // offsets inside a Q slot
+  static constexpr uint32_t kSL = kTile, kSD = kTile + 512u, kSLim = kTile + 1024u;
 };
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -80,10 +86,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t b0 = sbase + L::kBar;
   const uint32_t bar_kv_full = b0, bar_kv_empty = b0 + 8;
-  auto bar_st_full = [&](uint32_t s) { return b0 + 16 + 8 * s; };   // 4
-  auto bar_st_empty = [&](uint32_t s) { return b0 + 48 + 8 * s; };  // 4
-  auto bar_sd_full = [&](uint32_t s) { return b0 + 80 + 8 * s; };   // 2
-  auto bar_pd_full = [&](uint32_t s) { return b0 + 96 + 8 * s; };   // 2
+  auto bar_q_full = [&](uint32_t s) { return b0 + 16 + 8 * s; };
+  auto bar_q_empty = [&](uint32_t s) { return b0 + 32 + 8 * s; };
+  auto bar_o_full = [&](uint32_t s) { return b0 + 48 + 8 * s; };
+  auto bar_o_empty = [&](uint32_t s) { return b0 + 64 + 8 * s; };
+  const uint32_t bar_s_full = b0 + 80, bar_p_ready = b0 + 88, bar_dp_full = b0 + 96, bar_ds_ready = b0 + 104;
   const uint32_t bar_acc_full = b0 + 112, bar_acc_free = b0 + 120, bar_drain = b0 + 128;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -95,20 +102,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_kv_full, 1);
     ptx::mbar_init(bar_kv_empty, 1);
-    for (uint32_t i = 0; i < kStages; ++i) {
-      ptx::mbar_init(bar_st_full(i), 1);
-      ptx::mbar_init(bar_st_empty(i), 1);
+    for (uint32_t i = 0; i < kSlots; ++i) {
+      ptx::mbar_init(bar_q_full(i), 1);
+      ptx::mbar_init(bar_q_empty(i), 1);
+      ptx::mbar_init(bar_o_full(i), 1);
+      ptx::mbar_init(bar_o_empty(i), 1);
     }
-    for (uint32_t i = 0; i < 2; ++i) {
-      ptx::mbar_init(bar_sd_full(i), 1);
-      ptx::mbar_init(bar_pd_full(i), 128);
-    }
+    ptx::mbar_init(bar_s_full, 1);
+    ptx::mbar_init(bar_p_ready, 256);
+    ptx::mbar_init(bar_dp_full, 1);
+    ptx::mbar_init(bar_ds_ready, 256);
     ptx::mbar_init(bar_acc_full, 1);
-    ptx::mbar_init(bar_acc_free, 128);
+    ptx::mbar_init(bar_acc_free, 256);
     ptx::mbar_init(bar_drain, 1);
     for (uint32_t i = 0; i < ptx::kItemSlots; ++i) {
       ptx::mbar_init(ring.full + 8 * i, 1);
-      ptx::mbar_init(ring.empty + 8 * i, 129);  // MMA issuer + 128 gradient threads
+      ptx::mbar_init(ring.empty + 8 * i, 257);  // MMA issuer + 256 gradient threads
     }
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -133,8 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t kv_phase = 0, st = 0, st_phase = 0;
-      uint32_t pend_mask = 0, pend_par = 0, kv_fills = 0;
+      uint32_t kv_phase = 0, qs = 0, qph = 0, os = 0, oph = 0;
+      // fills that may still be in flight when an abort drains the CTA
+      uint32_t qpend = 0, qpar = 0, opend = 0, opar = 0, kv_fills = 0;
       bool ok = true;
       for (uint32_t rn = 0; ok; ++rn) {
         const int item = static_cast<int>(atomicAdd(a.counter, 1u));
@@ -145,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int g = code % a.Hkv;
         if (!ptx::mbar_wait(bar_kv_empty, kv_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 0, 1))) { ok = false; break; }
         kv_phase ^= 1u;
-        ptx::mbar_expect_tx(bar_kv_full, 2u * L::kKVBytes);
+        ptx::mbar_expect_tx(bar_kv_full, 2u * L::kTile);
         ++kv_fills;
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb) {
@@ -154,45 +164,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int ti = 0; ti < it.t_count && ok; ++ti) {
           const TileDesc td = a.tiles[it.t_first + it.t_count - 1 - ti];
-          const int nh = (td.n_rows + kHalf - 1) / kHalf;
-          for (int hh = 0; hh < G && ok; ++hh) {
+          for (int hh = 0; hh < G; ++hh) {
             const int h = g * G + hh;
-            for (int half = 0; half < nh; ++half) {
-              if (!ptx::mbar_wait(bar_st_empty(st), st_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 0, 2))) { ok = false; break; }
-              const uint32_t sb = sbase + L::kStage0 + st * L::kStageBytes;
-              const int slot0 = td.row_base + half * kHalf;
-              ptx::mbar_expect_tx(bar_st_full(st), L::kStageTx);
+            if (!ptx::mbar_wait(bar_q_empty(qs), qph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 0, 2))) { ok = false; break; }
+            const uint32_t sq = sbase + L::kQ0 + qs * L::kQSlot;
+            ptx::mbar_expect_tx(bar_q_full(qs), L::kTile + L::kMeta);
 #pragma unroll
-              for (int cb = 0; cb < D / 64; ++cb) {
-                ptx::tma_load_2d(sb + L::kSQ + cb * 8192u, &tmQ, bar_st_full(st), h * D + cb * 64, slot0);
-                ptx::tma_load_2d(sb + L::kSDO + cb * 8192u, &tmDO, bar_st_full(st), h * D + cb * 64, slot0);
-              }
-              bulk_load(sb + L::kSL, a.ls + int64_t(h) * a.n_slots + slot0, kHalf * 4u, bar_st_full(st));
-              bulk_load(sb + L::kSD, a.ds + int64_t(h) * a.n_slots + slot0, kHalf * 4u, bar_st_full(st));
-              bulk_load(sb + L::kSM, a.meta + slot0, kHalf * 16u, bar_st_full(st));
-              pend_mask |= 1u << st;
-              pend_par = (pend_par & ~(1u << st)) | (st_phase << st);
-              if (++st == kStages) { st = 0; st_phase ^= 1u; }
-            }
+            for (int cb = 0; cb < D / 64; ++cb)
+              ptx::tma_load_2d(sq + cb * 16384u, &tmQ, bar_q_full(qs), h * D + cb * 64, td.row_base);
+            bulk_load(sq + L::kSL, a.ls + int64_t(h) * a.n_slots + td.row_base, 512u, bar_q_full(qs));
+            bulk_load(sq + L::kSD, a.ds + int64_t(h) * a.n_slots + td.row_base, 512u, bar_q_full(qs));
+            bulk_load(sq + L::kSLim, a.lims + td.row_base, 512u, bar_q_full(qs));
+            qpend |= 1u << qs;
+            qpar = (qpar & ~(1u << qs)) | (qph << qs);
+            if (++qs == kSlots) { qs = 0; qph ^= 1u; }
+            if (!ptx::mbar_wait(bar_o_empty(os), oph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 0, 3))) { ok = false; break; }
+            const uint32_t so = sbase + L::kO0 + os * L::kTile;
+            ptx::mbar_expect_tx(bar_o_full(os), L::kTile);
+#pragma unroll
+            for (int cb = 0; cb < D / 64; ++cb)
+              ptx::tma_load_2d(so + cb * 16384u, &tmDO, bar_o_full(os), h * D + cb * 64, td.row_base);
+            opend |= 1u << os;
+            opar = (opar & ~(1u << os)) | (oph << os);
+            if (++os == kSlots) { os = 0; oph ^= 1u; }
           }
         }
       }
       if (*abort_flag) {
         volatile int never = 0;
-        for (int i = 0; i < kStages; ++i)
-          if (pend_mask & (1u << i))
-            ptx::mbar_wait(bar_st_full(i), (pend_par >> i) & 1u, &never, a.err, lim / 8);
+        for (uint32_t i = 0; i < kSlots; ++i) {
+          if (qpend & (1u << i)) ptx::mbar_wait(bar_q_full(i), (qpar >> i) & 1u, &never, a.err, lim / 8);
+          if (opend & (1u << i)) ptx::mbar_wait(bar_o_full(i), (opar >> i) & 1u, &never, a.err, lim / 8);
+        }
         if (kv_fills) ptx::mbar_wait(bar_kv_full, (kv_fills - 1) & 1u, &never, a.err, lim / 8);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, kHalf, false, false);
+      constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdG = ptx::idesc_bf16_f32(128, D, false, true);
-      uint32_t kv_phase = 0, st = 0, st_phase = 0, pd_phase = 0, acc_phase = 0, sd_cnt = 0;
+      uint32_t kv_phase = 0, qs = 0, qph = 0, os = 0, oph = 0, acc_phase = 0, sub = 0;
       bool ok = true;
-      const uint32_t sK = sbase + L::kK, sV = sbase + L::kV;
+      const uint64_t kd0 = ptx::sdesc_sw128(sbase + L::kK, 16u, 1024u);
+      const uint64_t vd0 = ptx::sdesc_sw128(sbase + L::kV, 16u, 1024u);
       for (uint32_t rn = 0; ok; ++rn) {
         int item = 0;
         if (!ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(3, 1, 14))) { ok = false; break; }
@@ -201,74 +216,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ptx::mbar_wait(bar_kv_full, kv_phase, abort_flag, a.err, lim, ptx::wait_site(3, 1, 3))) { ok = false; break; }
         kv_phase ^= 1u;
         ptx::tc_fence_after();
-        bool first_grad = true;
-        uint32_t prev_st = 0, prev_b = 0;
-        bool have_prev = false;
-        auto issue_grad = [&](uint32_t stg, uint32_t pb) -> bool {
-          // pd_phase bit pb: parity of buffer pb's next P^T / dS^T hand-over
-          if (!ptx::mbar_wait(bar_pd_full(pb), (pd_phase >> pb) & 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 4))) return false;
-          pd_phase ^= 1u << pb;
-          if (first_grad) {  // the previous item's epilogue has read dK / dV
-            if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 5))) return false;
-            acc_phase ^= 1u;
-          }
+        bool first_dv = true, first_dk = true, have_prev = false;
+        uint32_t prev_qs = 0;
+        // dK += dS^T Q for the previous sub-tile (its dS^T in DB, its Q in slot qslot)
+        auto issue_dk = [&](uint32_t qslot) -> bool {
+          if (!ptx::mbar_wait(bar_ds_ready, (sub - 1u) & 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 4))) return false;
           ptx::tc_fence_after();
-          const uint32_t sb = sbase + L::kStage0 + stg * L::kStageBytes;
-          const uint64_t od0 = ptx::sdesc_sw128(sb + L::kSDO, 8192u, 1024u);
-          const uint64_t qd0 = ptx::sdesc_sw128(sb + L::kSQ, 8192u, 1024u);
-          const uint32_t pt = tmem + kColS + pb * kHalf, dst = tmem + kColDP + pb * kHalf;
+          const uint64_t qd0 = ptx::sdesc_sw128(sbase + L::kQ0 + qslot * L::kQSlot, 16384u, 1024u);
 #pragma unroll
-          for (int kk = 0; kk < kHalf / 16; ++kk) {
-            const uint32_t acc = (!first_grad || kk > 0) ? 1u : 0u;
-            ptx::umma_ts(tmem + kColDV, pt + kk * 8u, ptx::sdesc_add(od0, kk * 2048u), kIdG, acc);
-            ptx::umma_ts(tmem + kColDK, dst + kk * 8u, ptx::sdesc_add(qd0, kk * 2048u), kIdG, acc);
-          }
-          first_grad = false;
-          ptx::umma_commit(bar_st_empty(stg));
+          for (int kk = 0; kk < 8; ++kk)
+            ptx::umma_ts(tmem + kColDK, tmem + kColDP + (kk >> 2) * 64u + (kk & 3) * 8u,
+                         ptx::sdesc_add(qd0, kk * 2048u), kIdG, (!first_dk || kk > 0) ? 1u : 0u);
+          first_dk = false;
+          ptx::umma_commit(bar_q_empty(qslot));
           return true;
         };
         for (int ti = 0; ti < it.t_count && ok; ++ti) {
-          const TileDesc td = a.tiles[it.t_first + it.t_count - 1 - ti];
-          const int nh = (td.n_rows + kHalf - 1) / kHalf;
-          for (int hh = 0; hh < G && ok; ++hh) {
-            for (int half = 0; half < nh; ++half) {
-              if (!ptx::mbar_wait(bar_st_full(st), st_phase, abort_flag, a.err, lim, ptx::wait_site(3, 1, 6))) { ok = false; break; }
-              // buffer b last held sub-tile sd_cnt - 2, whose gradient MMAs were issued above
-              const uint32_t b = sd_cnt & 1u;
-              ptx::tc_fence_after();
-              const uint32_t sb = sbase + L::kStage0 + st * L::kStageBytes;
-              const uint64_t kd0 = ptx::sdesc_sw128(sK, 16u, 1024u);
-              const uint64_t vd0 = ptx::sdesc_sw128(sV, 16u, 1024u);
-              const uint64_t qd0 = ptx::sdesc_sw128(sb + L::kSQ, 16u, 1024u);
-              const uint64_t od0 = ptx::sdesc_sw128(sb + L::kSDO, 16u, 1024u);
+          for (int hh = 0; hh < G; ++hh) {
+            // S^T_i = K Q_i^T -> SB (SB's last reader, dV_{i-1}, was issued before)
+            if (!ptx::mbar_wait(bar_q_full(qs), qph, abort_flag, a.err, lim, ptx::wait_site(3, 1, 5))) { ok = false; break; }
+            ptx::tc_fence_after();
+            const uint64_t qd0 = ptx::sdesc_sw128(sbase + L::kQ0 + qs * L::kQSlot, 16u, 1024u);
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t offA = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                const uint32_t offB = (kk >> 2) * 8192u + (kk & 3) * 32u;
-                ptx::umma_ss(tmem + kColS + b * kHalf, ptx::sdesc_add(kd0, offA), ptx::sdesc_add(qd0, offB),
-                             kIdS, kk > 0 ? 1u : 0u);
-              }
-#pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t offA = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                const uint32_t offB = (kk >> 2) * 8192u + (kk & 3) * 32u;
-                ptx::umma_ss(tmem + kColDP + b * kHalf, ptx::sdesc_add(vd0, offA), ptx::sdesc_add(od0, offB),
-                             kIdS, kk > 0 ? 1u : 0u);
-              }
-              ptx::umma_commit(bar_sd_full(b));
-              ++sd_cnt;
-              if (have_prev && !issue_grad(prev_st, prev_b)) { ok = false; break; }
-              prev_st = st;
-              prev_b = b;
-              have_prev = true;
-              if (++st == kStages) { st = 0; st_phase ^= 1u; }
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+              ptx::umma_ss(tmem + kColS, ptx::sdesc_add(kd0, off), ptx::sdesc_add(qd0, off), kIdS, kk > 0 ? 1u : 0u);
             }
+            ptx::umma_commit(bar_s_full);
+            if (have_prev && !issue_dk(prev_qs)) { ok = false; break; }
+            // dP^T_i = V dO_i^T -> DB (DB's last reader, dK_{i-1}, was issued just above)
+            if (!ptx::mbar_wait(bar_o_full(os), oph, abort_flag, a.err, lim, ptx::wait_site(3, 1, 6))) { ok = false; break; }
+            ptx::tc_fence_after();
+            const uint32_t so = sbase + L::kO0 + os * L::kTile;
+            const uint64_t od0 = ptx::sdesc_sw128(so, 16u, 1024u);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+              ptx::umma_ss(tmem + kColDP, ptx::sdesc_add(vd0, off), ptx::sdesc_add(od0, off), kIdS, kk > 0 ? 1u : 0u);
+            }
+            ptx::umma_commit(bar_dp_full);
+            // dV += P^T_i dO_i once the threads have written P^T_i
+            if (!ptx::mbar_wait(bar_p_ready, sub & 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 7))) { ok = false; break; }
+            if (first_dv) {  // the previous item's epilogue has read dK / dV
+              if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 8))) { ok = false; break; }
+              acc_phase ^= 1u;
+            }
+            ptx::tc_fence_after();
+            const uint64_t ogd0 = ptx::sdesc_sw128(so, 16384u, 1024u);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              ptx::umma_ts(tmem + kColDV, tmem + kColS + (kk >> 2) * 64u + (kk & 3) * 8u,
+                           ptx::sdesc_add(ogd0, kk * 2048u), kIdG, (!first_dv || kk > 0) ? 1u : 0u);
+            first_dv = false;
+            ptx::umma_commit(bar_o_empty(os));
+            prev_qs = qs;
+            have_prev = true;
+            ++sub;
+            if (++qs == kSlots) { qs = 0; qph ^= 1u; }
+            if (++os == kSlots) { os = 0; oph ^= 1u; }
           }
         }
         if (!ok) break;
-        if (have_prev && !issue_grad(prev_st, prev_b)) { ok = false; break; }
-        if (first_grad) {  // no gradient MMA in this item: still pair the epilogue handshake
-          if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 8))) { ok = false; break; }
+        if (have_prev && !issue_dk(prev_qs)) { ok = false; break; }
+        if (first_dv) {  // no sub-tile in this item: still pair the epilogue handshake
+          if (!ptx::mbar_wait(bar_acc_free, acc_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(3, 1, 9))) { ok = false; break; }
           acc_phase ^= 1u;
         }
         ptx::umma_commit(bar_kv_empty);
@@ -281,10 +292,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ P^T, dS^T / epilogue
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;  // key row within the tile
+    const int wg = (warp - 2) >> 2;        // which 64 query rows of a sub-tile
+    const int row = quarter * 32 + lane;   // key row within the tile
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t half_col = static_cast<uint32_t>(wg) * 64u;
     const float sl2 = a.scale_log2;
-    uint32_t st = 0, st_phase = 0, sd_cnt = 0, acc_cnt = 0;
+    uint32_t qs = 0, qph = 0, sub = 0, acc_cnt = 0;
     bool ok = true;
     for (uint32_t rn = 0; ok; ++rn) {
       int item = 0;
@@ -300,91 +313,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int warp_last_key = it.key0 + quarter * 32 + 31;
       bool any = false;
       for (int ti = 0; ti < it.t_count && ok; ++ti) {
-        const TileDesc td = a.tiles[it.t_first + it.t_count - 1 - ti];
-        const int nh = (td.n_rows + kHalf - 1) / kHalf;
-        for (int hh = 0; hh < G && ok; ++hh) {
-          for (int half = 0; half < nh; ++half) {
-            const uint32_t b = sd_cnt & 1u;
-            const uint32_t bph = (sd_cnt >> 1) & 1u;
-            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_sd_full(b), bph, abort_flag, a.err, lim, ptx::wait_site(3, 2, 9)))) {
-              ok = false;
-              break;
-            }
-            ++sd_cnt;
-            ptx::tc_fence_after();
-            uint32_t sv[2][32], pv[2][32];
-            ptx::tmem_ld32(tl + kColS + b * kHalf, sv[0]);
-            ptx::tmem_ld32(tl + kColS + b * kHalf + 32u, sv[1]);
-            ptx::tmem_ld32(tl + kColDP + b * kHalf, pv[0]);
-            ptx::tmem_ld32(tl + kColDP + b * kHalf + 32u, pv[1]);
-            ptx::tmem_wait_ld();
-            // the stage's L, D and metadata landed (TMA completion, seen by this thread)
-            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_st_full(st), st_phase, abort_flag, a.err, lim, ptx::wait_site(3, 2, 12)))) {
-              ok = false;
-              break;
-            }
-            const uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
-            const float4* L4 = reinterpret_cast<const float4*>(sb + L::kSL);  // -L * log2(e)
-            const float4* D4 = reinterpret_cast<const float4*>(sb + L::kSD);
-            const SlotMeta* Ms = reinterpret_cast<const SlotMeta*>(sb + L::kSM);
-            // exponent arguments S^T * scale*log2(e) - L*log2(e), two rows per instruction
-            const float2 c2 = make_float2(sl2, sl2);
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const float4 l = L4[q];
-              const int c = q >> 3, i = (q & 7) * 4;
-              const float2 x0 = ptx::fma2(make_float2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])), c2,
-                                          make_float2(l.x, l.y));
-              const float2 x1 = ptx::fma2(make_float2(__uint_as_float(sv[c][i + 2]), __uint_as_float(sv[c][i + 3])), c2,
-                                          make_float2(l.z, l.w));
-              sv[c][i] = __float_as_uint(x0.x);
-              sv[c][i + 1] = __float_as_uint(x0.y);
-              sv[c][i + 2] = __float_as_uint(x1.x);
-              sv[c][i + 3] = __float_as_uint(x1.y);
-            }
-            // The half's rows are sorted by limit (padding, limit -1, only at a tile's end), so
-            // when the warp's last key is visible to the first row, every pair is visible.
-            if (!(warp_last_key <= Ms[0].limit)) {
-#pragma unroll
-              for (int col = 0; col < 64; ++col)
-                if (kp > Ms[col].limit) sv[col >> 5][col & 31] = __float_as_uint(-INFINITY);
-            }
-            // P^T and dS^T = P^T (dP^T - D) of this key row over the 64 query rows
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const float4 dd = D4[q];
-              const int c = q >> 3, i = (q & 7) * 4;
-              const float2 p0 = make_float2(ptx::ex2(__uint_as_float(sv[c][i])), ptx::ex2(__uint_as_float(sv[c][i + 1])));
-              const float2 p1 = make_float2(ptx::ex2(__uint_as_float(sv[c][i + 2])), ptx::ex2(__uint_as_float(sv[c][i + 3])));
-              const float2 g0 = ptx::mul2(p0, ptx::sub2(make_float2(__uint_as_float(pv[c][i]), __uint_as_float(pv[c][i + 1])),
-                                                       make_float2(dd.x, dd.y)));
-              const float2 g1 = ptx::mul2(p1, ptx::sub2(make_float2(__uint_as_float(pv[c][i + 2]), __uint_as_float(pv[c][i + 3])),
-                                                       make_float2(dd.z, dd.w)));
-              sv[c][i] = __float_as_uint(p0.x);
-              sv[c][i + 1] = __float_as_uint(p0.y);
-              sv[c][i + 2] = __float_as_uint(p1.x);
-              sv[c][i + 3] = __float_as_uint(p1.y);
-              pv[c][i] = __float_as_uint(g0.x);
-              pv[c][i + 1] = __float_as_uint(g0.y);
-              pv[c][i + 2] = __float_as_uint(g1.x);
-              pv[c][i + 3] = __float_as_uint(g1.y);
-            }
-            // bf16 pairs (lower row in the low half) over S^T's / dP^T's first 32 columns
-            uint32_t pk[32], dk[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int c = j >> 4, i = (j & 15) * 2;
-              pk[j] = ptx::pack_bf16x2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
-              dk[j] = ptx::pack_bf16x2(__uint_as_float(pv[c][i]), __uint_as_float(pv[c][i + 1]));
-            }
-            ptx::tmem_st32(tl + kColS + b * kHalf, pk);
-            ptx::tmem_st32(tl + kColDP + b * kHalf, dk);
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(bar_pd_full(b));
-            any = true;
-            if (++st == kStages) { st = 0; st_phase ^= 1u; }
+        for (int hh = 0; hh < G; ++hh) {
+          // The slot's L, D and limits landed (TMA completion, seen by this thread);
+          // usually long before S^T_i, so this wait costs nothing on the critical path.
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_q_full(qs), qph, abort_flag, a.err, lim, ptx::wait_site(3, 2, 12)))) {
+            ok = false;
+            break;
           }
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_s_full, sub & 1u, abort_flag, a.err, lim, ptx::wait_site(3, 2, 9)))) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          uint32_t sv[2][32];
+          ptx::tmem_ld32(tl + kColS + half_col, sv[0]);
+          ptx::tmem_ld32(tl + kColS + half_col + 32u, sv[1]);
+          ptx::tmem_wait_ld();
+          const uint8_t* sq = smem + L::kQ0 + qs * L::kQSlot;
+          const float4* L4 = reinterpret_cast<const float4*>(sq + L::kSL) + wg * 16;  // -L * log2(e)
+          const float4* D4 = reinterpret_cast<const float4*>(sq + L::kSD) + wg * 16;
+          const int* Lim = reinterpret_cast<const int*>(sq + L::kSLim) + wg * 64;
+          // exponent arguments S^T * scale*log2(e) - L*log2(e), two rows per instruction
+          const float2 c2 = make_float2(sl2, sl2);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float4 l = L4[q];
+            const int c = q >> 3, i = (q & 7) * 4;
+            const float2 x0 = ptx::fma2(make_float2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])), c2,
+                                        make_float2(l.x, l.y));
+            const float2 x1 = ptx::fma2(make_float2(__uint_as_float(sv[c][i + 2]), __uint_as_float(sv[c][i + 3])), c2,
+                                        make_float2(l.z, l.w));
+            sv[c][i] = __float_as_uint(x0.x);
+            sv[c][i + 1] = __float_as_uint(x0.y);
+            sv[c][i + 2] = __float_as_uint(x1.x);
+            sv[c][i + 3] = __float_as_uint(x1.y);
+          }
+          // The rows are sorted by limit (padding, limit -1, only at a tile's end), so when
+          // the warp's last key is visible to this warpgroup's first row, every pair is.
+          if (!(warp_last_key <= Lim[0])) {
+#pragma unroll
+            for (int col = 0; col < 64; ++col)
+              if (kp > Lim[col]) sv[col >> 5][col & 31] = __float_as_uint(-INFINITY);
+          }
+          uint32_t pk[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int c = j >> 4, i = (j & 15) * 2;
+            // every other pair on the FMA pipe, the rest on the special-function unit
+            const float2 xx = make_float2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
+            const float2 pp = (j & 1) ? ptx::exp2_poly(xx) : ptx::exp2_sfu(xx);
+            sv[c][i] = __float_as_uint(pp.x);
+            sv[c][i + 1] = __float_as_uint(pp.y);
+            pk[j] = ptx::pack_bf16x2(pp.x, pp.y);  // lower row in the low half
+          }
+          ptx::tmem_st32(tl + kColS + half_col, pk);
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar_p_ready);
+          // dS^T = P^T (dP^T - D)
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_dp_full, sub & 1u, abort_flag, a.err, lim, ptx::wait_site(3, 2, 10)))) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          uint32_t pv[2][32];
+          ptx::tmem_ld32(tl + kColDP + half_col, pv[0]);
+          ptx::tmem_ld32(tl + kColDP + half_col + 32u, pv[1]);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float4 dd = D4[q];
+            const int c = q >> 3, i = (q & 7) * 4;
+            const float2 g0 = ptx::mul2(make_float2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])),
+                                        ptx::sub2(make_float2(__uint_as_float(pv[c][i]), __uint_as_float(pv[c][i + 1])),
+                                                  make_float2(dd.x, dd.y)));
+            const float2 g1 = ptx::mul2(make_float2(__uint_as_float(sv[c][i + 2]), __uint_as_float(sv[c][i + 3])),
+                                        ptx::sub2(make_float2(__uint_as_float(pv[c][i + 2]), __uint_as_float(pv[c][i + 3])),
+                                                  make_float2(dd.z, dd.w)));
+            pk[q * 2] = ptx::pack_bf16x2(g0.x, g0.y);
+            pk[q * 2 + 1] = ptx::pack_bf16x2(g1.x, g1.y);
+          }
+          ptx::tmem_st32(tl + kColDP + half_col, pk);
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar_ds_ready);
+          any = true;
+          ++sub;
+          if (++qs == kSlots) { qs = 0; qph ^= 1u; }
         }
       }
       if (!ok) break;
@@ -397,22 +412,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
       const bool own = kp < it.key_end && any;
       const bool zero = kp < it.key_end && !any;
+      // each warpgroup writes half of the D columns of dK and of dV
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         __nv_bfloat16* out = which == 0 ? a.dk : a.dv;
         const float mul = which == 0 ? a.scale : 1.f;
-        const uint32_t col0 = which == 0 ? kColDK : kColDV;
+        const uint32_t col0 = (which == 0 ? kColDK : kColDV) + static_cast<uint32_t>(wg) * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t v[32];
           ptx::tmem_ld32(tl + col0 + c * 32u, v);
           ptx::tmem_wait_ld();
           if (own || zero) {
-            __nv_bfloat16* dst = out + (int64_t(kp) * a.Hkv + g) * D + c * 32;
+            __nv_bfloat16* dst = out + (int64_t(kp) * a.Hkv + g) * D + wg * (D / 2) + c * 32;
+            const float z = zero ? 0.f : mul;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               uint4 wv;
-              const float z = zero ? 0.f : mul;
               wv.x = ptx::pack_bf16x2(__uint_as_float(v[q4 * 8 + 0]) * z, __uint_as_float(v[q4 * 8 + 1]) * z);
               wv.y = ptx::pack_bf16x2(__uint_as_float(v[q4 * 8 + 2]) * z, __uint_as_float(v[q4 * 8 + 3]) * z);
               wv.z = ptx::pack_bf16x2(__uint_as_float(v[q4 * 8 + 4]) * z, __uint_as_float(v[q4 * 8 + 5]) * z);

@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-              const float2 p = make_float2(ptx::ex2(__uint_as_float(sr[i])), ptx::ex2(__uint_as_float(sr[i + 1])));
+              const float2 p = ptx::exp2_sfu(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])));
               const float2 g = ptx::mul2(p, ptx::sub2(make_float2(__uint_as_float(dp[c][i]), __uint_as_float(dp[c][i + 1])), d2));
               pk[cc * 16 + (i >> 1)] = ptx::pack_bf16x2(g.x, g.y);
             }

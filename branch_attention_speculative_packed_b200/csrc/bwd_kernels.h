@@ -23,6 +23,7 @@ struct PrepArgs {
   float* ds;                 // [Hq, n_slots]
   float* drow;               // [Hq, rows]
   SlotMeta* meta;            // [n_slots]
+  int32_t* lims;             // [n_slots], meta[].limit on its own (-1 for padding)
 };
 cudaError_t launch_bwd_prep(const PrepArgs& a, int d, cudaStream_t st);
 
@@ -67,7 +68,7 @@ struct DkdvArgs {
   const KvItem* items;
   const int32_t* order;
   const TileDesc* tiles;
-  const SlotMeta* meta;
+  const int32_t* lims;  // [n_slots]: a row sees main keys <= its limit
   const float* ls;  // [Hq, n_slots], -LSE * log2(e)
   const float* ds;  // [Hq, n_slots]
   int Hq, Hkv, G, d;
@@ -81,7 +82,7 @@ struct DkdvArgs {
 };
 struct DkdvMaps {
   CUtensorMap k, v;      // [S, Hkv*d], box 64 x 128
-  CUtensorMap qg, dog;   // [n_slots, Hq*d], box 64 x 64
+  CUtensorMap qg, dog;   // [n_slots, Hq*d], box 64 x 128
 };
 cudaError_t launch_bwd_dkdv(const DkdvMaps& m, const DkdvArgs& a, int num_sms, cudaStream_t st);
 

@@ -418,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const float2 x = ptx::fma2(make_float2(__uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1])), c2, nm2);
-            const float2 p = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+            const float2 p = ptx::exp2_sfu(x);
             rs4[(i >> 1) & 3] = ptx::add2(rs4[(i >> 1) & 3], p);
             sr[c][i] = __float_as_uint(p.x);
             sr[c][i + 1] = __float_as_uint(p.y);

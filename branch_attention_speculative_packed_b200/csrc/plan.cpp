@@ -278,6 +278,8 @@ WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int whic
     off = align_up(off + slots * p->Hq * sizeof(float), 256);
     w.meta_off = off;
     off = align_up(off + slots * sizeof(SlotMeta), 256);
+    w.lims_off = off;
+    off = align_up(off + slots * sizeof(int32_t), 256);
     w.drow_off = off;
     off = align_up(off + rows * p->Hq * sizeof(float), 256);
   }

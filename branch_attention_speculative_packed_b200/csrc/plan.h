@@ -65,6 +65,7 @@ struct WorkspaceLayout {
   size_t qg_off = 0, dog_off = 0;    // Q and dO gathered into slot order, bf16 [slots, Hq, d]
   size_t ls_off = 0, ds_off = 0;     // log2-scaled LSE and D = rowsum(dO*O), fp32 [Hq, slots]
   size_t meta_off = 0;               // SlotMeta [slots]
+  size_t lims_off = 0;               // main-key limit per slot, int32 [slots]
   size_t drow_off = 0;               // D in row order, fp32 [Hq, rows]
   size_t total = 0;
   int64_t n_slots = 0;               // row-table entries (ntiles * 128)
