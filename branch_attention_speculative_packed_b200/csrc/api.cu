@@ -131,6 +131,8 @@ ba_status stage_plan(const ba_problem* p, const Plan& plan, const WorkspaceLayou
                       cudaMemcpyHostToDevice, st) != cudaSuccess ||
       cudaMemcpyAsync(ws + w.order_off, plan.order.data(), nt * sizeof(int32_t),
                       cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(ws + w.pairs_off, plan.pairs.data(), plan.pairs.size() * sizeof(int32_t),
+                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
       cudaMemcpyAsync(ws + w.chunks_off, plan.chunks_dev.data(),
                       plan.chunks_dev.size() * sizeof(ChunkDev), cudaMemcpyHostToDevice,
                       st) != cudaSuccess ||
@@ -193,7 +195,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   a.anchors = p->anchors_d;
   a.row_table = reinterpret_cast<const int32_t*>(ws + w.rows_off);
   a.tiles = reinterpret_cast<const TileDesc*>(ws + w.tiles_off);
-  a.order = reinterpret_cast<const int32_t*>(ws + w.order_off);
+  a.pairs = reinterpret_cast<const int32_t*>(ws + w.pairs_off);
   a.S = p->S;
   a.Nb = p->Nb;
   a.B = plan.B > 0 ? plan.B : 1;
@@ -201,7 +203,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   a.Hq = p->Hq;
   a.G = p->Hq / p->Hkv;
   a.d = p->d;
-  const int64_t items = int64_t(plan.tiles.size()) * p->Hq;
+  const int64_t items = int64_t(plan.pairs.size() / 2) * p->Hq;
   if (items > 0x7fffffff) return BA_ERR_UNSUPPORTED;
   a.n_items = static_cast<int>(items);
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;

@@ -1,38 +1,43 @@
 // Branch-attention forward on sm_100a: tcgen05 MMA with TMEM accumulators,
-// TMA-staged tiles, warp-specialised pipeline.
+// TMA-staged tiles, warp-specialised pipeline over two query tiles.
 //
 // Paper: arXiv 2609.07108 §3.2 / Eq. 2 (rcap.io post, branch-attention
 // paragraph; cere-bro wiki, "Obstacle one, context parallelism").  One
-// persistent CTA per SM walks (row tile, query head) work items, longest
-// first.  For each item it streams the item's main key tiles (the causal
-// prefix [doc start, largest limit]) and, in the fused variant, the key tiles
-// of the branch-local keys, through one online softmax.  Visiting key tiles
+// persistent CTA per SM walks (tile pair, query head) work items, longest
+// first.  A pair is two consecutive row tiles A and B of one document; they
+// share the document's main key tiles, so one K/V stream serves both: the
+// main key tiles [doc start, larger limit] (each tile takes those up to its
+// own limit), then A's branch-local key tiles, then B's.  Visiting key tiles
 // one after another with a running (max, sum) is the same log-sum-exp merge
 // ring attention applies between ring steps (Eq. 2), so the main-sequence
 // component, the branch-local component and their merge all happen here.
 //
-// Roles (192 threads):
-//   warp 0      producer: claims work items (one item ahead of the consumers)
-//               and streams the K/V key tiles through a 3-stage TMA ring.
-//   warp 1      TMEM allocator and single-thread MMA issuer:
-//               S[sb] = Q K^T into one of two TMEM buffers, then O += P V
-//               with P read from TMEM (A operand in tensor memory).
-//   warps 2-5   softmax / epilogue, one query row per thread.  Each thread
-//               copies its own query row into shared memory (cp.async): the
-//               next item's rows go in as soon as the current item's last
-//               S MMA, the only reader of Q, has finished, so the copy
-//               overlaps the last softmax step and the epilogue.  Per key
-//               tile: load S from
-//               TMEM, mask by the row's key range, update the running max
-//               (lazily: O in TMEM is rescaled only when the max grows by
-//               more than 2^8), write P (bf16) into one of two TMEM buffers
-//               for the P.V MMA, and finally normalise O and write O and LSE.
+// Per tile t in {A, B} and key tile j:
+//   S_t = Q_t K_j^T                   -> TMEM buffer S_t
+//   softmax warpgroup t: P = exp2(S * scale*log2e - m), bf16, written over
+//       the first 64 columns of S_t
+//   O_t += P V_j   (P read from TMEM) -> TMEM accumulator O_t
+// The tensor pipe runs, in issue order, ... PV_A(j), S_A(j+1), PV_B(j),
+// S_B(j+1) ...: S_t(j+1) overwrites S_t only after PV_t(j) has read P, and
+// while one warpgroup computes its softmax the pipe works on the other tile.
 //
-// Shared memory (D = head dim): Q [128 x D] | 3 x (K [128 x D], V [128 x D]),
+// Roles (320 threads):
+//   warp 0      producer: claims work items (one item ahead of the consumers)
+//               and streams the K/V key tiles through a 2-stage TMA ring.
+//   warp 1      TMEM allocator and single-thread MMA issuer.
+//   warps 2-5   softmax / epilogue of tile A, warps 6-9 of tile B, one query
+//               row per thread.  Each thread copies its own query row into
+//               shared memory (cp.async); the next item's row goes in as soon
+//               as the tile's last S MMA, the only reader of Q, has finished.
+//               Per key tile: load S, mask by the row's key range, update the
+//               running max (lazily: O is rescaled only when the max grows by
+//               more than 2^8), write P; finally normalise O, write O and LSE.
+//               A thread reads its S row twice, 32 columns at a time (once
+//               for the row max, once for P), rather than holding all of it.
+//
+// Shared memory (D = head dim): Q_A | Q_B [128 x D each] | 2 x (K, V [128 x D]),
 // bf16 in the 128-byte-swizzled layout (TMA writes K / V; the threads write Q
-// in the same pattern).
-// TMEM: S buffers at columns 0 and 128, O at 256, P buffers at 384 and 448
-// (128 rows x 128 bf16 keys = 64 columns each).
+// in the same pattern).  TMEM: S_A 0, S_B 128, O_A 256, O_B 384.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -42,33 +47,73 @@
 namespace ba {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kStages = 3;
+constexpr int kThreads = 320;
+constexpr int kWarpProducer = 0, kWarpMma = 1;  // warps 2-9: softmax
+constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColP = 384;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kColS = 0, kColO = 256;  // tile t: S at kColS + 128 t, O at kColO + 128 t
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 template <int D>
 struct Smem {
-  static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kTileBytes = 128u * D * 2u;  // one 128-row bf16 tile
-  static constexpr uint32_t kK0 = kQ + kTileBytes;
+  static constexpr uint32_t kQ0 = 0;                     // Q_A, then Q_B
+  static constexpr uint32_t kK0 = 2u * kTileBytes;
   static constexpr uint32_t kStageBytes = 2u * kTileBytes;  // K + V
   static constexpr uint32_t kBar = kK0 + kStages * kStageBytes;
-  // barriers: q_full, kv_full[3], kv_empty[3], s_full[2], s_empty[2], p_full[2], o_done[2],
-  // drain, item_full[4], item_empty[4]
-  static constexpr uint32_t kNumBars = 24;
+  // barriers: q_full[2], kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done[2], drain,
+  // item_full[4], item_empty[4]
+  static constexpr uint32_t kNumBars = 21;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base, abort, item slots[4]
   static constexpr uint32_t kTotal = kMisc + 32u;
   static constexpr uint32_t kAlloc = kTotal + 1024u;  // slack to align the base to 1024
 };
 
 struct Bars {
-  uint32_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full[2],
-      o_done[2], drain;
+  uint32_t q_full[2], kv_full[kStages], kv_empty[kStages], s_full[2], p_full[2], o_done[2], drain;
 };
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// The key-tile stream of a tile pair.
+struct PairPlan {
+  TileDesc t[2];
+  bool on[2];   // tile present (the second tile of a pair may be absent)
+  int nkv[2];   // main key tiles of each tile
+  int nbr[2];   // branch key tiles of each tile
+  int nmain;    // main key tiles streamed: max(nkv)
+  int n;        // key tiles streamed
+};
+
+__device__ __forceinline__ PairPlan load_pair(const FwdArgs& a, int pair) {
+  PairPlan pp;
+  const int2 ids = reinterpret_cast<const int2*>(a.pairs)[pair];
+  const int id[2] = {ids.x, ids.y};
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    pp.on[t] = id[t] >= 0;
+    pp.nkv[t] = pp.nbr[t] = 0;
+    if (pp.on[t]) {
+      pp.t[t] = a.tiles[id[t]];
+      pp.nkv[t] = ceil_div(pp.t[t].kv_end - pp.t[t].doc_start, 128);
+      if (a.with_branch && pp.t[t].br_hi > pp.t[t].br_lo)
+        pp.nbr[t] = ceil_div(pp.t[t].br_hi - pp.t[t].br_lo, 128);
+    } else {
+      pp.t[t] = pp.t[0];
+    }
+  }
+  pp.nmain = max(pp.nkv[0], pp.nkv[1]);
+  pp.n = pp.nmain + pp.nbr[0] + pp.nbr[1];
+  return pp;
+}
+
+// Does tile t take key tile j of the stream?
+__device__ __forceinline__ bool takes(const PairPlan& pp, int t, int j) {
+  if (!pp.on[t]) return false;
+  if (j < pp.nmain) return j < pp.nkv[t];
+  j -= pp.nmain;
+  return t == 0 ? j < pp.nbr[0] : j >= pp.nbr[0];
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -86,11 +131,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bars bar;
   {
     uint32_t b = sbase + L::kBar;
-    bar.q_full = b; b += 8;
+    for (int i = 0; i < 2; ++i) { bar.q_full[i] = b; b += 8; }
     for (int i = 0; i < kStages; ++i) { bar.kv_full[i] = b; b += 8; }
     for (int i = 0; i < kStages; ++i) { bar.kv_empty[i] = b; b += 8; }
     for (int i = 0; i < 2; ++i) { bar.s_full[i] = b; b += 8; }
-    for (int i = 0; i < 2; ++i) { bar.s_empty[i] = b; b += 8; }
     for (int i = 0; i < 2; ++i) { bar.p_full[i] = b; b += 8; }
     for (int i = 0; i < 2; ++i) { bar.o_done[i] = b; b += 8; }
     bar.drain = b;
@@ -103,34 +147,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   ring.empty = ring.full + 8 * ptx::kItemSlots;
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(bar.q_full, 128);  // one arrival per softmax thread (its copied row)
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar.q_full[i], 128);  // one arrival per softmax thread (its copied row)
+      ptx::mbar_init(bar.s_full[i], 1);
+      ptx::mbar_init(bar.p_full[i], 128);
+      ptx::mbar_init(bar.o_done[i], 1);
+    }
     for (int i = 0; i < kStages; ++i) {
       ptx::mbar_init(bar.kv_full[i], 1);
       ptx::mbar_init(bar.kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(bar.s_full[i], 1);
-      ptx::mbar_init(bar.s_empty[i], 128);
-    }
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(bar.p_full[i], 128);
-      ptx::mbar_init(bar.o_done[i], 1);
-    }
     ptx::mbar_init(bar.drain, 1);
     for (uint32_t i = 0; i < ptx::kItemSlots; ++i) {
       ptx::mbar_init(ring.full + 8 * i, 1);
-      ptx::mbar_init(ring.empty + 8 * i, 129);  // MMA issuer + 128 softmax threads
+      ptx::mbar_init(ring.empty + 8 * i, 257);  // MMA issuer + 256 softmax threads
     }
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kWarpProducer && lane == 0) {
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
     ptx::prefetch_tmap(&tmKb);
     ptx::prefetch_tmap(&tmVb);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     ptx::tmem_alloc(sbase + L::kMisc, kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -142,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int Hq = a.Hq;
   const long long lim = a.wait_limit;
 
-  if (warp == 0) {
+  if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t kv_stage = 0, kv_phase = 0;
@@ -155,11 +196,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t rn = 1; ok && cur < a.n_items; ++rn) {
         const int nxt = static_cast<int>(atomicAdd(a.counter, 1u));
         if (!ptx::ring_put(ring, rn, nxt, abort_flag, a.err, lim, ptx::wait_site(1, 0, 12))) { ok = false; break; }
-        const TileDesc td = a.tiles[a.order[cur / Hq]];
+        const PairPlan pp = load_pair(a, cur / Hq);
         const int g = (cur % Hq) / a.G;
-        const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
-        const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
-        for (int j = 0; j < nkv + nbr; ++j) {
+        for (int j = 0; j < pp.n; ++j) {
           if (!ptx::mbar_wait(bar.kv_empty[kv_stage], kv_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(1, 0, 2))) {
             ok = false;
             break;
@@ -168,10 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const void* mk = &tmK;
           const void* mv = &tmV;
           int y;
-          if (j < nkv) {
-            y = td.doc_start + 128 * j;
+          if (j < pp.nmain) {
+            y = pp.t[0].doc_start + 128 * j;
           } else {
-            y = td.br_lo + 128 * (j - nkv);
+            const int jb = j - pp.nmain;
+            y = jb < pp.nbr[0] ? pp.t[0].br_lo + 128 * jb : pp.t[1].br_lo + 128 * (jb - pp.nbr[0]);
             mk = &tmKb;
             mv = &tmVb;
           }
@@ -196,68 +236,77 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_wait(bar.kv_full[i], (pend_par >> i) & 1u, &never, a.err, lim / 8);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdPV = ptx::idesc_bf16_f32(128, D, false, true);
-      uint32_t kv_stage = 0, kv_phase = 0, q_phase = 0, s_cnt = 0, pv_cnt = 0;
+      uint32_t kv_stage = 0, kv_phase = 0;
+      uint32_t q_phase[2] = {0u, 0u};
+      uint32_t p_cnt[2] = {0u, 0u};  // P tiles consumed per tile slot (p_full parity)
       bool ok = true;
-      const uint32_t sQ = sbase + L::kQ;
-      // O += P V for key tile jj: P from TMEM buffer pv_cnt % 2, V from the stage.
-      auto issue_pv = [&](int jj, uint32_t stage) -> bool {
-        const uint32_t pb = pv_cnt & 1u;
-        if (!ptx::mbar_wait(bar.p_full[pb], (pv_cnt >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 1, 3))) return false;
-        ptx::tc_fence_after();
-        const uint32_t sv = sbase + L::kK0 + stage * L::kStageBytes + L::kTileBytes;
-        const uint64_t bd0 = ptx::sdesc_sw128(sv, 16384u, 1024u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = ptx::sdesc_add(bd0, kk * 2048u);
-          ptx::umma_ts(tmem + kColO, tmem + kColP + pb * 64u + kk * 8u, bd, kIdPV,
-                       (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        ptx::umma_commit(bar.o_done[pb]);
-        ptx::umma_commit(bar.kv_empty[stage]);
-        ++pv_cnt;
-        return true;
-      };
       for (uint32_t rn = 0; ok; ++rn) {
         int item = 0;
         if (!ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(1, 1, 13))) { ok = false; break; }
         if (item >= a.n_items) break;
-        const TileDesc td = a.tiles[a.order[item / Hq]];
-        const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
-        const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
-        const int n = nkv + nbr;
-        if (!ptx::mbar_wait(bar.q_full, q_phase, abort_flag, a.err, lim, ptx::wait_site(1, 1, 4))) { ok = false; break; }
-        q_phase ^= 1u;
-        ptx::tc_fence_after();
-        uint32_t prev_stage = 0;
-        for (int j = 0; j < n; ++j) {
-          if (!ptx::mbar_wait(bar.kv_full[kv_stage], kv_phase, abort_flag, a.err, lim, ptx::wait_site(1, 1, 5))) { ok = false; break; }
-          const uint32_t sb = s_cnt & 1u;
-          const uint32_t sph = (s_cnt >> 1) & 1u;
-          if (!ptx::mbar_wait(bar.s_empty[sb], sph ^ 1u, abort_flag, a.err, lim, ptx::wait_site(1, 1, 6))) { ok = false; break; }
-          ptx::tc_fence_after();
-          const uint32_t sk = sbase + L::kK0 + kv_stage * L::kStageBytes;
-          const uint64_t ad0 = ptx::sdesc_sw128(sQ, 16u, 1024u);
-          const uint64_t bd0 = ptx::sdesc_sw128(sk, 16u, 1024u);
+        const PairPlan pp = load_pair(a, item / Hq);
+        bool first_s[2] = {true, true}, first_pv[2] = {true, true};
+        // S_t(j) = Q_t K_j^T into tile t's S buffer (the P.V that last read it was issued before).
+        auto issue_s = [&](int t, uint32_t stage) -> bool {
+          if (first_s[t]) {  // this tile's query rows have been copied in
+            if (!ptx::mbar_wait(bar.q_full[t], q_phase[t], abort_flag, a.err, lim, ptx::wait_site(1, 1, 4))) return false;
+            q_phase[t] ^= 1u;
+            ptx::tc_fence_after();
+            first_s[t] = false;
+          }
+          const uint64_t ad0 = ptx::sdesc_sw128(sbase + L::kQ0 + t * L::kTileBytes, 16u, 1024u);
+          const uint64_t bd0 = ptx::sdesc_sw128(sbase + L::kK0 + stage * L::kStageBytes, 16u, 1024u);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-            const uint64_t ad = ptx::sdesc_add(ad0, off);
-            const uint64_t bd = ptx::sdesc_add(bd0, off);
-            ptx::umma_ss(tmem + kColS0 + sb * 128u, ad, bd, kIdS, kk > 0 ? 1u : 0u);
+            ptx::umma_ss(tmem + kColS + t * 128u, ptx::sdesc_add(ad0, off), ptx::sdesc_add(bd0, off), kIdS,
+                         kk > 0 ? 1u : 0u);
           }
-          ptx::umma_commit(bar.s_full[sb]);
-          ++s_cnt;
-          if (j > 0 && !issue_pv(j - 1, prev_stage)) { ok = false; break; }
-          prev_stage = kv_stage;
-          if (++kv_stage == kStages) { kv_stage = 0; kv_phase ^= 1u; }
+          ptx::umma_commit(bar.s_full[t]);
+          return true;
+        };
+        // O_t += P_t V_j with P_t read from tile t's S buffer in TMEM.
+        auto issue_pv = [&](int t, uint32_t stage) -> bool {
+          if (!ptx::mbar_wait(bar.p_full[t], p_cnt[t] & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 1, 3))) return false;
+          ++p_cnt[t];
+          ptx::tc_fence_after();
+          const uint64_t bd0 = ptx::sdesc_sw128(sbase + L::kK0 + stage * L::kStageBytes + L::kTileBytes, 16384u, 1024u);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            ptx::umma_ts(tmem + kColO + t * 128u, tmem + kColS + t * 128u + kk * 8u, ptx::sdesc_add(bd0, kk * 2048u),
+                         kIdPV, (!first_pv[t] || kk > 0) ? 1u : 0u);
+          first_pv[t] = false;
+          ptx::umma_commit(bar.o_done[t]);
+          return true;
+        };
+        if (pp.n == 0) continue;
+        // prologue: the S MMAs of key tile 0
+        if (!ptx::mbar_wait(bar.kv_full[kv_stage], kv_phase, abort_flag, a.err, lim, ptx::wait_site(1, 1, 5))) { ok = false; break; }
+        ptx::tc_fence_after();
+        for (int t = 0; t < 2 && ok; ++t)
+          if (takes(pp, t, 0) && !issue_s(t, kv_stage)) ok = false;
+        for (int j = 0; j < pp.n && ok; ++j) {
+          const uint32_t st_j = kv_stage;
+          uint32_t st_n = kv_stage + 1, ph_n = kv_phase;
+          if (st_n == kStages) { st_n = 0; ph_n ^= 1u; }
+          const bool more = j + 1 < pp.n;
+          if (takes(pp, 0, j) && !issue_pv(0, st_j)) { ok = false; break; }
+          if (more) {
+            if (!ptx::mbar_wait(bar.kv_full[st_n], ph_n, abort_flag, a.err, lim, ptx::wait_site(1, 1, 5))) { ok = false; break; }
+            ptx::tc_fence_after();
+            if (takes(pp, 0, j + 1) && !issue_s(0, st_n)) { ok = false; break; }
+          }
+          if (takes(pp, 1, j) && !issue_pv(1, st_j)) { ok = false; break; }
+          ptx::umma_commit(bar.kv_empty[st_j]);
+          if (more && takes(pp, 1, j + 1) && !issue_s(1, st_n)) { ok = false; break; }
+          kv_stage = st_n;
+          kv_phase = ph_n;
         }
-        if (!ok) break;
-        if (!issue_pv(n - 1, prev_stage)) { ok = false; break; }
       }
       // Drain: every MMA this thread issued completes before TMEM is freed.
       ptx::umma_commit(bar.drain);
@@ -266,29 +315,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int t = (warp - 2) >> 2;  // tile of the pair this warpgroup serves
+    const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t colS = kColS + static_cast<uint32_t>(t) * 128u;
+    const uint32_t colO = kColO + static_cast<uint32_t>(t) * 128u;
+    const uint32_t sQ = sbase + L::kQ0 + static_cast<uint32_t>(t) * L::kTileBytes;
+    // this warpgroup's barriers (selected, not indexed, so `bar` stays in registers)
+    const uint32_t my_q_full = t ? bar.q_full[1] : bar.q_full[0];
+    const uint32_t my_s_full = t ? bar.s_full[1] : bar.s_full[0];
+    const uint32_t my_p_full = t ? bar.p_full[1] : bar.p_full[0];
+    const uint32_t my_o_done = t ? bar.o_done[1] : bar.o_done[0];
     const float sl2 = a.scale_log2;
-    uint32_t s_cnt = 0, pv_cnt = 0;  // S tiles consumed, P tiles produced
+    uint32_t s_cnt = 0, p_cnt = 0;  // S tiles consumed, P tiles produced
 
-    // This thread's row of a work item.
+    // This thread's row of the warpgroup's tile in a work item.
     struct RowItem {
-      bool valid;
-      int h, n, nkv, doc_start, br_lo, r, limit, blo, bhi;
+      bool valid, on;
+      int h, n, nmain, nkv, nbr0, last, doc_start, br_lo, r, limit, blo, bhi;
     };
-    auto fetch = [&](uint32_t rn, RowItem& it) -> bool {
-      int item = 0;
-      if (!__all_sync(0xffffffffu, ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(1, 2, 14))))
-        return false;
+    auto get_item = [&](uint32_t rn, int& item) -> bool {
+      return __all_sync(0xffffffffu, ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(1, 2, 14)));
+    };
+    auto make_row = [&](int item, RowItem& it) {
       it.valid = item < a.n_items;
-      if (!it.valid) return true;
-      const TileDesc td = a.tiles[a.order[item / Hq]];
+      it.on = false;
+      if (!it.valid) return;
+      const PairPlan pp = load_pair(a, item / Hq);
+      it.on = t ? pp.on[1] : pp.on[0];
+      if (!it.on) return;
+      const TileDesc td = t ? pp.t[1] : pp.t[0];
       it.h = item % Hq;
+      it.n = pp.n;
+      it.nmain = pp.nmain;
+      it.nkv = t ? pp.nkv[1] : pp.nkv[0];
+      it.nbr0 = pp.nbr[0];
+      it.last = (t ? pp.nbr[1] : pp.nbr[0]) > 0 ? (t == 0 ? pp.nmain + pp.nbr[0] - 1 : pp.n - 1) : it.nkv - 1;
       it.doc_start = td.doc_start;
       it.br_lo = td.br_lo;
-      it.nkv = ceil_div(td.kv_end - td.doc_start, 128);
-      it.n = it.nkv + ((a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0);
       it.r = a.row_table[td.row_base + row];
       it.limit = td.doc_start;  // padding rows see one key: keeps their math finite
       it.blo = it.bhi = 0;      // visible branch key rows [blo, bhi)
@@ -296,26 +361,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         it.limit = it.r;
       } else if (it.r >= a.S) {
         const int b = (it.r - a.S) / a.B;
-        const int t = (it.r - a.S) - b * a.B;
+        const int tt = (it.r - a.S) - b * a.B;
         it.limit = a.anchors[b];
         it.blo = b * a.B;
-        it.bhi = it.blo + (a.mode == 1 ? a.B : t + 1);
+        it.bhi = it.blo + (a.mode == 1 ? a.B : tt + 1);
+      }
+    };
+    // Where this thread's query row of `item` lives (false: the tile is absent).
+    auto q_src = [&](int item, const __nv_bfloat16*& src, uint32_t& bytes) -> bool {
+      if (item >= a.n_items) return false;
+      const int2 ids = reinterpret_cast<const int2*>(a.pairs)[item / Hq];
+      const int id = t == 0 ? ids.x : ids.y;
+      if (id < 0) return false;
+      const int r = a.row_table[a.tiles[id].row_base + row];
+      const int h = item % Hq;
+      src = a.q;  // padding row: zero-filled
+      bytes = 0;
+      if (r >= 0 && r < a.S) {
+        src = a.q + (int64_t(r) * Hq + h) * D;
+        bytes = 16;
+      } else if (r >= a.S) {
+        src = a.qb + (int64_t(r - a.S) * Hq + h) * D;
+        bytes = 16;
       }
       return true;
     };
+    // Does this warpgroup's tile take key tile j of the item's stream?
+    auto takes_own = [&](const RowItem& it, int j) -> bool {
+      if (j < it.nmain) return j < it.nkv;
+      return t == 0 ? j - it.nmain < it.nbr0 : j - it.nmain >= it.nbr0;
+    };
     // Copy this thread's query row (bf16, D values) into row `row` of the
     // swizzled Q tile; padding rows are zero-filled.
-    auto copy_q = [&](const RowItem& it) {
-      const __nv_bfloat16* src = a.q;
-      uint32_t bytes = 0;
-      if (it.r >= 0 && it.r < a.S) {
-        src = a.q + (int64_t(it.r) * Hq + it.h) * D;
-        bytes = 16;
-      } else if (it.r >= a.S) {
-        src = a.qb + (int64_t(it.r - a.S) * Hq + it.h) * D;
-        bytes = 16;
-      }
-      const uint32_t dst = sbase + L::kQ + static_cast<uint32_t>(row) * 128u;
+    auto copy_q = [&](const __nv_bfloat16* src, uint32_t bytes) {
+      const uint32_t dst = sQ + static_cast<uint32_t>(row) * 128u;
 #pragma unroll
       for (int cb = 0; cb < D / 64; ++cb)
 #pragma unroll
@@ -328,190 +407,207 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto publish_q = [&]() {
       ptx::cp_async_wait_all();
       ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(bar.q_full);
+      ptx::mbar_arrive(my_q_full);
     };
 
     RowItem cur;
-    bool ok = fetch(0, cur);
-    if (ok && cur.valid) {
-      copy_q(cur);
-      publish_q();
+    int item0 = 0;
+    bool ok = get_item(0, item0);
+    if (ok) {
+      make_row(item0, cur);
+      const __nv_bfloat16* src;
+      uint32_t bytes;
+      if (q_src(item0, src, bytes)) {
+        copy_q(src, bytes);
+        publish_q();
+      }
     }
     for (uint32_t rn = 1; ok && cur.valid; ++rn) {
-      const int h = cur.h, n = cur.n, nkv = cur.nkv, r = cur.r;
-      const int limit = cur.limit, blo = cur.blo, bhi = cur.bhi;
-      RowItem nxt;
-      nxt.valid = false;
-      float m_used = -INFINITY;
-      float l = 0.f;
-      for (int j = 0; j < n; ++j) {
-        if (j == n - 1 && !fetch(rn, nxt)) {
-          ok = false;
-          break;
-        }
-        const uint32_t sb = s_cnt & 1u;
-        const uint32_t sph = (s_cnt >> 1) & 1u;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.s_full[sb], sph, abort_flag, a.err, lim, ptx::wait_site(1, 2, 7)))) {
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tl + kColS0 + sb * 128u + c * 32u, sr[c]);
-        ptx::tmem_wait_ld();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(bar.s_empty[sb]);
-        ++s_cnt;
-        // The item's last S MMA has finished: the next item's rows may overwrite Q.
-        if (j == n - 1 && nxt.valid) copy_q(nxt);
-        // visible columns [lo, hi) of this key tile
-        int lo, hi;
-        if (j < nkv) {
-          lo = 0;
-          hi = limit - (cur.doc_start + 128 * j) + 1;
-        } else {
-          const int kr0 = cur.br_lo + 128 * (j - nkv);
-          lo = blo - kr0;
-          hi = bhi - kr0;
-        }
-        lo = max(lo, 0);
-        hi = min(hi, 128);
-        if (!(lo == 0 && hi == 128)) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int col = c * 32 + i;
-              if (col < lo || col >= hi) sr[c][i] = __float_as_uint(-INFINITY);
+      int nxt_item = 0;
+      bool nxt_on = false, fetched = false;
+      const __nv_bfloat16* nsrc = a.q;
+      uint32_t nbytes = 0;
+      if (cur.on) {
+        const int h = cur.h, nmain = cur.nmain, r = cur.r;
+        const int limit = cur.limit, blo = cur.blo, bhi = cur.bhi;
+        float m_used = -INFINITY;
+        float l = 0.f;
+        bool first = true;
+        for (int j = 0; j < cur.n; ++j) {
+          if (!takes_own(cur, j)) continue;
+          if (j == cur.last) {
+            if (!get_item(rn, nxt_item)) {
+              ok = false;
+              break;
             }
-        }
-        // Row max over 8 independent accumulators, two new values per instruction.
-        float mx8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; i += 2)
-            mx8[(i >> 1) & 7] = ptx::max3(mx8[(i >> 1) & 7], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
-        const float mx = fmaxf(ptx::max3(mx8[0], mx8[1], mx8[2]),
-                               fmaxf(ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float mxs = mx * sl2;
-        float alpha = 1.f;
-        bool rescale = false;
-        if (m_used == -INFINITY) {
-          m_used = mxs;
-        } else if (mxs > m_used + kRescaleThreshold) {
-          alpha = ptx::ex2(m_used - mxs);
-          m_used = mxs;
-          rescale = true;
-        }
-        // P = exp2(S * scale*log2(e) - m), row sum over 4 paired accumulators
-        const float2 c2 = make_float2(sl2, sl2);
-        const float2 nm2 = make_float2(-m_used, -m_used);
-        float2 rs4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) rs4[u] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 x = ptx::fma2(make_float2(__uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1])), c2, nm2);
-            const float2 p = ptx::exp2_sfu(x);
-            rs4[(i >> 1) & 3] = ptx::add2(rs4[(i >> 1) & 3], p);
-            sr[c][i] = __float_as_uint(p.x);
-            sr[c][i + 1] = __float_as_uint(p.y);
+            fetched = true;
+            nxt_on = q_src(nxt_item, nsrc, nbytes);
           }
-        const float2 rsa = ptx::add2(ptx::add2(rs4[0], rs4[1]), ptx::add2(rs4[2], rs4[3]));
-        l = l * alpha + (rsa.x + rsa.y);
-        const uint32_t pb = pv_cnt & 1u;
-        // P buffer pb is free once the P.V that last read it (two tiles ago) finished.
-        bool w = true;
-        if (pv_cnt >= 2)
-          w = ptx::mbar_wait(bar.o_done[pb], ((pv_cnt >> 1) - 1u) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 9));
-        // Rescaling O needs the previous P.V (the other buffer) to have finished.
-        const bool any_rescale = __any_sync(0xffffffffu, rescale);
-        if (any_rescale && j > 0)
-          w = w && ptx::mbar_wait(bar.o_done[pb ^ 1u], ((pv_cnt - 1u) >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 10));
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        ptx::tc_fence_after();
-        if (any_rescale && j > 0) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            ptx::tmem_ld32(tl + kColO + c * 32u, ov);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            ptx::tmem_st32(tl + kColO + c * 32u, ov);
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(my_s_full, s_cnt & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 7)))) {
+            ok = false;
+            break;
           }
-        }
-        // P (bf16, two keys per 32-bit column) -> TMEM buffer pb
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t pw[32];
-#pragma unroll
-          for (int wi = 0; wi < 32; ++wi) {
-            const int key = (h2 * 32 + wi) * 2;
-            pw[wi] = ptx::pack_bf16x2(__uint_as_float(sr[key >> 5][key & 31]),
-                                      __uint_as_float(sr[key >> 5][(key & 31) + 1]));
-          }
-          ptx::tmem_st32(tl + kColP + pb * 64u + h2 * 32u, pw);
-        }
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(bar.p_full[pb]);
-        ++pv_cnt;
-      }
-      if (!ok) break;
-      // The next item's S MMAs may start while this item's epilogue runs.
-      if (nxt.valid) publish_q();
-      // ---------------------------------------------------------- epilogue
-      {  // the item's last P.V (and, in order, every earlier one) finished
-        const uint32_t last = pv_cnt - 1u;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar.o_done[last & 1u], (last >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 11)))) {
-          ok = false;
-          break;
-        }
-      }
-      ptx::tc_fence_after();
-      const float inv_l = 1.f / l;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        ptx::tmem_ld32(tl + kColO + c * 32u, ov);
-        ptx::tmem_wait_ld();
-        if (r >= 0) {
-          if (a.out_bf16) {
-            __nv_bfloat16* dst = (r < a.S ? a.o + (int64_t(r) * Hq + h) * D
-                                          : a.ob + (int64_t(r - a.S) * Hq + h) * D) + c * 32;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint4 w;
-              w.x = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 0]) * inv_l, __uint_as_float(ov[q4 * 8 + 1]) * inv_l);
-              w.y = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 2]) * inv_l, __uint_as_float(ov[q4 * 8 + 3]) * inv_l);
-              w.z = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 4]) * inv_l, __uint_as_float(ov[q4 * 8 + 5]) * inv_l);
-              w.w = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 6]) * inv_l, __uint_as_float(ov[q4 * 8 + 7]) * inv_l);
-              reinterpret_cast<uint4*>(dst)[q4] = w;
-            }
+          ++s_cnt;
+          ptx::tc_fence_after();
+          // The tile's last S MMA has finished: the next item's rows may overwrite Q.
+          if (j == cur.last && nxt_on) copy_q(nsrc, nbytes);
+          // visible columns [lo, hi) of this key tile
+          int lo, hi;
+          if (j < nmain) {
+            lo = 0;
+            hi = limit - (cur.doc_start + 128 * j) + 1;
           } else {
-            float* dst = a.o_part + (int64_t(r) * Hq + h) * D + c * 32;
+            const int kb = t == 0 ? j - nmain : j - nmain - cur.nbr0;
+            const int kr0 = cur.br_lo + 128 * kb;
+            lo = blo - kr0;
+            hi = bhi - kr0;
+          }
+          lo = max(lo, 0);
+          hi = min(hi, 128);
+          const bool full = lo == 0 && hi == 128;
+          // Pass 1: row max, 32 columns at a time, 8 independent accumulators.
+          float mx8[8];
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              float4 w;
-              w.x = __uint_as_float(ov[q4 * 4 + 0]) * inv_l;
-              w.y = __uint_as_float(ov[q4 * 4 + 1]) * inv_l;
-              w.z = __uint_as_float(ov[q4 * 4 + 2]) * inv_l;
-              w.w = __uint_as_float(ov[q4 * 4 + 3]) * inv_l;
-              reinterpret_cast<float4*>(dst)[q4] = w;
+          for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t sr[32];
+            ptx::tmem_ld32(tl + colS + c * 32u, sr);
+            ptx::tmem_wait_ld();
+            if (!full) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c * 32 + i < lo || c * 32 + i >= hi) sr[i] = __float_as_uint(-INFINITY);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 2)
+              mx8[(i >> 1) & 7] = ptx::max3(mx8[(i >> 1) & 7], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+          }
+          const float mx = fmaxf(ptx::max3(mx8[0], mx8[1], mx8[2]),
+                                 fmaxf(ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float mxs = mx * sl2;
+          float alpha = 1.f;
+          bool rescale = false;
+          if (m_used == -INFINITY) {
+            m_used = mxs;
+          } else if (mxs > m_used + kRescaleThreshold) {
+            alpha = ptx::ex2(m_used - mxs);
+            m_used = mxs;
+            rescale = true;
+          }
+          // Rescaling O needs this tile's previous P.V to have finished.
+          const bool any_rescale = __any_sync(0xffffffffu, rescale);
+          if (any_rescale && !first) {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(my_o_done, (p_cnt - 1u) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 10)))) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t ov[32];
+              ptx::tmem_ld32(tl + colO + c * 32u, ov);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              ptx::tmem_st32(tl + colO + c * 32u, ov);
+            }
+          }
+          // Pass 2: P = exp2(S * scale*log2(e) - m) as bf16 pairs over the first
+          // 64 columns of S, row sum over 4 paired accumulators.
+          const float2 c2 = make_float2(sl2, sl2);
+          const float2 nm2 = make_float2(-m_used, -m_used);
+          float2 rs4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) rs4[u] = make_float2(0.f, 0.f);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t sr[32];
+            ptx::tmem_ld32(tl + colS + c * 32u, sr);
+            ptx::tmem_wait_ld();
+            if (!full) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c * 32 + i < lo || c * 32 + i >= hi) sr[i] = __float_as_uint(-INFINITY);
+            }
+            uint32_t pw[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float2 x = ptx::fma2(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2, nm2);
+              const float2 p = ptx::exp2_sfu(x);
+              rs4[(i >> 1) & 3] = ptx::add2(rs4[(i >> 1) & 3], p);
+              pw[i >> 1] = ptx::pack_bf16x2(p.x, p.y);
+            }
+            // keys 32c..32c+31 -> P columns 16c..16c+15, S columns read in this or an earlier chunk
+            ptx::tmem_st16(tl + colS + c * 16u, pw);
+          }
+          const float2 rsa = ptx::add2(ptx::add2(rs4[0], rs4[1]), ptx::add2(rs4[2], rs4[3]));
+          l = l * alpha + (rsa.x + rsa.y);
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(my_p_full);
+          ++p_cnt;
+          first = false;
+        }
+        if (!ok) break;
+        // The next item's S MMAs may start while this item's epilogue runs.
+        if (nxt_on) publish_q();
+        // ---------------------------------------------------------- epilogue
+        // the tile's last P.V (and, in order, every earlier one) finished
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(my_o_done, (p_cnt - 1u) & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 2, 11)))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const float inv_l = 1.f / l;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(tl + colO + c * 32u, ov);
+          ptx::tmem_wait_ld();
+          if (r >= 0) {
+            if (a.out_bf16) {
+              __nv_bfloat16* dst = (r < a.S ? a.o + (int64_t(r) * Hq + h) * D
+                                            : a.ob + (int64_t(r - a.S) * Hq + h) * D) + c * 32;
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 w;
+                w.x = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 0]) * inv_l, __uint_as_float(ov[q4 * 8 + 1]) * inv_l);
+                w.y = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 2]) * inv_l, __uint_as_float(ov[q4 * 8 + 3]) * inv_l);
+                w.z = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 4]) * inv_l, __uint_as_float(ov[q4 * 8 + 5]) * inv_l);
+                w.w = ptx::pack_bf16x2(__uint_as_float(ov[q4 * 8 + 6]) * inv_l, __uint_as_float(ov[q4 * 8 + 7]) * inv_l);
+                reinterpret_cast<uint4*>(dst)[q4] = w;
+              }
+            } else {
+              float* dst = a.o_part + (int64_t(r) * Hq + h) * D + c * 32;
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4) {
+                float4 w;
+                w.x = __uint_as_float(ov[q4 * 4 + 0]) * inv_l;
+                w.y = __uint_as_float(ov[q4 * 4 + 1]) * inv_l;
+                w.z = __uint_as_float(ov[q4 * 4 + 2]) * inv_l;
+                w.w = __uint_as_float(ov[q4 * 4 + 3]) * inv_l;
+                reinterpret_cast<float4*>(dst)[q4] = w;
+              }
             }
           }
         }
+        if (r >= 0) a.lse[int64_t(h) * a.lse_ld + r] = (m_used + __log2f(l)) * 0.69314718055994531f;
+        ptx::tc_fence_before();
       }
-      if (r >= 0) a.lse[int64_t(h) * a.lse_ld + r] = (m_used + __log2f(l)) * 0.69314718055994531f;
-      ptx::tc_fence_before();
-      cur = nxt;
+      if (!fetched) {
+        // This tile had no part in the item: take the next one now; the tile's
+        // Q buffer is free (its last S MMA finished before this item began).
+        if (!get_item(rn, nxt_item)) {
+          ok = false;
+          break;
+        }
+        if (q_src(nxt_item, nsrc, nbytes)) {
+          copy_q(nsrc, nbytes);
+          publish_q();
+        }
+      }
+      make_row(nxt_item, cur);
     }
     // Copies this thread issued must land before the CTA's shared memory goes away.
     ptx::cp_async_wait_all();
@@ -519,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }

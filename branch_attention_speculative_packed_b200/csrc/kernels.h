@@ -18,9 +18,9 @@ struct FwdArgs {
   const int32_t* anchors;    // [Nb]
   const int32_t* row_table;  // [ntiles * 128], -1 = padding
   const TileDesc* tiles;     // [ntiles]
-  const int32_t* order;      // [ntiles], longest first
+  const int32_t* pairs;      // [n_pairs][2] tile indices (second -1: single), longest first
   int S, Nb, B, mode, Hq, G, d;
-  int n_items;               // ntiles * Hq
+  int n_items;               // n_pairs * Hq
   float scale_log2;          // softmax scale * log2(e)
   int with_branch;           // also visit the branch key tiles (fused forward)
   int out_bf16;              // 1: bf16 o / ob; 0: fp32 o_part

@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <numeric>
+#include <utility>
 
 namespace ba {
 
@@ -191,6 +192,32 @@ void build_plan(const ba_problem* p, Plan* plan) {
   }
   std::stable_sort(plan->order.begin(), plan->order.end(),
                    [&](int a, int b) { return cost[a] > cost[b]; });
+  // Forward pairs: tiles 2k and 2k+1 of each document share the document's
+  // main key tiles; a pair streams max(main tiles) plus both branch ranges.
+  std::vector<std::pair<int32_t, int32_t>> prs;
+  std::vector<int64_t> pcost;
+  for (int i = 0; i < nt;) {
+    const bool two = i + 1 < nt && plan->tiles[i + 1].doc_start == plan->tiles[i].doc_start;
+    const TileDesc& ta = plan->tiles[i];
+    int64_t c = cost[i];
+    if (two) {
+      const TileDesc& tb = plan->tiles[i + 1];
+      const int64_t ma = (int64_t(ta.kv_end) - ta.doc_start + kKeysPerTile - 1) / kKeysPerTile;
+      const int64_t mb = (int64_t(tb.kv_end) - tb.doc_start + kKeysPerTile - 1) / kKeysPerTile;
+      c = cost[i] + cost[i + 1] - std::min(ma, mb);
+    }
+    prs.emplace_back(i, two ? i + 1 : -1);
+    pcost.push_back(c);
+    i += two ? 2 : 1;
+  }
+  std::vector<int> pidx(prs.size());
+  std::iota(pidx.begin(), pidx.end(), 0);
+  std::stable_sort(pidx.begin(), pidx.end(), [&](int a, int b) { return pcost[a] > pcost[b]; });
+  plan->pairs.clear();
+  for (int k : pidx) {
+    plan->pairs.push_back(prs[k].first);
+    plan->pairs.push_back(prs[k].second);
+  }
 }
 
 void build_kv_plan(const ba_problem* p, Plan* plan) {
@@ -259,6 +286,8 @@ WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int whic
   off = align_up(off + plan.chunks_dev.size() * sizeof(ChunkDev), 256);
   w.rows_off = off;
   off = align_up(off + size_t(w.n_slots) * sizeof(int32_t), 256);
+  w.pairs_off = off;
+  off = align_up(off + 2 * nt * sizeof(int32_t), 256);
   if (which == BA_WS_BWD) {
     const size_t rows = size_t(p->S) + size_t(p->Nb) * (p->Nb > 0 ? p->B : 0);
     const size_t slots = size_t(w.n_slots);

@@ -35,6 +35,9 @@ struct Plan {
   std::vector<Chunk> chunks;       // doc-major, chunk-index minor (= position order)
   std::vector<TileDesc> tiles;     // in position order
   std::vector<int32_t> order;      // tile indices, longest (most key tiles) first
+  // Forward work items: two consecutive row tiles of one document (the second
+  // -1 when the document has an odd tile left), two int32 per pair, longest first.
+  std::vector<int32_t> pairs;
   std::vector<ChunkDev> chunks_dev;
   std::vector<int64_t> rank_pairs; // main (row tile, key tile) pairs per virtual rank
   std::vector<KvItem> kv_items;    // key tiles of the dK/dV pass
@@ -59,7 +62,7 @@ void build_kv_plan(const ba_problem* p, Plan* plan);
 // Workspace layout shared by the forward and backward paths.
 struct WorkspaceLayout {
   size_t counters_off = 0;  // uint32 work-item counters (forward, dQ pass, dK/dV pass)
-  size_t tiles_off = 0, order_off = 0, chunks_off = 0, rows_off = 0;
+  size_t tiles_off = 0, order_off = 0, chunks_off = 0, rows_off = 0, pairs_off = 0;
   // backward only
   size_t kv_items_off = 0, kv_order_off = 0;
   size_t qg_off = 0, dog_off = 0;    // Q and dO gathered into slot order, bf16 [slots, Hq, d]
