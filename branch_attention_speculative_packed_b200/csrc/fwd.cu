@@ -534,7 +534,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
               const float2 x = ptx::fma2(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2, nm2);
-              const float2 p = ptx::exp2_sfu(x);
+              // every other pair on the FMA pipe: two warpgroups share one special-function unit
+              const float2 p = ((i >> 1) & 1) ? ptx::exp2_poly(x) : ptx::exp2_sfu(x);
               rs4[(i >> 1) & 3] = ptx::add2(rs4[(i >> 1) & 3], p);
               pw[i >> 1] = ptx::pack_bf16x2(p.x, p.y);
             }
