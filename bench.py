@@ -215,6 +215,29 @@ def workload_config(world: int, index: int = WORKLOAD_INDEX) -> dict:
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
+# DRAM traffic of one launch of a kernel on the 64K workload, from the ncu
+# capture summarised in profiles/ncu_tensor_kernels_eagle3_8k.md (8K case,
+# scaled to the 64K launch by its slot count), valid for the kernel source it
+# was taken on: reported only while that source file is unchanged.
+KERNEL_TRAFFIC = {
+    "bwd_dkdv": {"bytes_per_launch": 4.926e9, "source": "bwd_dkdv.cu",
+                 "sha1": "19c28833510a7bc2f14b450208644ff60b80db62"},
+}
+
+
+def kernel_traffic(kind: str):
+    import hashlib
+    t = KERNEL_TRAFFIC.get(kind)
+    if t is None:
+        return None
+    path = os.path.join(ROOT, "branch_attention_speculative_packed_b200", "csrc", t["source"])
+    try:
+        digest = hashlib.sha1(open(path, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return t["bytes_per_launch"] if digest == t["sha1"] else None
+
+
 def kernel_flops(kind: str, d: int, pairs: int, Hq: int) -> float:
     """Algorithmic FLOPs of one launch of a tensor-core kernel over the
     visible pairs: forward 2 GEMMs (QK^T, PV), dQ pass 3 (QK^T, dO V^T, dS K),
@@ -353,7 +376,8 @@ def run_gpu(args):
                        useful_flop_per_step=useful),
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": None, "peak_source": f"{peak_src} bf16_tflops_sustained"},
+                     "traffic": kernel_traffic(dom) if widx == WORKLOAD_INDEX else None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained"},
         "kernels": {k: {"ms": round(v["ms_per_launch"], 4), "launches": v["launches"],
                         "share": round(v["share"], 4)} for k, v in per_kernel.items()},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
