@@ -329,6 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_ld32(tl + kColS + half_col, sv[0]);
           ptx::tmem_ld32(tl + kColS + half_col + 32u, sv[1]);
           ptx::tmem_wait_ld();
+          ptx::tmem_regs_ready(sv[0]);
+          ptx::tmem_regs_ready(sv[1]);
           const uint8_t* sq = smem + L::kQ0 + qs * L::kQSlot;
           const float4* L4 = reinterpret_cast<const float4*>(sq + L::kSL) + wg * 16;  // -L * log2(e)
           const float4* D4 = reinterpret_cast<const float4*>(sq + L::kSD) + wg * 16;
@@ -380,6 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_ld32(tl + kColDP + half_col, pv[0]);
           ptx::tmem_ld32(tl + kColDP + half_col + 32u, pv[1]);
           ptx::tmem_wait_ld();
+          ptx::tmem_regs_ready(pv[0]);
+          ptx::tmem_regs_ready(pv[1]);
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
             const float4 dd = D4[q];
@@ -423,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t v[32];
           ptx::tmem_ld32(tl + col0 + c * 32u, v);
           ptx::tmem_wait_ld();
+          ptx::tmem_regs_ready(v);
           if (own || zero) {
             __nv_bfloat16* dst = out + (int64_t(kp) * a.Hkv + g) * D + wg * (D / 2) + c * 32;
             const float z = zero ? 0.f : mul;

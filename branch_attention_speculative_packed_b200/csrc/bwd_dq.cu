@@ -322,6 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tl + kColDP + c * 32u, dp[c]);
         ptx::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_regs_ready(dp[c]);
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar_dp_empty);
         int lo, hi;
@@ -348,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t sr[32];
             ptx::tmem_ld32(tl + kColS0 + sb * 128u + c * 32u, sr);
             ptx::tmem_wait_ld();
+            ptx::tmem_regs_ready(sr);
             // exponent arguments S * scale*log2(e) - L*log2(e), two keys per instruction
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
@@ -390,6 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t qv[32];
         ptx::tmem_ld32(tl + kColDQ + c * 32u, qv);
         ptx::tmem_wait_ld();
+        ptx::tmem_regs_ready(qv);
         if (r >= 0) {
           __nv_bfloat16* dst = (r < a.S ? a.dq + (int64_t(r) * Hq + h) * D
                                         : a.dqb + (int64_t(r - a.S) * Hq + h) * D) + c * 32;

@@ -474,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t sr[32];
             ptx::tmem_ld32(tl + colS + c * 32u, sr);
             ptx::tmem_wait_ld();
+            ptx::tmem_regs_ready(sr);
             if (!full) {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
@@ -508,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint32_t ov[32];
               ptx::tmem_ld32(tl + colO + c * 32u, ov);
               ptx::tmem_wait_ld();
+              ptx::tmem_regs_ready(ov);
 #pragma unroll
               for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
               ptx::tmem_st32(tl + colO + c * 32u, ov);
@@ -525,6 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t sr[32];
             ptx::tmem_ld32(tl + colS + c * 32u, sr);
             ptx::tmem_wait_ld();
+            ptx::tmem_regs_ready(sr);
             if (!full) {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
@@ -566,6 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t ov[32];
           ptx::tmem_ld32(tl + colO + c * 32u, ov);
           ptx::tmem_wait_ld();
+          ptx::tmem_regs_ready(ov);
           if (r >= 0) {
             if (a.out_bf16) {
               __nv_bfloat16* dst = (r < a.S ? a.o + (int64_t(r) * Hq + h) * D
