@@ -49,7 +49,6 @@ def build(force: bool = False, verbose: bool = False) -> str:
            "-Xcompiler", "-fvisibility=hidden", "-cudart", "static", "-Xptxas", "-v" if verbose else "-O3",
            "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp"]
     cmd += [os.path.join(CSRC, s) for s in SOURCES]
-    cmd += ["-lcuda"] if False else []
     res = subprocess.run(cmd, cwd=CSRC, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
