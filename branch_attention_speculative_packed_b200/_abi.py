@@ -30,6 +30,7 @@ EXPORTED = (
     "ba_workspace_size", "ba_main_fwd", "ba_branch_fwd", "ba_lse_merge", "ba_fused_fwd",
     "ba_bwd", "ba_status_string", "ba_sync_status", "ba_plan_stats", "ba_profile_enable",
     "ba_profile_collect", "ba_last_error_word", "ba_fused_fwd_noalloc", "ba_plan_rank_work",
+    "ba_plan_fwd_pairs",
 )
 
 
@@ -86,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.ba_plan_stats.argtypes = [P, i64p, i64p, i64p]
         L.ba_plan_rank_work.argtypes = [P, i64p, i32]
         L.ba_plan_rank_work.restype = ctypes.c_int
+        L.ba_plan_fwd_pairs.argtypes = [P, ctypes.POINTER(ctypes.c_int32), ctypes.c_int64]
+        L.ba_plan_fwd_pairs.restype = ctypes.c_int64
         L.ba_last_error_word.argtypes = []
         L.ba_last_error_word.restype = ctypes.c_uint32
         L.ba_profile_enable.argtypes = [i32]

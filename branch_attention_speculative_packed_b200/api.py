@@ -101,6 +101,15 @@ class BranchAttention:
             check(n, "ba_plan_rank_work")
         return list(buf)
 
+    def fwd_pairs(self):
+        """Forward work items: (tile, tile or -1) pairs in claim order."""
+        n = _abi.lib().ba_plan_fwd_pairs(ctypes.byref(self._problem()), None, 0)
+        if n < 0:
+            check(n, "ba_plan_fwd_pairs")
+        buf = (ctypes.c_int32 * (2 * max(n, 1)))()
+        _abi.lib().ba_plan_fwd_pairs(ctypes.byref(self._problem()), buf, n)
+        return [(buf[2 * i], buf[2 * i + 1]) for i in range(n)]
+
     # ------------------------------------------------------------------ forward
     def fused_fwd(self, q, k, v, qb, kb, vb, out=None, stream=None):
         """Steps a2+a3+a4: returns (o bf16 [S,Hq,d], ob bf16 [Nb,B,Hq,d], lse fp32 [Hq,rows])."""

@@ -259,6 +259,19 @@ int ba_plan_rank_work(const ba_problem* p, int64_t* pairs, int cap) {
   return p->R;
 }
 
+int64_t ba_plan_fwd_pairs(const ba_problem* p, int32_t* tiles, int64_t cap) {
+  ba_status s = validate(p, false);
+  if (s != BA_OK) return s;
+  Plan plan;
+  build_plan(p, &plan);
+  const int64_t n = static_cast<int64_t>(plan.pairs.size() / 2);
+  for (int64_t i = 0; tiles && i < cap && i < n; ++i) {
+    tiles[2 * i] = plan.pairs[2 * i];
+    tiles[2 * i + 1] = plan.pairs[2 * i + 1];
+  }
+  return n;
+}
+
 ba_status ba_main_fwd(const ba_problem* p, float* o_part, float* lse_part, ba_stream_t stream) {
   return run_fwd(p, false, o_part, nullptr, nullptr, lse_part, reinterpret_cast<cudaStream_t>(stream));
 }

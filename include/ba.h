@@ -243,6 +243,16 @@ BA_API int ba_profile_collect(const char** names, double* total_ms, int* launche
  * nearly equal (the pages: the split balances the triangular causal work). */
 BA_API int ba_plan_rank_work(const ba_problem* p, int64_t* pairs, int cap);
 
+/* Work items of the fused / main forward (host only, no GPU needed): each
+ * item is a pair of consecutive row tiles of one document (tile indices in
+ * position order; the second is -1 when a document has an odd tile left),
+ * which share the document's main key tiles, in the order the kernel claims
+ * them (most key tiles first).  Writes min(cap, n) pairs as 2 x int32 each to
+ * `tiles` (may be NULL) and returns n, the number of pairs, or a negative
+ * status for an invalid problem.  Each forward work item is one pair times
+ * one query head. */
+BA_API int64_t ba_plan_fwd_pairs(const ba_problem* p, int32_t* tiles, int64_t cap);
+
 #ifdef __cplusplus
 }
 #endif

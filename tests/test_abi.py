@@ -143,8 +143,57 @@ def test_planner_on_workload_layouts(ba, idx):
         t, p, rp = _restated_plan(cu.tolist(), anc.tolist(), cfg.B, cfg.R)
         assert (st["row_tiles"], st["tile_pairs"]) == (t, p)
         assert a.rank_work() == rp
+        assert a.fwd_pairs() == _restated_pairs(cu.tolist(), anc.tolist(), cfg.B)
     # every visible pair lies in a visited tile pair
     assert st["tile_pairs"] * 128 * 128 >= st["visible_pairs"] - cfg.n_anchors * cfg.B * cfg.B
+
+
+def _restated_pairs(cu, anc, B):
+    """Forward work items restated: per document, tiles 2k and 2k+1 (the last
+    alone when the count is odd); a tile costs its main key tiles plus its
+    branch key tiles (the branches with a row in the tile, B keys each); a pair
+    costs both minus the shorter main range they share; most cost first,
+    position order among equals."""
+    tiles = []  # (doc, main key tiles, branch key tiles)
+    for di in range(len(cu) - 1):
+        s, e = cu[di], cu[di + 1]
+        rows = [(p, 0, 0, 0) for p in range(s, e)]
+        rows += [(a, 1, b, t) for b, a in enumerate(anc) if s <= a < e for t in range(B)]
+        rows.sort()
+        for i in range(0, len(rows), 128):
+            tile = rows[i:i + 128]
+            nkv = -(-(tile[-1][0] - s + 1) // 128)
+            bs = [r[2] for r in tile if r[1] == 1]
+            nbr = -(-((max(bs) - min(bs) + 1) * B) // 128) if bs else 0
+            tiles.append((di, nkv, nbr))
+    pairs, cost = [], []
+    i = 0
+    while i < len(tiles):
+        two = i + 1 < len(tiles) and tiles[i + 1][0] == tiles[i][0]
+        c = tiles[i][1] + tiles[i][2]
+        if two:
+            c += tiles[i + 1][1] + tiles[i + 1][2] - min(tiles[i][1], tiles[i + 1][1])
+        pairs.append((i, i + 1 if two else -1))
+        cost.append(c)
+        i += 2 if two else 1
+    order = sorted(range(len(pairs)), key=lambda k: -cost[k])  # stable
+    return [pairs[k] for k in order]
+
+
+@pytest.mark.parametrize("case", [
+    ([0, 256], [23, 43, 60, 72, 179, 200, 201, 255], 4, 2),
+    ([0, 3, 10, 700, 1000], list(range(0, 1000, 7)), 3, 4),
+    ([0, 1, 2, 3], [0, 1, 2], 2, 8),
+    ([0, 500], [], 3, 3),
+    ([0, 300, 301], [299, 299, 300], 16, 1),
+])
+def test_forward_pairs_match_restatement(ba, case):
+    cu, anc, B, R = case
+    a = _attn(ba, cu, anc, B=B, R=R)
+    got = a.fwd_pairs()
+    assert got == _restated_pairs(cu, anc, B)
+    covered = sorted(t for p in got for t in p if t >= 0)
+    assert covered == list(range(a.plan_stats()["row_tiles"]))  # every tile exactly once
 
 
 @pytest.mark.parametrize("R", [2, 4, 8])
