@@ -246,6 +246,36 @@ def kernel_flops(kind: str, d: int, pairs: int, Hq: int) -> float:
     return 2.0 * g * d * pairs * Hq
 
 
+def merge_bandwidth(ba, cfg, rows: int, dev, world: int, hbm_gbs: float, parts: int = 2) -> dict:
+    """HBM bandwidth of the k-way Eq. 2 merge (`ba_lse_merge`) over `rows`
+    rows of the workload's head layout: k fp32 partials in, bf16 O and fp32
+    LSE out; inputs far larger than L2, timed with CUDA events."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(2024)
+    o_parts = [torch.randn(rows, cfg.Hq, cfg.d, device=dev, generator=g) for _ in range(parts)]
+    lse_parts = [torch.randn(cfg.Hq, rows, device=dev, generator=g) * 4.0 for _ in range(parts)]
+    o = torch.empty(rows, cfg.Hq, cfg.d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(cfg.Hq, rows, dtype=torch.float32, device=dev)
+    for _ in range(2):
+        ba.lse_merge(o_parts, lse_parts, out=(o, lse))
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    reps = 5
+    e0.record()
+    for _ in range(reps):
+        ba.lse_merge(o_parts, lse_parts, out=(o, lse))
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    nbytes = rows * cfg.Hq * (parts * (4 * cfg.d + 4) + 2 * cfg.d + 4)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del o_parts, lse_parts, o, lse
+    return {"kernel": "lse_merge", "parts": parts, "rows": rows, "bytes_per_launch": nbytes,
+            "ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "peak_gbs": hbm_gbs,
+            "frac": round(gbs / hbm_gbs, 4)}
+
+
 def run_gpu(args):
     import torch
     import branch_attention_speculative_packed_b200 as ba
@@ -390,6 +420,9 @@ def run_gpu(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = total_useful * e2e_steps / (e2e_ms / 1e3) / 1e12
 
+    merge = merge_bandwidth(ba, cfg, Nb * cfg.B if Nb else S, dev, world,
+                            float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])))
+
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -416,6 +449,7 @@ def run_gpu(args):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "pipelined": "h2d / compute / d2h on three streams, two buffer sets"},
         "gpu_launches": launches,
+        "merge": merge,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline and widx == WORKLOAD_INDEX:

@@ -156,34 +156,52 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const MergeArgs a) {
     if (live) a.lse_out[int64_t(h) * a.lse_out_ld + my] = Lr;
     const int64_t left = int64_t(a.rows) - r0;
     const int nr = left < 32 ? static_cast<int>(left) : 32;
-    for (int i = 0; i < nr; ++i) {
-      const int64_t base = ((r0 + i) * a.H + h) * D + lane * E;
-      float acc[E];
+    // Four rows at a time, so each warp keeps 4 x nparts row loads in flight.
+    for (int i0 = 0; i0 < nr; i0 += 4) {
+      float acc[4][E];
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[u][e] = 0.f;
 #pragma unroll
       for (int p = 0; p < 16; ++p) {
         if (p >= a.nparts) break;
-        const float wp = __shfl_sync(0xffffffffu, wt[p], i);
-        if constexpr (E == 4) {
-          const float4 v = *reinterpret_cast<const float4*>(a.o[p] + base);
-          acc[0] = fmaf(wp, v.x, acc[0]);
-          acc[1] = fmaf(wp, v.y, acc[1]);
-          acc[2] = fmaf(wp, v.z, acc[2]);
-          acc[3] = fmaf(wp, v.w, acc[3]);
-        } else {
-          const float2 v = *reinterpret_cast<const float2*>(a.o[p] + base);
-          acc[0] = fmaf(wp, v.x, acc[0]);
-          acc[1] = fmaf(wp, v.y, acc[1]);
+        float v[4][E];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t base = ((r0 + i0 + u) * a.H + h) * D + lane * E;
+          if (i0 + u < nr) {
+            if constexpr (E == 4) {
+              const float4 x = *reinterpret_cast<const float4*>(a.o[p] + base);
+              v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
+            } else {
+              const float2 x = *reinterpret_cast<const float2*>(a.o[p] + base);
+              v[u][0] = x.x; v[u][1] = x.y;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) v[u][e] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float wp = __shfl_sync(0xffffffffu, wt[p], (i0 + u) & 31);
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[u][e] = fmaf(wp, v[u][e], acc[u][e]);
         }
       }
-      if constexpr (E == 4) {
-        uint2 o;
-        o.x = ptx::pack_bf16x2(acc[0], acc[1]);
-        o.y = ptx::pack_bf16x2(acc[2], acc[3]);
-        *reinterpret_cast<uint2*>(a.o_out + base) = o;
-      } else {
-        *reinterpret_cast<uint32_t*>(a.o_out + base) = ptx::pack_bf16x2(acc[0], acc[1]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (i0 + u >= nr) break;
+        const int64_t base = ((r0 + i0 + u) * a.H + h) * D + lane * E;
+        if constexpr (E == 4) {
+          uint2 o;
+          o.x = ptx::pack_bf16x2(acc[u][0], acc[u][1]);
+          o.y = ptx::pack_bf16x2(acc[u][2], acc[u][3]);
+          *reinterpret_cast<uint2*>(a.o_out + base) = o;
+        } else {
+          *reinterpret_cast<uint32_t*>(a.o_out + base) = ptx::pack_bf16x2(acc[u][0], acc[u][1]);
+        }
       }
     }
   }
