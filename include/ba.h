@@ -167,8 +167,8 @@ BA_API ba_status ba_fused_fwd(const ba_problem* p, void* o, void* ob, float* lse
  * start-up, or a caller that must not trigger an allocation's implicit
  * synchronisation in the middle of a stream.  This entry point computes
  * exactly what ba_fused_fwd computes (same kernels, same plan, same outputs)
- * but takes its scratch space (the plan: tile table, order, chunk table and
- * row table) from a file-scope device array inside the library instead of
+ * but takes its scratch space (the plan: tile table, order, tile pairs, chunk
+ * table and row table) from a file-scope device array inside the library instead of
  * p->workspace, which is ignored along with p->workspace_bytes.
  *   - Capacity: BA_STATIC_SCRATCH_BYTES (8 MiB), enough for problems of up to
  *     about 1.9 million rows (S + Nb*B).  Every GPU that loads the library
