@@ -110,3 +110,67 @@ def sub_heads(problem, groups):
                    None if problem.do is None else problem.do.index_select(1, hq),
                    None if problem.dob is None else problem.dob.index_select(2, hq))
     return p, heads
+
+
+def oracle_rows_by_group(problem, rows=None, groups=None, backward=False):
+    """The row-set oracle over the given concatenated rows (default: all) for
+    the query heads of every listed KV group (default: all), one thread per
+    group.
+
+    Each thread runs the oracle, unchanged, on a view of the problem restricted
+    to one KV group (``sub_heads``); numpy's BLAS calls and ufunc loops release
+    the GIL, so the groups run side by side (BLAS itself is limited to one
+    thread per caller meanwhile).  Inputs may stay on the device: the oracle
+    converts only the rows it reads.
+
+    Returns a dict with ``heads`` (query heads, group-major), ``rows``,
+    ``O`` [n, len(heads), d] and ``L`` [len(heads), n]; with ``backward`` (dO
+    in the problem) also ``dQ`` [n, len(heads), d] and, per listed group in
+    that order, the key gradients those rows' dO produce: ``dk``/``dv``
+    [S, len(groups), d] and ``dkb``/``dvb`` [Nb, B, len(groups), d]."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    from threadpoolctl import threadpool_limits
+
+    c = problem.cfg
+    G = c.Hq // c.Hkv
+    groups = list(range(c.Hkv)) if groups is None else list(groups)
+    if rows is None:
+        rows = np.arange(problem.S + problem.Nb * c.B)
+    rows = np.asarray(rows, dtype=np.int64)
+    cu, anc = problem.cu_seqlens.numpy(), problem.anchors.numpy()
+
+    def one(g):
+        sub, _ = sub_heads(problem, [g])
+        args = (sub.q, sub.k, sub.v, sub.qb, sub.kb, sub.vb)
+        _, O, L = orc.forward_rows(*args, cu, anc, c.B, c.mode, rows=rows)
+        if not backward:
+            return O, L
+        _, dQ, dk, dv, dkb, dvb = orc.backward_rows(*args, sub.do, sub.dob, cu, anc, c.B, c.mode,
+                                                    rows=rows)
+        return O, L, dQ, dk, dv, dkb, dvb
+
+    workers = max(1, min(len(groups), os.cpu_count() or 1))
+    with threadpool_limits(limits=max(1, (os.cpu_count() or 1) // workers)):
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            res = list(ex.map(one, groups))
+    out = {"heads": [g * G + i for g in groups for i in range(G)], "rows": rows,
+           "O": np.concatenate([r[0] for r in res], axis=1),
+           "L": np.concatenate([r[1] for r in res], axis=0)}
+    if backward:
+        out["dQ"] = np.concatenate([r[2] for r in res], axis=1)
+        out["dk"] = np.concatenate([r[3] for r in res], axis=1)
+        out["dv"] = np.concatenate([r[4] for r in res], axis=1)
+        out["dkb"] = np.concatenate([r[5] for r in res], axis=2)
+        out["dvb"] = np.concatenate([r[6] for r in res], axis=2)
+    return out
+
+
+def config_rows(problem, n_rows, seed):
+    """Seeded, stratified query rows of a large configuration: about half main
+    and half branch rows, plus the first and last row of every document, every
+    zigzag chunk edge and the branch rows of anchors at document ends."""
+    edges = [e[2] for e in orc.zigzag_chunks(problem.cu_seqlens.numpy(), problem.cfg.R)]
+    return wl.sample_rows(problem.cu_seqlens, problem.anchors, problem.cfg.B, n_rows, seed=seed,
+                          extra=edges).numpy()

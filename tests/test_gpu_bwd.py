@@ -9,8 +9,8 @@ import torch
 
 import oracle as orc
 import workloads as wl
-from gpu_cases import (SMALL_CASES, TOL_GRAD, attn_for, make_case, max_abs, sub_heads,
-                       to_device)
+from gpu_cases import (SMALL_CASES, TOL_GRAD, attn_for, config_rows, make_case, max_abs,
+                       oracle_rows_by_group, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -90,66 +90,56 @@ def _check_invariants(prob, grads, rel=2e-2):
     assert sdk.abs().max().item() <= rel * mag + 1e-3
 
 
-@pytest.mark.parametrize("idx,groups", [(1, [2]), (2, [5])])
-def test_bwd_config_full(ba, idx, groups):
-    """8K chain and 32K block configs, every row and key, query heads of the
-    listed KV groups in the oracle (all heads on the GPU)."""
+@pytest.mark.parametrize("idx", [1, pytest.param(2, marks=pytest.mark.slow)])
+def test_bwd_config_full(ba, idx):
+    """8K chain and 32K block configs: every row, every key and every head
+    against the oracle."""
     prob = wl.make_problem(idx, device="cuda")
     grads = _fwd_bwd(ba, prob)
     for g_ in grads:
         assert bool(torch.isfinite(g_.float()).all())
     _check_invariants(prob, grads)
-    sub, heads = sub_heads(prob, groups)
-    host = [t.cpu() for t in (sub.q, sub.k, sub.v, sub.qb, sub.kb, sub.vb, sub.do, sub.dob)]
+    ref = oracle_rows_by_group(prob, backward=True)
     c = prob.cfg
-    _, dQ, dk, dv, dkb, dvb = orc.backward_rows(*host, prob.cu_seqlens.numpy(), prob.anchors.numpy(),
-                                                c.B, c.mode)
     dq, dkd, dvd, dqb, dkbd, dvbd = grads
     S = prob.S
-    gi = torch.as_tensor(groups, device="cuda")
-    hi = torch.as_tensor(heads, device="cuda")
-    assert max_abs(_np(dq.index_select(1, hi)), dQ[:S]) <= TOL_GRAD
-    assert max_abs(_np(dqb.index_select(2, hi)).reshape(-1, len(heads), c.d), dQ[S:]) <= TOL_GRAD
-    assert max_abs(_np(dkd.index_select(1, gi)), dk) <= TOL_GRAD
-    assert max_abs(_np(dvd.index_select(1, gi)), dv) <= TOL_GRAD
-    assert max_abs(_np(dkbd.index_select(2, gi)), dkb) <= TOL_GRAD
-    assert max_abs(_np(dvbd.index_select(2, gi)), dvb) <= TOL_GRAD
+    assert max_abs(_np(dq), ref["dQ"][:S]) <= TOL_GRAD
+    assert max_abs(_np(dqb).reshape(-1, c.Hq, c.d), ref["dQ"][S:]) <= TOL_GRAD
+    assert max_abs(_np(dkd), ref["dk"]) <= TOL_GRAD
+    assert max_abs(_np(dvd), ref["dv"]) <= TOL_GRAD
+    assert max_abs(_np(dkbd), ref["dkb"]) <= TOL_GRAD
+    assert max_abs(_np(dvbd), ref["dvb"]) <= TOL_GRAD
 
 
-@pytest.mark.parametrize("idx,n_rows,groups", [(3, 1024, [6]), (4, 256, [1])])
-def test_bwd_config_sampled(ba, idx, n_rows, groups):
-    """64K and 256K configs.  (1) Full random dO: dQ of sampled rows matches
-    the oracle (a row's dQ depends only on that row), gradient invariants hold.
-    (2) dO zero outside the sampled rows: then every dK, dV is exactly the
-    oracle's sum over those rows, checked for every key of the listed group."""
+@pytest.mark.parametrize("idx,group", [(3, 6), pytest.param(4, 1, marks=pytest.mark.slow)])
+def test_bwd_config_sampled(ba, idx, group):
+    """64K and 256K configs on 4096 seeded, stratified rows.  (1) Full random
+    dO: dQ of the sampled rows matches the oracle for every head (a row's dQ
+    depends only on that row), and the gradient invariants hold.  (2) dO zero
+    outside the sampled rows: then every dK, dV is exactly the oracle's sum
+    over those rows, checked for every key of one KV group."""
     prob = wl.make_problem(idx, device="cuda")
     c = prob.cfg
-    edges = [e[2] for e in orc.zigzag_chunks(prob.cu_seqlens.numpy(), c.R)]
-    rows = wl.sample_rows(prob.cu_seqlens, prob.anchors, c.B, n_rows, seed=idx, extra=edges).numpy()
+    rows = config_rows(prob, 4096, seed=idx)
+    assert len(rows) >= 4096
     S = prob.S
     grads = _fwd_bwd(ba, prob)
     _check_invariants(prob, grads)
-    sub, heads = sub_heads(prob, groups)
-    host = [t.cpu() for t in (sub.q, sub.k, sub.v, sub.qb, sub.kb, sub.vb, sub.do, sub.dob)]
-    r2, dQ, _, _, _, _ = orc.backward_rows(*host, prob.cu_seqlens.numpy(), prob.anchors.numpy(),
-                                           c.B, c.mode, rows=rows)
-    hi = torch.as_tensor(heads, device="cuda")
-    dq_all = torch.cat([grads[0].index_select(1, hi), grads[3].index_select(2, hi).reshape(-1, len(heads), c.d)])
-    assert max_abs(_np(dq_all[torch.as_tensor(r2, device="cuda")]), dQ) <= TOL_GRAD
-    del grads
+    dq_all = torch.cat([grads[0], grads[3].reshape(-1, c.Hq, c.d)])
+    got = _np(dq_all[torch.as_tensor(rows, device="cuda")])
+    del grads, dq_all
+    ref = oracle_rows_by_group(prob, rows, backward=True)
+    assert max_abs(got, ref["dQ"]) <= TOL_GRAD
+    del ref
     # sparse dO
     mask = torch.zeros(S + prob.Nb * c.B, dtype=torch.bool, device="cuda")
     mask[torch.as_tensor(rows, device="cuda")] = True
-    do = prob.do * mask[:S, None, None]
-    dob = prob.dob * mask[S:].view(prob.Nb, c.B)[..., None, None]
-    grads = _fwd_bwd(ba, prob, do, dob)
-    sub.do = do.index_select(1, hi)
-    sub.dob = dob.index_select(2, hi)
-    host = [t.cpu() for t in (sub.q, sub.k, sub.v, sub.qb, sub.kb, sub.vb, sub.do, sub.dob)]
-    r2, dQ, dk, dv, dkb, dvb = orc.backward_rows(*host, prob.cu_seqlens.numpy(), prob.anchors.numpy(),
-                                                 c.B, c.mode, rows=rows)
-    gi = torch.as_tensor(groups, device="cuda")
-    assert max_abs(_np(grads[1].index_select(1, gi)), dk) <= TOL_GRAD
-    assert max_abs(_np(grads[2].index_select(1, gi)), dv) <= TOL_GRAD
-    assert max_abs(_np(grads[4].index_select(2, gi)), dkb) <= TOL_GRAD
-    assert max_abs(_np(grads[5].index_select(2, gi)), dvb) <= TOL_GRAD
+    prob.do = prob.do * mask[:S, None, None]
+    prob.dob = prob.dob * mask[S:].view(prob.Nb, c.B)[..., None, None]
+    grads = _fwd_bwd(ba, prob)
+    ref = oracle_rows_by_group(prob, rows, groups=[group], backward=True)
+    gi = torch.as_tensor([group], device="cuda")
+    assert max_abs(_np(grads[1].index_select(1, gi)), ref["dk"]) <= TOL_GRAD
+    assert max_abs(_np(grads[2].index_select(1, gi)), ref["dv"]) <= TOL_GRAD
+    assert max_abs(_np(grads[4].index_select(2, gi)), ref["dkb"]) <= TOL_GRAD
+    assert max_abs(_np(grads[5].index_select(2, gi)), ref["dvb"]) <= TOL_GRAD

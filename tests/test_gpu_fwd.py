@@ -6,8 +6,8 @@ import torch
 
 import oracle as orc
 import workloads as wl
-from gpu_cases import (SMALL_CASES, TOL_LSE, TOL_O, attn_for, gather_rows, make_case, max_abs,
-                       oracle_fwd, sub_heads, to_device)
+from gpu_cases import (SMALL_CASES, TOL_LSE, TOL_O, attn_for, config_rows, gather_rows, make_case,
+                       max_abs, oracle_fwd, oracle_rows_by_group, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -122,40 +122,30 @@ def test_fused_fwd_config_tiny(ba):
     assert max_abs(lse.cpu().numpy(), L) <= TOL_LSE
 
 
-@pytest.mark.parametrize("idx,groups", [(1, [0, 5]), (2, [3])])
-def test_fused_fwd_config_full_rows(ba, idx, groups):
-    """Configs at 8K (chain) and 32K (block): every row, the query heads of
-    the listed KV groups (the oracle's cost), all heads computed on the GPU."""
-    prob = to_device(wl.make_problem(idx))
+@pytest.mark.parametrize("idx", [1, pytest.param(2, marks=pytest.mark.slow)])
+def test_fused_fwd_config_full_rows(ba, idx):
+    """Configs at 8K (chain) and 32K (block): every row and every query head
+    against the oracle."""
+    prob = to_device(wl.make_problem(idx, with_grad_inputs=False))
     o, ob, lse = _fused(ba, prob)
-    assert torch.isfinite(o.float()).all() and torch.isfinite(ob.float()).all()
-    assert torch.isfinite(lse).all()
-    sub, heads = sub_heads(prob, groups)
-    cpu_sub = wl.Problem(sub.cfg, sub.seed, sub.cu_seqlens, sub.anchors,
-                         *(t.cpu() for t in (sub.q, sub.k, sub.v, sub.qb, sub.kb, sub.vb)))
-    c = prob.cfg
-    rows, O, L = orc.forward_rows(cpu_sub.q, cpu_sub.k, cpu_sub.v, cpu_sub.qb, cpu_sub.kb, cpu_sub.vb,
-                                  prob.cu_seqlens.numpy(), prob.anchors.numpy(), c.B, c.mode)
-    got = gather_rows(o[:, heads], ob[:, :, heads], rows, prob.S)
-    assert max_abs(got, O) <= TOL_O
-    assert max_abs(lse[heads].cpu().numpy(), L) <= TOL_LSE
+    ref = oracle_rows_by_group(prob)
+    assert ref["heads"] == list(range(prob.cfg.Hq))
+    assert max_abs(gather_rows(o, ob, ref["rows"], prob.S), ref["O"]) <= TOL_O
+    assert max_abs(lse.cpu().numpy(), ref["L"]) <= TOL_LSE
 
 
-@pytest.mark.parametrize("idx,n_rows,groups", [(3, 2048, [0, 7]), (4, 512, [2])])
-def test_fused_fwd_config_sampled_rows(ba, idx, n_rows, groups):
-    """64K and 256K configs: seeded, stratified sample of rows (document ends,
-    zigzag chunk edges, anchors at document ends), heads of the listed groups."""
+@pytest.mark.parametrize("idx", [3, pytest.param(4, marks=pytest.mark.slow)])
+def test_fused_fwd_config_sampled_rows(ba, idx):
+    """64K and 256K configs: 4096 seeded, stratified rows (plus document ends,
+    zigzag chunk edges and anchors at document ends), every query head."""
     prob = wl.make_problem(idx, device="cuda", with_grad_inputs=False)
     o, ob, lse = _fused(ba, prob)
-    c = prob.cfg
-    edges = [e[2] for e in orc.zigzag_chunks(prob.cu_seqlens.numpy(), c.R)]
-    rows = wl.sample_rows(prob.cu_seqlens, prob.anchors, c.B, n_rows, seed=idx, extra=edges).numpy()
-    sub, heads = sub_heads(prob, groups)
-    host = [t.cpu() for t in (sub.q, sub.k, sub.v, sub.qb, sub.kb, sub.vb)]
-    r2, O, L = orc.forward_rows(*host, prob.cu_seqlens.numpy(), prob.anchors.numpy(), c.B, c.mode,
-                                rows=rows)
-    got = gather_rows(o[:, heads], ob[:, :, heads], r2, prob.S)
-    assert max_abs(got, O) <= TOL_O
-    assert max_abs(lse[heads][:, torch.as_tensor(r2, device="cuda")].cpu().numpy(), L) <= TOL_LSE
+    rows = config_rows(prob, 4096, seed=idx)
+    assert len(rows) >= 4096
+    ref = oracle_rows_by_group(prob, rows)
+    assert ref["heads"] == list(range(prob.cfg.Hq))
+    assert max_abs(gather_rows(o, ob, rows, prob.S), ref["O"]) <= TOL_O
+    assert max_abs(lse[:, torch.as_tensor(rows, device="cuda")].cpu().numpy(), ref["L"]) <= TOL_LSE
     # every output written (canaries were NaN)
     assert bool(torch.isfinite(lse).all())
+    assert bool(torch.isfinite(o.float()).all()) and bool(torch.isfinite(ob.float()).all())
