@@ -38,6 +38,7 @@ METRIC = "branch-attn fwd+bwd useful TFLOPS at 64K tokens; % of B200 BF16 dense 
 WORKLOAD_INDEX = 3  # the 64K-token EAGLE-3 configuration (the headline)
 REFERENCE_PREFIX = 640  # tokens per reference-arm step: about 3 s of oracle time
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0  # B200 dense bf16, nominal
 
 
 def load_peaks():
@@ -215,10 +216,11 @@ def workload_config(world: int, index: int = WORKLOAD_INDEX) -> dict:
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
-# DRAM traffic of one launch of a kernel on the 64K workload, from the ncu
-# capture summarised in profiles/ncu_tensor_kernels_eagle3_8k.md (8K case,
-# scaled to the 64K launch by its slot count), valid for the kernel source it
-# was taken on: reported only while that source file is unchanged.
+# DRAM traffic of one launch of a kernel on the 64K workload, from an ncu
+# capture of the same kernel on the 8K configuration (dram__bytes_read.sum +
+# dram__bytes_write.sum, scaled to the 64K launch by its slot count), valid
+# for the kernel source it was taken on: reported only while that source file
+# is unchanged.
 KERNEL_TRAFFIC = {
     "bwd_dkdv": {"bytes_per_launch": 4.911e9, "source": "bwd_dkdv.cu",
                  "sha1": "0258f84042c1f140d19577fe2843802c00db0e36"},
@@ -354,6 +356,7 @@ def run_gpu(args):
     dom_ms = per_kernel[dom]["ms_per_launch"]
     achieved = kernel_flops(dom, cfg.d, P, cfg.Hq) / (dom_ms / 1e3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     launches = sum(v[1] for v in prof.values())
 
     # ------------------------------------------------------------ end to end (host buffers)
@@ -428,6 +431,9 @@ def run_gpu(args):
         "value": round(value, 2),
         "unit": "TFLOPS",
         "pct_of_peak": round(100.0 * value / (peak * world), 2),
+        "pct_of_peak_basis": f"{peak_src} sustained cuBLAS bf16 rate, {peak} TF/s per GPU",
+        "pct_of_burst_peak": round(100.0 * value / (burst * world), 2),
+        "pct_of_datasheet_peak": round(100.0 * value / (DATASHEET_BF16_TFLOPS * world), 2),
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
