@@ -30,7 +30,7 @@ EXPORTED = (
     "ba_workspace_size", "ba_main_fwd", "ba_branch_fwd", "ba_lse_merge", "ba_fused_fwd",
     "ba_bwd", "ba_status_string", "ba_sync_status", "ba_plan_stats", "ba_profile_enable",
     "ba_profile_collect", "ba_last_error_word", "ba_fused_fwd_noalloc", "ba_plan_rank_work",
-    "ba_plan_fwd_pairs",
+    "ba_plan_fwd_pairs", "ba_plan_prepare", "ba_clear_cache", "ba_plan_cache_stats",
 )
 
 
@@ -89,6 +89,12 @@ def lib() -> ctypes.CDLL:
         L.ba_plan_rank_work.restype = ctypes.c_int
         L.ba_plan_fwd_pairs.argtypes = [P, ctypes.POINTER(ctypes.c_int32), ctypes.c_int64]
         L.ba_plan_fwd_pairs.restype = ctypes.c_int64
+        L.ba_plan_prepare.argtypes = [P, ctypes.POINTER(ctypes.c_double)]
+        L.ba_plan_prepare.restype = ctypes.c_int
+        L.ba_clear_cache.argtypes = []
+        L.ba_clear_cache.restype = None
+        L.ba_plan_cache_stats.argtypes = [i64p, i64p, i64p]
+        L.ba_plan_cache_stats.restype = None
         L.ba_last_error_word.argtypes = []
         L.ba_last_error_word.restype = ctypes.c_uint32
         L.ba_profile_enable.argtypes = [i32]
@@ -102,6 +108,18 @@ def lib() -> ctypes.CDLL:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
+
+
+def clear_cache() -> None:
+    """Drop every cached host plan (ba_clear_cache)."""
+    lib().ba_clear_cache()
+
+
+def plan_cache_stats() -> dict:
+    """{entries, hits, misses} of the library's host plan cache."""
+    e, h, m = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    lib().ba_plan_cache_stats(ctypes.byref(e), ctypes.byref(h), ctypes.byref(m))
+    return {"entries": e.value, "hits": h.value, "misses": m.value}
 
 
 def status_string(status: int) -> str:

@@ -93,6 +93,14 @@ class BranchAttention:
                                        ctypes.byref(b), ctypes.byref(c)), "ba_plan_stats")
         return {"row_tiles": a.value, "tile_pairs": b.value, "visible_pairs": c.value}
 
+    def prepare(self) -> float:
+        """Build (or find) this problem's host plan in the library's cache;
+        returns the host milliseconds building it took (ba_plan_prepare)."""
+        ms = ctypes.c_double()
+        check(_abi.lib().ba_plan_prepare(ctypes.byref(self._problem()), ctypes.byref(ms)),
+              "ba_plan_prepare")
+        return ms.value
+
     def rank_work(self):
         """(row tile, main key tile) pairs owned by each of the R virtual ranks."""
         buf = (ctypes.c_int64 * self.R)()

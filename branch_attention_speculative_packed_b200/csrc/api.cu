@@ -2,11 +2,16 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <chrono>
 #include <cmath>
 #include <cstring>
+#include <list>
 #include <map>
+#include <memory>
 #include <mutex>
 #include <string>
+#include <unordered_map>
+#include <utility>
 #include <vector>
 
 #include "../../include/ba.h"
@@ -121,27 +126,144 @@ float scale_of(const ba_problem* p) {
   return p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->d));
 }
 
-// Uploads the plan into the workspace and scatters the row table.
-ba_status stage_plan(const ba_problem* p, const Plan& plan, const WorkspaceLayout& w,
-                     cudaStream_t st) {
-  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
-  const size_t nt = plan.tiles.size();
-  if (nt == 0) return BA_OK;
-  if (cudaMemcpyAsync(ws + w.tiles_off, plan.tiles.data(), nt * sizeof(TileDesc),
-                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(ws + w.order_off, plan.order.data(), nt * sizeof(int32_t),
-                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(ws + w.pairs_off, plan.pairs.data(), plan.pairs.size() * sizeof(int32_t),
-                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(ws + w.chunks_off, plan.chunks_dev.data(),
-                      plan.chunks_dev.size() * sizeof(ChunkDev), cudaMemcpyHostToDevice,
-                      st) != cudaSuccess ||
-      cudaMemsetAsync(ws + w.rows_off, 0xFF, size_t(w.n_slots) * sizeof(int32_t), st) !=
-          cudaSuccess ||
+// ------------------------------------------------------------------ plan cache
+// A host plan depends only on the problem's sizes and on the contents of its
+// host cu_seqlens and anchors.  Plans are kept, least recently used first
+// out, so repeated calls on one packing (every training step, forward and
+// backward) plan once.  Each entry also holds the bytes the workspace needs
+// from the host, in pageable memory and, once a device call has used it, in a
+// page-locked copy so the upload is a plain asynchronous copy.
+constexpr size_t kPlanCacheCapacity = 16;
+
+struct CachedPlan {
+  Plan plan;
+  WorkspaceLayout ws_fwd, ws_bwd;
+  std::vector<uint8_t> image;  // workspace bytes [tiles_off, rows_off), same for both layouts
+  double build_ms = 0.0;       // host time it took to build this entry
+  std::mutex mu;               // guards the fields below
+  void* pinned = nullptr;      // page-locked copy of `image`
+  bool pinned_failed = false;
+  // one event per stream that uploaded from `pinned`: its last upload there
+  std::vector<std::pair<cudaStream_t, cudaEvent_t>> uploads;
+
+  ~CachedPlan() {
+    // The page-locked copy goes only after every upload from it has finished.
+    for (auto& u : uploads) {
+      cudaEventSynchronize(u.second);
+      cudaEventDestroy(u.second);
+    }
+    if (pinned) cudaFreeHost(pinned);
+  }
+};
+
+struct PlanCache {
+  std::mutex mu;
+  std::list<std::pair<std::string, std::shared_ptr<CachedPlan>>> lru;  // most recent first
+  std::unordered_map<std::string, decltype(lru)::iterator> index;
+  int64_t hits = 0, misses = 0;
+};
+
+// Never destroyed: entries may hold CUDA resources, which must not be
+// released from a static destructor after the runtime has shut down.
+PlanCache& plan_cache() {
+  static PlanCache* c = new PlanCache;
+  return *c;
+}
+
+std::string plan_key(const ba_problem* p) {
+  const int32_t dims[] = {p->S, p->ndoc, p->Hq, p->Hkv, p->d, p->Nb, p->Nb > 0 ? p->B : 0,
+                          p->mode, p->R};
+  std::string key(reinterpret_cast<const char*>(dims), sizeof(dims));
+  key.append(reinterpret_cast<const char*>(p->cu_seqlens_h), size_t(p->ndoc + 1) * sizeof(int32_t));
+  if (p->Nb > 0) key.append(reinterpret_cast<const char*>(p->anchors_h), size_t(p->Nb) * sizeof(int32_t));
+  return key;
+}
+
+// The cached plan of a validated problem (built on a miss).  Without
+// `may_evict` a miss never drops older entries (dropping one may free its
+// page-locked copy); the next call that may evict trims the cache.
+std::shared_ptr<CachedPlan> get_plan(const ba_problem* p, bool may_evict = true) {
+  PlanCache& c = plan_cache();
+  std::string key = plan_key(p);
+  {
+    std::lock_guard<std::mutex> lk(c.mu);
+    auto it = c.index.find(key);
+    if (it != c.index.end()) {
+      c.lru.splice(c.lru.begin(), c.lru, it->second);
+      ++c.hits;
+      return it->second->second;
+    }
+  }
+  auto e = std::make_shared<CachedPlan>();
+  const auto t0 = std::chrono::steady_clock::now();
+  build_plan(p, &e->plan);
+  build_kv_plan(p, &e->plan);
+  e->ws_fwd = workspace_layout(p, e->plan, BA_WS_FWD);
+  e->ws_bwd = workspace_layout(p, e->plan, BA_WS_BWD);
+  build_image(e->plan, e->ws_fwd, &e->image);
+  e->build_ms = std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t0).count();
+  std::vector<std::shared_ptr<CachedPlan>> evicted;  // released after the lock
+  std::lock_guard<std::mutex> lk(c.mu);
+  ++c.misses;
+  auto it = c.index.find(key);
+  if (it != c.index.end()) return it->second->second;  // built concurrently by another caller
+  c.lru.emplace_front(key, e);
+  c.index.emplace(std::move(key), c.lru.begin());
+  while (may_evict && c.lru.size() > kPlanCacheCapacity) {
+    c.index.erase(c.lru.back().first);
+    evicted.push_back(std::move(c.lru.back().second));
+    c.lru.pop_back();
+  }
+  return e;
+}
+
+// Uploads the plan into the workspace and scatters the row table.  With
+// `pinned_ok` the bytes come from the entry's page-locked copy (made on first
+// use); otherwise straight from pageable memory.
+ba_status stage_plan(const ba_problem* p, CachedPlan& e, const WorkspaceLayout& w, void* workspace,
+                     bool pinned_ok, cudaStream_t st) {
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (e.plan.tiles.empty()) return BA_OK;
+  const size_t n = e.image.size();
+  const void* src = e.image.data();
+  cudaEvent_t* done = nullptr;
+  std::unique_lock<std::mutex> lk(e.mu, std::defer_lock);
+  if (pinned_ok) {
+    lk.lock();
+    if (!e.pinned && !e.pinned_failed) {
+      void* h = nullptr;
+      if (cudaHostAlloc(&h, n, cudaHostAllocPortable) == cudaSuccess && h) {
+        std::memcpy(h, e.image.data(), n);
+        e.pinned = h;
+      } else {
+        cudaGetLastError();  // not sticky; fall back to the pageable copy
+        e.pinned_failed = true;
+      }
+    }
+    if (e.pinned) {
+      src = e.pinned;
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone) {
+        for (auto& u : e.uploads)
+          if (u.first == st) done = &u.second;
+        if (!done) {
+          cudaEvent_t ev;
+          if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return BA_ERR_CUDA;
+          e.uploads.emplace_back(st, ev);
+          done = &e.uploads.back().second;
+        }
+      }
+    }
+  }
+  if (cudaMemcpyAsync(ws + w.tiles_off, src, n, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return BA_ERR_CUDA;
+  if (done && cudaEventRecord(*done, st) != cudaSuccess) return BA_ERR_CUDA;
+  if (lk.owns_lock()) lk.unlock();
+  if (cudaMemsetAsync(ws + w.rows_off, 0xFF, size_t(w.n_slots) * sizeof(int32_t), st) != cudaSuccess ||
       cudaMemsetAsync(ws + w.counters_off, 0, 4 * sizeof(uint32_t), st) != cudaSuccess)
     return BA_ERR_CUDA;
   ProfScope prof("plan_rows", st);
-  if (launch_plan_rows(p->cu_seqlens_d, p->ndoc, p->anchors_d, p->S, p->Nb, plan.B,
+  if (launch_plan_rows(p->cu_seqlens_d, p->ndoc, p->anchors_d, p->S, p->Nb, e.plan.B,
                        reinterpret_cast<const ChunkDev*>(ws + w.chunks_off),
                        reinterpret_cast<int32_t*>(ws + w.rows_off), w.n_slots,
                        st) != cudaSuccess)
@@ -149,15 +271,19 @@ ba_status stage_plan(const ba_problem* p, const Plan& plan, const WorkspaceLayou
   return BA_OK;
 }
 
-ba_status check_workspace(const ba_problem* p, const WorkspaceLayout& w) {
-  if (!p->workspace || (reinterpret_cast<uintptr_t>(p->workspace) & 255u) != 0)
-    return BA_ERR_WORKSPACE;
-  if (p->workspace_bytes < w.total) return BA_ERR_WORKSPACE;
+ba_status check_workspace(const void* ws, size_t bytes, const WorkspaceLayout& w) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BA_ERR_WORKSPACE;
+  if (bytes < w.total) return BA_ERR_WORKSPACE;
   return BA_OK;
 }
 
+// The forward (fused or main component only).  `scratch` / `scratch_bytes`
+// replace the caller's workspace when set (the no-allocation entry point);
+// there a plan too large for the scratch is refused with `too_big` before
+// anything is enqueued, and the plan is uploaded from pageable memory.
 ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void* ob, float* lse,
-                  cudaStream_t st) {
+                  cudaStream_t st, void* scratch = nullptr, size_t scratch_bytes = 0,
+                  ba_status too_big = BA_ERR_WORKSPACE) {
   ba_status s = validate(p, true);
   if (s != BA_OK) return s;
   if (!lse || !aligned16(lse)) return BA_ERR_INVALID_ARG;
@@ -166,13 +292,20 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   } else if (!o_part || !aligned16(o_part)) {
     return BA_ERR_INVALID_ARG;
   }
+  const std::shared_ptr<CachedPlan> cp = get_plan(p, scratch == nullptr);
+  const Plan& plan = cp->plan;
+  const WorkspaceLayout& w = cp->ws_fwd;
+  void* ws_ptr = scratch ? scratch : p->workspace;
+  if (scratch) {
+    if (w.total > scratch_bytes) return too_big;
+  } else if ((s = check_workspace(p->workspace, p->workspace_bytes, w)) != BA_OK) {
+    return s;
+  }
+  const int64_t items = int64_t(plan.pairs.size() / 2) * p->Hq;
+  if (items > 0x7fffffff) return BA_ERR_UNSUPPORTED;
   DeviceInfo di;
   if ((s = device_info(&di)) != BA_OK) return s;
-  Plan plan;
-  build_plan(p, &plan);
-  const WorkspaceLayout w = workspace_layout(p, plan, BA_WS_FWD);
-  if ((s = check_workspace(p, w)) != BA_OK) return s;
-  if ((s = stage_plan(p, plan, w, st)) != BA_OK) return s;
+  if ((s = stage_plan(p, *cp, w, ws_ptr, scratch == nullptr, st)) != BA_OK) return s;
 
   const int64_t nbr_rows = int64_t(p->Nb) * plan.B;
   const int64_t rows = int64_t(p->S) + nbr_rows;
@@ -187,7 +320,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
       encode_2d(&maps.vb, vb, nb_rows_map, int64_t(p->Hkv) * p->d, 128) != BA_OK)
     return BA_ERR_CUDA;
 
-  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  uint8_t* ws = static_cast<uint8_t*>(ws_ptr);
   FwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.q = static_cast<const __nv_bfloat16*>(p->q);
@@ -203,8 +336,6 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   a.Hq = p->Hq;
   a.G = p->Hq / p->Hkv;
   a.d = p->d;
-  const int64_t items = int64_t(plan.pairs.size() / 2) * p->Hq;
-  if (items > 0x7fffffff) return BA_ERR_UNSUPPORTED;
   a.n_items = static_cast<int>(items);
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.with_branch = fused && p->Nb > 0 ? 1 : 0;
@@ -232,44 +363,68 @@ extern "C" {
 size_t ba_workspace_size(const ba_problem* p, int which) {
   if (validate(p, false) != BA_OK) return 0;
   if (which != BA_WS_FWD && which != BA_WS_BWD) return 0;
-  Plan plan;
-  build_plan(p, &plan);
-  return workspace_layout(p, plan, which).total;
+  const std::shared_ptr<CachedPlan> cp = get_plan(p);
+  return (which == BA_WS_FWD ? cp->ws_fwd : cp->ws_bwd).total;
 }
 
 ba_status ba_plan_stats(const ba_problem* p, int64_t* n_row_tiles, int64_t* n_tile_pairs,
                         int64_t* n_visible_pairs) {
   ba_status s = validate(p, false);
   if (s != BA_OK) return s;
-  Plan plan;
-  build_plan(p, &plan);
-  if (n_row_tiles) *n_row_tiles = static_cast<int64_t>(plan.tiles.size());
-  if (n_tile_pairs) *n_tile_pairs = plan.n_tile_pairs;
-  if (n_visible_pairs) *n_visible_pairs = plan.n_visible_pairs;
+  const std::shared_ptr<CachedPlan> cp = get_plan(p);
+  if (n_row_tiles) *n_row_tiles = static_cast<int64_t>(cp->plan.tiles.size());
+  if (n_tile_pairs) *n_tile_pairs = cp->plan.n_tile_pairs;
+  if (n_visible_pairs) *n_visible_pairs = cp->plan.n_visible_pairs;
   return BA_OK;
 }
 
 int ba_plan_rank_work(const ba_problem* p, int64_t* pairs, int cap) {
   ba_status s = validate(p, false);
   if (s != BA_OK) return s;
-  Plan plan;
-  build_plan(p, &plan);
+  const std::shared_ptr<CachedPlan> cp = get_plan(p);
   for (int r = 0; r < cap && r < p->R; ++r)
-    if (pairs) pairs[r] = plan.rank_pairs[r];
+    if (pairs) pairs[r] = cp->plan.rank_pairs[r];
   return p->R;
 }
 
 int64_t ba_plan_fwd_pairs(const ba_problem* p, int32_t* tiles, int64_t cap) {
   ba_status s = validate(p, false);
   if (s != BA_OK) return s;
-  Plan plan;
-  build_plan(p, &plan);
+  const std::shared_ptr<CachedPlan> cp = get_plan(p);
+  const Plan& plan = cp->plan;
   const int64_t n = static_cast<int64_t>(plan.pairs.size() / 2);
   for (int64_t i = 0; tiles && i < cap && i < n; ++i) {
     tiles[2 * i] = plan.pairs[2 * i];
     tiles[2 * i + 1] = plan.pairs[2 * i + 1];
   }
   return n;
+}
+
+ba_status ba_plan_prepare(const ba_problem* p, double* build_ms) {
+  ba_status s = validate(p, false);
+  if (s != BA_OK) return s;
+  const std::shared_ptr<CachedPlan> cp = get_plan(p);
+  if (build_ms) *build_ms = cp->build_ms;
+  return BA_OK;
+}
+
+void ba_clear_cache(void) {
+  PlanCache& c = plan_cache();
+  std::list<std::pair<std::string, std::shared_ptr<CachedPlan>>> dropped;
+  {
+    std::lock_guard<std::mutex> lk(c.mu);
+    c.index.clear();
+    dropped.swap(c.lru);
+  }
+  // entries still used by a call in progress go when that call returns
+}
+
+void ba_plan_cache_stats(int64_t* entries, int64_t* hits, int64_t* misses) {
+  PlanCache& c = plan_cache();
+  std::lock_guard<std::mutex> lk(c.mu);
+  if (entries) *entries = static_cast<int64_t>(c.lru.size());
+  if (hits) *hits = c.hits;
+  if (misses) *misses = c.misses;
 }
 
 ba_status ba_main_fwd(const ba_problem* p, float* o_part, float* lse_part, ba_stream_t stream) {
@@ -347,27 +502,19 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   DeviceInfo di;
   if ((s = device_info(&di)) != BA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  Plan plan;
-  build_plan(p, &plan);
-  build_kv_plan(p, &plan);
-  const WorkspaceLayout w = workspace_layout(p, plan, BA_WS_BWD);
-  if ((s = check_workspace(p, w)) != BA_OK) return s;
-  if ((s = stage_plan(p, plan, w, st)) != BA_OK) return s;
-  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  const std::shared_ptr<CachedPlan> cp = get_plan(p);
+  const Plan& plan = cp->plan;
+  const WorkspaceLayout& w = cp->ws_bwd;
+  if ((s = check_workspace(p->workspace, p->workspace_bytes, w)) != BA_OK) return s;
   const size_t nkv = plan.kv_items.size();
-  if (nkv > 0 &&
-      (cudaMemcpyAsync(ws + w.kv_items_off, plan.kv_items.data(), nkv * sizeof(KvItem),
-                       cudaMemcpyHostToDevice, st) != cudaSuccess ||
-       cudaMemcpyAsync(ws + w.kv_order_off, plan.kv_order.data(),
-                       plan.kv_order.size() * sizeof(int32_t), cudaMemcpyHostToDevice,
-                       st) != cudaSuccess))
-    return BA_ERR_CUDA;
-  const int64_t rows = int64_t(p->S) + int64_t(p->Nb) * plan.B;
-  const float scale = scale_of(p);
-  const int G = p->Hq / p->Hkv;
   const int64_t items_q = int64_t(plan.tiles.size()) * p->Hq;
   const int64_t items_kv = int64_t(nkv) * p->Hkv;
   if (items_q > 0x7fffffff || items_kv > 0x7fffffff) return BA_ERR_UNSUPPORTED;
+  if ((s = stage_plan(p, *cp, w, p->workspace, true, st)) != BA_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  const int64_t rows = int64_t(p->S) + int64_t(p->Nb) * plan.B;
+  const float scale = scale_of(p);
+  const int G = p->Hq / p->Hkv;
 
   // 1. pre-pass
   PrepArgs pa;
@@ -599,13 +746,9 @@ ba_status static_scratch(void** out) {
 
 extern "C" ba_status ba_fused_fwd_noalloc(const ba_problem* p, void* o, void* ob, float* lse,
                                            ba_stream_t stream) {
-  ba_status s = validate(p, true);
-  if (s != BA_OK) return s;
-  if (ba_workspace_size(p, BA_WS_FWD) > BA_STATIC_SCRATCH_BYTES) return BA_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
-  if ((s = static_scratch(&scratch)) != BA_OK) return s;
-  ba_problem q = *p;
-  q.workspace = scratch;
-  q.workspace_bytes = BA_STATIC_SCRATCH_BYTES;
-  return ba_fused_fwd(&q, o, ob, lse, stream);
+  ba_status s = static_scratch(&scratch);
+  if (s != BA_OK) return s;
+  return run_fwd(p, true, nullptr, o, ob, lse, reinterpret_cast<cudaStream_t>(stream), scratch,
+                 BA_STATIC_SCRATCH_BYTES, BA_ERR_SCRATCH_LIMIT);
 }

@@ -3,6 +3,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstring>
 #include <numeric>
 #include <utility>
 
@@ -272,6 +273,10 @@ void build_kv_plan(const ba_problem* p, Plan* plan) {
 }
 
 WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int which) {
+  // Layout: counters | tiles | order | chunks | pairs | kv items | kv order |
+  // rows | backward buffers.  Everything in [tiles_off, rows_off) comes from
+  // the host plan (one upload image); the row table is scattered on the
+  // device; the rest is written by the kernels.
   WorkspaceLayout w;
   const size_t nt = plan.tiles.size();
   w.n_slots = int64_t(nt) * kRowsPerTile;
@@ -284,19 +289,17 @@ WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int whic
   off = align_up(off + nt * sizeof(int32_t), 256);
   w.chunks_off = off;
   off = align_up(off + plan.chunks_dev.size() * sizeof(ChunkDev), 256);
+  w.pairs_off = off;
+  off = align_up(off + plan.pairs.size() * sizeof(int32_t), 256);
+  w.kv_items_off = off;
+  off = align_up(off + plan.kv_items.size() * sizeof(KvItem), 256);
+  w.kv_order_off = off;
+  off = align_up(off + plan.kv_order.size() * sizeof(int32_t), 256);
   w.rows_off = off;
   off = align_up(off + size_t(w.n_slots) * sizeof(int32_t), 256);
-  w.pairs_off = off;
-  off = align_up(off + 2 * nt * sizeof(int32_t), 256);
   if (which == BA_WS_BWD) {
     const size_t rows = size_t(p->S) + size_t(p->Nb) * (p->Nb > 0 ? p->B : 0);
     const size_t slots = size_t(w.n_slots);
-    // key tiles: one per 128 keys of each document, at most S/128 + ndoc
-    const size_t nkv = size_t(p->S) / kKeysPerTile + p->ndoc;
-    w.kv_items_off = off;
-    off = align_up(off + nkv * sizeof(KvItem), 256);
-    w.kv_order_off = off;
-    off = align_up(off + nkv * p->Hkv * sizeof(int32_t), 256);
     w.qg_off = off;
     off = align_up(off + slots * p->Hq * p->d * 2, 1024);
     w.dog_off = off;
@@ -314,6 +317,20 @@ WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int whic
   }
   w.total = off;
   return w;
+}
+
+void build_image(const Plan& plan, const WorkspaceLayout& w, std::vector<uint8_t>* image) {
+  image->assign(w.rows_off - w.tiles_off, 0);
+  uint8_t* base = image->data() - w.tiles_off;  // so that base + x_off addresses region x
+  auto put = [&](size_t off, const void* src, size_t bytes) {
+    if (bytes) std::memcpy(base + off, src, bytes);
+  };
+  put(w.tiles_off, plan.tiles.data(), plan.tiles.size() * sizeof(TileDesc));
+  put(w.order_off, plan.order.data(), plan.order.size() * sizeof(int32_t));
+  put(w.chunks_off, plan.chunks_dev.data(), plan.chunks_dev.size() * sizeof(ChunkDev));
+  put(w.pairs_off, plan.pairs.data(), plan.pairs.size() * sizeof(int32_t));
+  put(w.kv_items_off, plan.kv_items.data(), plan.kv_items.size() * sizeof(KvItem));
+  put(w.kv_order_off, plan.kv_order.data(), plan.kv_order.size() * sizeof(int32_t));
 }
 
 }  // namespace ba

@@ -75,4 +75,9 @@ struct WorkspaceLayout {
 };
 WorkspaceLayout workspace_layout(const ba_problem* p, const Plan& plan, int which);
 
+// The host bytes of the workspace region [tiles_off, rows_off): tiles, order,
+// chunks, pairs and the dK/dV key-tile list, at their layout offsets.  The
+// region is the same for the forward and the backward layout.
+void build_image(const Plan& plan, const WorkspaceLayout& w, std::vector<uint8_t>* image);
+
 }  // namespace ba

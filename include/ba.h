@@ -40,7 +40,8 @@
  *   - scale <= 0 selects 1/sqrt(d).
  *   - Ownership: the caller owns every buffer, including the workspace whose
  *     size ba_workspace_size() returns.  The library allocates no device
- *     memory on these paths and keeps no per-call state.
+ *     memory on these paths.  Its only state between calls is a cache of host
+ *     plans (see ba_plan_prepare / ba_clear_cache).
  *   - Work is enqueued on `stream` and runs asynchronously.  Argument errors are
  *     detected on the host before anything is enqueued.  A device-side bounded
  *     wait that expires sets a device error word and the kernel returns;
@@ -182,7 +183,11 @@ BA_API ba_status ba_fused_fwd(const ba_problem* p, void* o, void* ob, float* lse
  *     reset to -1 on every call), so nothing relies on earlier contents.
  *     Calls whose work overlaps on the GPU (different streams, or different
  *     host threads, on the same device) race on the array: serialise them.
- *   - Allocates no device memory and calls no allocating library routine. */
+ *   - Allocates no device memory and calls no allocating library routine.
+ *     The host plan comes from the plan cache (built on the host if absent;
+ *     this call never evicts an entry) and is uploaded into the array with a
+ *     copy from pageable host memory on every call, so the call returns only
+ *     after the driver has staged those bytes. */
 #define BA_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
 BA_API ba_status ba_fused_fwd_noalloc(const ba_problem* p, void* o, void* ob, float* lse,
                                       ba_stream_t stream);
@@ -198,6 +203,33 @@ BA_API ba_status ba_fused_fwd_noalloc(const ba_problem* p, void* o, void* ob, fl
 BA_API ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float* lse,
                  const void* dout, const void* doutb, void* dq, void* dk, void* dv,
                  void* dqb, void* dkb, void* dvb, ba_stream_t stream);
+
+/* Plan cache (no counterpart on the pages; the plan is this library's own
+ * work list).  Every entry point plans on the host from cu_seqlens_h and
+ * anchors_h: the zigzag split, row tiles, their order and the key tiles of the
+ * backward.  Plans are cached, keyed by the problem's sizes (S, ndoc, Hq,
+ * Hkv, d, Nb, B, mode, R) and the contents of cu_seqlens_h and anchors_h, so
+ * the forward and backward of one packing, and later steps over the same
+ * packing, plan once.  The cache keeps the 16 most recently used plans.  A
+ * cached plan also keeps a page-locked copy of the bytes a device call
+ * uploads into the workspace (made by the first device call that uses it), so
+ * that upload is one asynchronous copy; an entry's page-locked copy is freed
+ * only after every upload from it has finished.
+ *
+ * ba_plan_prepare builds (or finds) the plan of a problem without touching a
+ * GPU and reports, in *build_ms (may be NULL), how long building it took on
+ * the host.  It returns BA_ERR_INVALID_ARG / BA_ERR_UNSUPPORTED as
+ * ba_plan_stats does.  Host only; reads cu_seqlens_h and anchors_h. */
+BA_API ba_status ba_plan_prepare(const ba_problem* p, double* build_ms);
+
+/* Drops every cached plan (an entry still in use by a call in progress goes
+ * when that call returns).  Freeing a page-locked copy waits for the uploads
+ * from it to finish. */
+BA_API void ba_clear_cache(void);
+
+/* Number of cached plans and the cache's hit and miss counts since the
+ * library was loaded (any argument may be NULL).  Host only. */
+BA_API void ba_plan_cache_stats(int64_t* entries, int64_t* hits, int64_t* misses);
 
 /* Static description of a status code. */
 BA_API const char* ba_status_string(ba_status s);

@@ -207,3 +207,46 @@ def test_zigzag_split_balances_causal_work(ba, R):
     w = a.rank_work()
     assert len(w) == R and sum(w) == a.plan_stats()["tile_pairs"]
     assert max(w) / min(w) < 1.05, w
+
+
+def test_plan_cache_reuses_and_clears(ba):
+    """A second call with identical sizes and packing contents reuses the
+    cached plan; a different packing (same sizes) misses; ba_clear_cache drops
+    every entry, after which the same problem plans again."""
+    ba.clear_cache()
+    assert ba.plan_cache_stats()["entries"] == 0
+    a = _attn(ba, [0, 300, 700], [5, 299, 301, 650])
+    s0 = ba.plan_cache_stats()
+    first = a.plan_stats()
+    s1 = ba.plan_cache_stats()
+    assert (s1["misses"], s1["hits"], s1["entries"]) == (s0["misses"] + 1, s0["hits"], 1)
+    assert a.plan_stats() == first
+    a.workspace_size(ba.BA_WS_BWD)  # forward and backward share the entry
+    s2 = ba.plan_cache_stats()
+    assert (s2["misses"], s2["hits"], s2["entries"]) == (s1["misses"], s1["hits"] + 2, 1)
+    # same sizes, different anchor contents: a different plan
+    b = _attn(ba, [0, 300, 700], [5, 299, 302, 650])
+    b.plan_stats()
+    s3 = ba.plan_cache_stats()
+    assert (s3["misses"], s3["entries"]) == (s2["misses"] + 1, 2)
+    assert a.prepare() >= 0.0
+    ba.clear_cache()
+    assert ba.plan_cache_stats()["entries"] == 0
+    assert a.plan_stats() == first
+    s4 = ba.plan_cache_stats()
+    assert s4["misses"] == s3["misses"] + 1 and s4["entries"] == 1
+    ba.clear_cache()
+
+
+def test_plan_cache_keeps_the_16_most_recent(ba):
+    ba.clear_cache()
+    probs = [_attn(ba, [0, 100 + i], [i]) for i in range(20)]
+    for p in probs:
+        p.plan_stats()
+    assert ba.plan_cache_stats()["entries"] == 16
+    before = ba.plan_cache_stats()
+    probs[-1].plan_stats()   # most recent: still cached
+    assert ba.plan_cache_stats()["hits"] == before["hits"] + 1
+    probs[0].plan_stats()    # least recent: evicted, plans again
+    assert ba.plan_cache_stats()["misses"] == before["misses"] + 1
+    ba.clear_cache()
