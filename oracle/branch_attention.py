@@ -29,6 +29,13 @@ up to rounding order, plain masked softmax attention over the concatenated
   t = 0..B-1.  Row (b, t) sees main keys j in [s(a_b), a_b] and branch keys
   (b, u) with u <= t (CHAIN, EAGLE-3 training-time test) or all u < B (BLOCK,
   DFlash-style block draft);
+* BITMASK (a generic per-branch mask, the form DSpark's Markov head needs;
+  the pages do not spell that mask out): row (b, t) sees branch key (b, u)
+  iff bit u of branch_mask[b, t] is set (branch_mask uint64 [Nb, B]);
+* optional main-prefix window W > 0 (the pages call the recipe independent of
+  the draft architecture; windowed drafts are one such variant): a row whose
+  last visible main key is l sees only main keys [max(s(l), l - W + 1), l];
+  branch keys are unaffected; W <= 0 means no window;
 * main rows never see branch keys; no branch sees another branch's keys;
 * s_ij = scale * <q_i, k_j>, scale = 1/sqrt(d) unless given;
   L_i = log sum_j exp(s_ij) (natural log), O_i = sum_j exp(s_ij - L_i) v_j;
@@ -71,6 +78,7 @@ import numpy as np
 
 CHAIN = 0
 BLOCK = 1
+BITMASK = 2
 
 
 # --------------------------------------------------------------------------
@@ -113,7 +121,32 @@ def row_limits(cu, anchors, B):
     return doc_start_of(cu, lim), lim
 
 
-def visible_mask(cu, anchors, B: int, mode: int) -> np.ndarray:
+def row_first_keys(starts, lim, window=0):
+    """First visible main key of each row: its document start, or with a
+    window W > 0 the later of that and lim - W + 1."""
+    starts = np.asarray(starts)
+    if window is None or window <= 0:
+        return starts
+    return np.maximum(starts, np.asarray(lim) - int(window) + 1)
+
+
+def branch_sees(mode, t, u, mask_bits=None):
+    """Does depth t of a branch see that branch's key u?  CHAIN: u <= t;
+    BLOCK: always; BITMASK: bit u of the row's mask word.  Works elementwise
+    on arrays (mask_bits: the row's uint64 word, broadcast like t)."""
+    t = np.asarray(t)
+    u = np.asarray(u)
+    if mode == CHAIN:
+        return u <= t
+    if mode == BLOCK:
+        return np.ones(np.broadcast(t, u).shape, dtype=bool)
+    if mode == BITMASK:
+        bits = np.asarray(mask_bits, dtype=np.uint64)
+        return ((bits >> u.astype(np.uint64)) & np.uint64(1)) == np.uint64(1)
+    raise ValueError(f"unknown mask mode {mode}")
+
+
+def visible_mask(cu, anchors, B: int, mode: int, window: int = 0, branch_mask=None) -> np.ndarray:
     """Explicit [R, R] boolean mask over concatenated rows x keys, written
     entry by entry from the definition (tiny sizes only)."""
     cu = i64(cu)
@@ -124,17 +157,27 @@ def visible_mask(cu, anchors, B: int, mode: int) -> np.ndarray:
     M = np.zeros((R, R), dtype=bool)
     for i in range(S):
         s = int(doc_start_of(cu, i))
+        if window and window > 0:
+            s = max(s, i - window + 1)
         for j in range(s, i + 1):
             M[i, j] = True
     for b in range(Nb):
         a = int(anchors[b])
         s = int(doc_start_of(cu, a))
+        if window and window > 0:
+            s = max(s, a - window + 1)
         for t in range(B):
             r = S + b * B + t
             for j in range(s, a + 1):
                 M[r, j] = True
             for u in range(B):
-                if mode == BLOCK or u <= t:
+                if mode == BLOCK:
+                    seen = True
+                elif mode == CHAIN:
+                    seen = u <= t
+                else:
+                    seen = (int(branch_mask[b][t]) >> u) & 1 == 1
+                if seen:
                     M[r, S + b * B + u] = True
     return M
 
@@ -187,7 +230,8 @@ def _split_rows(x, S, Nb, B):
 # form 1: brute force over the full mask
 # --------------------------------------------------------------------------
 
-def forward_brute(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None):
+def forward_brute(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None, window=0,
+                  branch_mask=None):
     """Returns (O_main [S,Hq,d], O_branch [Nb,B,Hq,d], LSE [Hq,R])."""
     Q, K, V = _concat(q, qb), _concat(k, kb), _concat(v, vb)
     S = int(i64(cu)[-1])
@@ -195,7 +239,7 @@ def forward_brute(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None):
     Hq, Hkv, d = Q.shape[1], K.shape[1], Q.shape[2]
     G = Hq // Hkv
     sc = default_scale(d, scale)
-    M = visible_mask(cu, anchors, B, mode)
+    M = visible_mask(cu, anchors, B, mode, window, branch_mask)
     O = np.zeros_like(Q)
     lse = np.zeros((Hq, Q.shape[0]))
     for h in range(Hq):
@@ -211,7 +255,8 @@ def forward_brute(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None):
     return om, ob, lse
 
 
-def backward_brute(q, k, v, qb, kb, vb, do, dob, cu, anchors, B, mode, scale=None):
+def backward_brute(q, k, v, qb, kb, vb, do, dob, cu, anchors, B, mode, scale=None, window=0,
+                   branch_mask=None):
     """Closed-form gradients over the full mask.
     Returns (dq, dk, dv, dqb, dkb, dvb) in the input layouts (fp64)."""
     Q, K, V = _concat(q, qb), _concat(k, kb), _concat(v, vb)
@@ -221,7 +266,7 @@ def backward_brute(q, k, v, qb, kb, vb, do, dob, cu, anchors, B, mode, scale=Non
     Hq, Hkv, d = Q.shape[1], K.shape[1], Q.shape[2]
     G = Hq // Hkv
     sc = default_scale(d, scale)
-    M = visible_mask(cu, anchors, B, mode)
+    M = visible_mask(cu, anchors, B, mode, window, branch_mask)
     dQ = np.zeros_like(Q)
     dK = np.zeros_like(K)
     dV = np.zeros_like(V)
@@ -248,14 +293,16 @@ def backward_brute(q, k, v, qb, kb, vb, do, dob, cu, anchors, B, mode, scale=Non
 # form 2: per-row visible key sets (row blocks), any subset of rows
 # --------------------------------------------------------------------------
 
-def _row_blocks(rows, cu, anchors, B, block):
+def _row_blocks(rows, cu, anchors, B, block, window=0):
     """Group requested concatenated row indices into blocks whose rows share a
-    document; yields (rows, doc_start, limits, branch_id, depth)."""
+    document; yields (rows, first main key of the block, per-row first main
+    keys, limits, branch_id, depth)."""
     cu = i64(cu)
     anchors = i64(anchors)
     S = int(cu[-1])
     rows = np.asarray(rows, dtype=np.int64)
     starts, lim = row_limits(cu, anchors, B)
+    first = row_first_keys(starts, lim, window)
     doc = np.searchsorted(cu, lim[rows], side="right") - 1
     order = np.lexsort((lim[rows], doc))
     rows = rows[order]
@@ -270,7 +317,7 @@ def _row_blocks(rows, cu, anchors, B, block):
         isb = r >= S
         bid = np.where(isb, (r - S) // max(B, 1), -1)
         dep = np.where(isb, (r - S) % max(B, 1), -1)
-        yield r, int(starts[r[0]]), lim[r], bid, dep
+        yield r, int(first[r].min()), first[r], lim[r], bid, dep
         i = j
 
 
@@ -282,28 +329,32 @@ class _Window:
         self.data, self.s0, self.ids = data, s0, ids
 
 
-def _block_scores(Qh, Kmain, Kbr, s0, lim, bid, dep, B, mode, sc):
+def _block_scores(Qh, Kmain, Kbr, s0, first, lim, bid, dep, B, mode, sc, branch_mask=None):
     """Scores of a row block against its visible keys: main keys [s0, max lim]
-    (masked to each row's limit) and the branch keys of the block's branches
-    (masked to each row's own branch and depth rule).  Returns
+    (masked to each row's own [first, limit]) and the branch keys of the
+    block's branches (masked to each row's own branch and mask rule).  Returns
     (scores [nr, nk], main key index array, branch key index array)."""
     hi = int(lim.max())
     mk = np.arange(s0, hi + 1)
     s_main = sc * (Qh @ Kmain.data.T)
-    s_main = np.where(mk[None, :] <= lim[:, None], s_main, -np.inf)
+    s_main = np.where((mk[None, :] <= lim[:, None]) & (mk[None, :] >= first[:, None]), s_main, -np.inf)
     if Kbr is None:
         return s_main, mk, np.zeros(0, dtype=np.int64)
     bk = Kbr.ids
     kb_b = bk // B
     kb_u = bk % B
     s_br = sc * (Qh @ Kbr.data.T)
-    vis = (kb_b[None, :] == bid[:, None]) & ((mode == BLOCK) | (kb_u[None, :] <= dep[:, None]))
+    bits = None
+    if mode == BITMASK:
+        bm = np.asarray(branch_mask, dtype=np.uint64)
+        bits = np.where(bid >= 0, bm[np.maximum(bid, 0), np.maximum(dep, 0)], 0)[:, None]
+    vis = (kb_b[None, :] == bid[:, None]) & branch_sees(mode, dep[:, None], kb_u[None, :], bits)
     s_br = np.where(vis, s_br, -np.inf)
     return np.concatenate([s_main, s_br], axis=1), mk, bk
 
 
 def forward_rows(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None, rows=None,
-                 heads=None, block=512):
+                 heads=None, block=512, window=0, branch_mask=None):
     """O and LSE of the requested concatenated rows (default: all rows).
     Returns (rows [n], O [n, Hq, d], LSE [Hq, n]); heads outside ``heads`` are 0."""
     S, Hq, d = q.shape
@@ -321,7 +372,7 @@ def forward_rows(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None, rows=Non
     pos = {int(r): n for n, r in enumerate(rows)}
     O = np.zeros((len(rows), Hq, d))
     L = np.full((Hq, len(rows)), np.nan)
-    for r, s0, lim, bid, dep in _row_blocks(rows, cu, anchors, B, block):
+    for r, s0, first, lim, bid, dep in _row_blocks(rows, cu, anchors, B, block, window):
         idx = np.array([pos[int(x)] for x in r])
         hi = int(lim.max())
         mk = np.arange(s0, hi + 1)
@@ -331,7 +382,8 @@ def forward_rows(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None, rows=Non
             g = h // G
             Kmain = _Window(Km.rows(mk, g), s0)
             Kbr = _Window(Kb.rows(bk, g), None, bk) if len(bk) else None
-            s, _, _ = _block_scores(Qc.rows(r, h), Kmain, Kbr, s0, lim, bid, dep, B, mode, sc)
+            s, _, _ = _block_scores(Qc.rows(r, h), Kmain, Kbr, s0, first, lim, bid, dep, B, mode, sc,
+                                    branch_mask)
             m = s.max(axis=1, keepdims=True)
             e = np.exp(s - m)
             l = e.sum(axis=1, keepdims=True)
@@ -342,7 +394,7 @@ def forward_rows(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None, rows=Non
 
 
 def backward_rows(q, k, v, qb, kb, vb, do, dob, cu, anchors, B, mode, scale=None, rows=None,
-                  heads=None, block=512):
+                  heads=None, block=512, window=0, branch_mask=None):
     """Closed-form backward restricted to the contributions of the requested
     rows (default: all rows).  With dO zero outside ``rows`` this is the exact
     full gradient.  Returns (rows, dQ [n, Hq, d] of those rows,
@@ -367,7 +419,7 @@ def backward_rows(q, k, v, qb, kb, vb, do, dob, cu, anchors, B, mode, scale=None
     dvbf = np.zeros((Nb * B, Hkv, d))
     pos = {int(r): n for n, r in enumerate(rows)}
     dQ = np.zeros((len(rows), Hq, d))
-    for r, s0, lim, bid, dep in _row_blocks(rows, cu, anchors, B, block):
+    for r, s0, first, lim, bid, dep in _row_blocks(rows, cu, anchors, B, block, window):
         idx = np.array([pos[int(x)] for x in r])
         hi = int(lim.max())
         mk = np.arange(s0, hi + 1)
@@ -379,7 +431,7 @@ def backward_rows(q, k, v, qb, kb, vb, do, dob, cu, anchors, B, mode, scale=None
             Kb_g = Kb.rows(bk, g) if len(bk) else np.zeros((0, d))
             Qh = Qc.rows(r, h)
             s, _, _ = _block_scores(Qh, _Window(Km_g, s0), _Window(Kb_g, None, bk) if len(bk) else None,
-                                    s0, lim, bid, dep, B, mode, sc)
+                                    s0, first, lim, bid, dep, B, mode, sc, branch_mask)
             m = s.max(axis=1, keepdims=True)
             e = np.exp(s - m)
             P = e / e.sum(axis=1, keepdims=True)
@@ -446,9 +498,10 @@ def lse_merge(o_parts, lse_parts):
     return O, L
 
 
-def main_part(q, k, v, qb, cu, anchors, B, scale=None):
+def main_part(q, k, v, qb, cu, anchors, B, scale=None, window=0):
     """Main-sequence component for every row (main rows then branch rows):
-    each row against main keys [s(limit), limit].  Returns O [R,Hq,d], LSE [Hq,R]."""
+    each row against main keys [s(limit), limit] (with a window W > 0:
+    [max(s(limit), limit - W + 1), limit]).  Returns O [R,Hq,d], LSE [Hq,R]."""
     q, k, v, qb = (f64(x) for x in (q, k, v, qb))
     S, Hq, d = q.shape
     Hkv = k.shape[1]
@@ -466,16 +519,18 @@ def main_part(q, k, v, qb, cu, anchors, B, scale=None):
         if len(r) == 0:
             continue
         keys = np.arange(s, e)
-        mask = keys[None, :] <= lim[r][:, None]
+        first = row_first_keys(starts[r], lim[r], window)
+        mask = (keys[None, :] <= lim[r][:, None]) & (keys[None, :] >= first[:, None])
         for h in range(Hq):
             g = h // G
             O[r, h], L[h, r] = attend(Qc[r, h], k[s:e, g], v[s:e, g], mask, sc)
     return O, L
 
 
-def branch_part(qb, kb, vb, B, mode, scale=None):
+def branch_part(qb, kb, vb, B, mode, scale=None, branch_mask=None):
     """Branch-local component: each branch row against its own branch's keys
-    (u <= t for CHAIN, all u for BLOCK).  Returns O [Nb*B,Hq,d], LSE [Hq,Nb*B]."""
+    (u <= t for CHAIN, all u for BLOCK, the row's bits for BITMASK).  Returns
+    O [Nb*B,Hq,d], LSE [Hq,Nb*B]."""
     qb, kb, vb = (f64(x) for x in (qb, kb, vb))
     Nb, _, Hq, d = qb.shape
     Hkv = kb.shape[2]
@@ -484,23 +539,25 @@ def branch_part(qb, kb, vb, B, mode, scale=None):
     O = np.zeros((Nb * B, Hq, d))
     L = np.zeros((Hq, Nb * B))
     t = np.arange(B)
-    mask = (t[None, :] <= t[:, None]) if mode == CHAIN else np.ones((B, B), dtype=bool)
     for b in range(Nb):
+        bits = np.asarray(branch_mask, dtype=np.uint64)[b][:, None] if mode == BITMASK else None
+        mask = branch_sees(mode, t[:, None], t[None, :], bits)
         for h in range(Hq):
             g = h // G
             O[b * B:(b + 1) * B, h], L[h, b * B:(b + 1) * B] = attend(qb[b, :, h], kb[b, :, g], vb[b, :, g], mask, sc)
     return O, L
 
 
-def forward_decomposed(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None):
+def forward_decomposed(q, k, v, qb, kb, vb, cu, anchors, B, mode, scale=None, window=0,
+                       branch_mask=None):
     """Main part + branch part merged by Eq. 2.  Same outputs as forward_brute."""
     S = q.shape[0]
     Nb = qb.shape[0]
-    Om, Lm = main_part(q, k, v, qb, cu, anchors, B, scale)
+    Om, Lm = main_part(q, k, v, qb, cu, anchors, B, scale, window)
     O = Om.copy()
     L = Lm.copy()
     if Nb:
-        Ob, Lb = branch_part(qb, kb, vb, B, mode, scale)
+        Ob, Lb = branch_part(qb, kb, vb, B, mode, scale, branch_mask)
         ob, lb = lse_merge([Om[S:], Ob], [Lm[:, S:].T, Lb.T])
         O[S:] = ob
         L[:, S:] = lb.T
@@ -524,13 +581,19 @@ def zigzag_chunks(cu, R: int):
     return out
 
 
-def forward_ring(q, k, v, qb, kb, vb, cu, anchors, B, mode, R, scale=None, step_order=None):
+def forward_ring(q, k, v, qb, kb, vb, cu, anchors, B, mode, R, scale=None, step_order=None,
+                 window=0, branch_mask=None, partials=False):
     """Ring form with R CPU ranks.  Rank r holds the main Q/K/V rows of its
     zigzag chunks and the branches anchored in them.  For ring step st (in
     ``step_order``, default 0..R-1) rank r holds the K/V chunks sent from rank
     (r - st) mod R, attends its rows to the visible ones and merges the step's
     partial into its running (O, LSE) with Eq. 2.  Finally each rank merges its
-    branch rows' branch-local part.  Branch K/V never leave their rank."""
+    branch rows' branch-local part.  Branch K/V never leave their rank.
+
+    With ``partials`` it returns instead, for every rank k, the partial
+    (O, LSE) of every row over the visible main keys of rank k's chunks, i.e.
+    what the row's rank computes at the ring step where k's K/V visit it:
+    (O [R, rows, Hq, d], LSE [R, Hq, rows]); empty partials are (0, -inf)."""
     q, k, v, qb, kb, vb = (f64(x) for x in (q, k, v, qb, kb, vb))
     S, Hq, d = q.shape
     Hkv = k.shape[1]
@@ -540,6 +603,7 @@ def forward_ring(q, k, v, qb, kb, vb, cu, anchors, B, mode, R, scale=None, step_
     anc = i64(anchors)
     chunks = zigzag_chunks(cu, R)
     starts, lim = row_limits(cu, anchors, B)
+    first = row_first_keys(starts, lim, window)
     Qc = np.concatenate([q, qb.reshape(-1, Hq, d)], axis=0)
     owner_rows = {r: [] for r in range(R)}
     owner_keys = {r: [] for r in range(R)}
@@ -555,6 +619,9 @@ def forward_ring(q, k, v, qb, kb, vb, cu, anchors, B, mode, R, scale=None, step_
     L = np.full((Hq, S + Nb * B), -np.inf)
     steps = list(range(R)) if step_order is None else list(step_order)
     assert sorted(steps) == list(range(R))
+    if partials:
+        PO = np.zeros((R, S + Nb * B, Hq, d))
+        PL = np.full((R, Hq, S + Nb * B), -np.inf)
     for r in range(R):
         rows = np.array(sorted(owner_rows[r]), dtype=np.int64)
         if len(rows) == 0:
@@ -563,16 +630,19 @@ def forward_ring(q, k, v, qb, kb, vb, cu, anchors, B, mode, R, scale=None, step_
         run_L = np.full((Hq, len(rows)), -np.inf)
         for st in steps:
             kidx, Ks, Vs = shard[(r - st) % R]  # the chunk pair received at this step
-            mask = (kidx[None, :] >= starts[rows][:, None]) & (kidx[None, :] <= lim[rows][:, None])
+            mask = (kidx[None, :] >= first[rows][:, None]) & (kidx[None, :] <= lim[rows][:, None])
             pO = np.zeros_like(run_O)
             pL = np.full_like(run_L, -np.inf)
             for h in range(Hq):
                 g = h // G
                 pO[:, h], pL[h] = attend(Qc[rows, h], Ks[:, g], Vs[:, g], mask, sc)
+            if partials:
+                PO[(r - st) % R, rows] = pO
+                PL[(r - st) % R][:, rows] = pL
             mo, ml = lse_merge([run_O, pO], [run_L.T, pL.T])
             run_O, run_L = mo, ml.T
         isb = rows >= S
-        if isb.any():
+        if isb.any() and not partials:
             br_rows = rows[isb]
             bid = (br_rows - S) // B
             dep = (br_rows - S) % B
@@ -580,7 +650,8 @@ def forward_ring(q, k, v, qb, kb, vb, cu, anchors, B, mode, R, scale=None, step_
             bL = np.full((Hq, len(br_rows)), -np.inf)
             for n, (bi, t) in enumerate(zip(bid, dep)):
                 u = np.arange(B)
-                m = ((u <= t) | (mode == BLOCK))[None, :]
+                bits = np.asarray(branch_mask, dtype=np.uint64)[bi, t] if mode == BITMASK else None
+                m = branch_sees(mode, t, u, bits)[None, :]
                 for h in range(Hq):
                     g = h // G
                     o1, l1 = attend(qb[bi, t, h][None, :], kb[bi, :, g], vb[bi, :, g], m, sc)
@@ -590,6 +661,8 @@ def forward_ring(q, k, v, qb, kb, vb, cu, anchors, B, mode, R, scale=None, step_
             run_L[:, isb] = ml.T
         O[rows] = run_O
         L[:, rows] = run_L
+    if partials:
+        return PO, PL
     om, obr = _split_rows(O, S, Nb, B)
     return om, obr, L
 
@@ -598,17 +671,31 @@ def forward_ring(q, k, v, qb, kb, vb, cu, anchors, B, mode, R, scale=None, step_
 # counting
 # --------------------------------------------------------------------------
 
-def visible_pair_count(cu, anchors, B, mode) -> int:
+def visible_pair_count(cu, anchors, B, mode, window=0, branch_mask=None) -> int:
     """Exact number of visible (row, key) pairs per q head, from the
     definition: sum over main rows of (i - s(i) + 1) plus, per branch,
-    B * (a_b - s(a_b) + 1) main pairs and B(B+1)/2 (CHAIN) or B*B (BLOCK)
-    branch pairs."""
+    B * (a_b - s(a_b) + 1) main pairs and B(B+1)/2 (CHAIN), B*B (BLOCK) or the
+    set bits of its mask rows (BITMASK) branch pairs.  With a window W > 0 a
+    prefix of n keys counts min(n, W)."""
     cu = i64(cu)
     anc = i64(anchors)
-    L = np.diff(cu)
-    main = int((L * (L + 1) // 2).sum())
+    S = int(cu[-1])
+    pos = np.arange(S)
+    n_main = pos - doc_start_of(cu, pos) + 1
+    if window and window > 0:
+        n_main = np.minimum(n_main, window)
+    main = int(n_main.sum())
     if len(anc) == 0:
         return main
-    pre = int((anc - doc_start_of(cu, anc) + 1).sum()) * B
-    loc = len(anc) * (B * (B + 1) // 2 if mode == CHAIN else B * B)
+    n_pre = anc - doc_start_of(cu, anc) + 1
+    if window and window > 0:
+        n_pre = np.minimum(n_pre, window)
+    pre = int(n_pre.sum()) * B
+    if mode == CHAIN:
+        loc = len(anc) * (B * (B + 1) // 2)
+    elif mode == BLOCK:
+        loc = len(anc) * B * B
+    else:
+        words = np.asarray(branch_mask, dtype=np.uint64).reshape(-1)
+        loc = sum(bin(int(x) & ((1 << B) - 1)).count("1") for x in words)
     return main + pre + loc
