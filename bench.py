@@ -298,6 +298,15 @@ def run_gpu(args):
     prob = wl._draw(cfg, wl.seed_of(widx) + rank_seed_offset(rank), cu, anc, dev, True)
     a = ba.BranchAttention(cu, anc, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, B=cfg.B, mode=cfg.mode,
                            R=cfg.R, device=dev)
+    # host planning cost (cold: the library's plan cache is cleared first); later
+    # calls on the same packing reuse the cached plan
+    ba.clear_cache()
+    host_plan_ms = {cfg.name: round(a.prepare(), 3)}
+    big = wl.CONFIGS[4]
+    cu_big, anc_big = wl.make_layout(4)
+    host_plan_ms[big.name] = round(ba.BranchAttention(
+        cu_big, anc_big, Hq=big.Hq, Hkv=big.Hkv, d=big.d, B=big.B, mode=big.mode, R=big.R,
+        device="cpu").prepare(), 3)
     stats = a.plan_stats()
     P = stats["visible_pairs"]
     useful = 14.0 * cfg.d * P * cfg.Hq
@@ -455,6 +464,8 @@ def run_gpu(args):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "pipelined": "h2d / compute / d2h on three streams, two buffer sets"},
         "gpu_launches": launches,
+        "host_plan_ms": dict(host_plan_ms, note="cold host planning per packing; every step "
+                                                "reuses the cached plan"),
         "merge": merge,
         "clocks": clocks,
     }

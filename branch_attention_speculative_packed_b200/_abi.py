@@ -22,6 +22,7 @@ BA_ERR_SCRATCH_LIMIT = -6
 
 BA_MASK_CHAIN = 0
 BA_MASK_BLOCK = 1
+BA_MASK_BITMASK = 2
 
 BA_WS_FWD = 0
 BA_WS_BWD = 1
@@ -31,6 +32,7 @@ EXPORTED = (
     "ba_bwd", "ba_status_string", "ba_sync_status", "ba_plan_stats", "ba_profile_enable",
     "ba_profile_collect", "ba_last_error_word", "ba_fused_fwd_noalloc", "ba_plan_rank_work",
     "ba_plan_fwd_pairs", "ba_plan_prepare", "ba_clear_cache", "ba_plan_cache_stats",
+    "ba_main_fwd_ring",
 )
 
 
@@ -44,6 +46,8 @@ class BaProblem(ctypes.Structure):
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("qb", ctypes.c_void_p), ("kb", ctypes.c_void_p), ("vb", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("window", ctypes.c_int),
+        ("branch_mask_h", ctypes.c_void_p), ("branch_mask_d", ctypes.c_void_p),
     ]
 
 
@@ -75,6 +79,7 @@ def lib() -> ctypes.CDLL:
         L.ba_workspace_size.argtypes = [P, i32]
         L.ba_workspace_size.restype = ctypes.c_size_t
         L.ba_main_fwd.argtypes = [P, vp, vp, vp]
+        L.ba_main_fwd_ring.argtypes = [P, vp, vp, vp]
         L.ba_branch_fwd.argtypes = [P, vp, vp, vp]
         L.ba_fused_fwd.argtypes = [P, vp, vp, vp, vp]
         L.ba_fused_fwd_noalloc.argtypes = [P, vp, vp, vp, vp]
@@ -102,7 +107,7 @@ def lib() -> ctypes.CDLL:
         L.ba_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
                                          ctypes.POINTER(ctypes.c_int), i32]
         L.ba_profile_collect.restype = ctypes.c_int
-        for name in ("ba_main_fwd", "ba_branch_fwd", "ba_fused_fwd", "ba_fused_fwd_noalloc", "ba_bwd",
+        for name in ("ba_main_fwd", "ba_main_fwd_ring", "ba_branch_fwd", "ba_fused_fwd", "ba_fused_fwd_noalloc", "ba_bwd",
                      "ba_lse_merge",
                      "ba_sync_status", "ba_plan_stats"):
             getattr(L, name).restype = ctypes.c_int

@@ -29,11 +29,13 @@ class BranchAttention:
 
     cu_seqlens: int32 [ndoc+1]; anchors: int32 [Nb] ascending; B: branch depth
     (chain) or block size (block); mode: 0 chain (EAGLE-3 training-time test),
-    1 block (DFlash-style); R: virtual zigzag ranks; scale: softmax scale
-    (None: 1/sqrt(d))."""
+    1 block (DFlash-style), 2 bitmask (``branch_mask``: [Nb, B] 64-bit words,
+    row (b, t) sees branch key u iff bit u of branch_mask[b, t]); R: virtual
+    zigzag ranks; scale: softmax scale (None: 1/sqrt(d)); window: main-prefix
+    window W (0: none)."""
 
     def __init__(self, cu_seqlens, anchors, *, Hq, Hkv, d, B, mode, R=1, scale=None,
-                 device="cuda"):
+                 device="cuda", window=0, branch_mask=None):
         self.cu_h = torch.as_tensor(cu_seqlens, dtype=torch.int32).cpu().contiguous()
         self.anc_h = torch.as_tensor(anchors, dtype=torch.int32).cpu().contiguous()
         self.device = torch.device(device)
@@ -49,6 +51,14 @@ class BranchAttention:
         self.Nb = int(self.anc_h.numel())
         self.Hq, self.Hkv, self.d, self.B, self.mode, self.R = Hq, Hkv, d, B, mode, R
         self.scale = -1.0 if scale is None else float(scale)
+        self.window = int(window)
+        self.bm_h = self.bm_d = None
+        if branch_mask is not None:
+            bm = torch.as_tensor(branch_mask)
+            if bm.dtype != torch.int64:  # uint64 words from numpy: keep the bits
+                bm = torch.from_numpy(__import__("numpy").asarray(branch_mask).astype("uint64").view("int64"))
+            self.bm_h = bm.reshape(-1).cpu().contiguous()
+            self.bm_d = self.bm_h.to(self.device) if self.device.type == "cuda" else self.bm_h
         self._ws = {}
 
     @property
@@ -63,6 +73,10 @@ class BranchAttention:
         p.cu_seqlens_d = self.cu_d.data_ptr()
         p.anchors_h = self.anc_h.data_ptr() if self.Nb else None
         p.anchors_d = self.anc_d.data_ptr() if self.Nb else None
+        p.window = self.window
+        if self.bm_h is not None:
+            p.branch_mask_h = self.bm_h.data_ptr()
+            p.branch_mask_d = self.bm_d.data_ptr()
         for name, t in (("q", q), ("k", k), ("v", v), ("qb", qb), ("kb", kb), ("vb", vb)):
             if t is not None:
                 if not t.is_contiguous() or t.dtype != torch.bfloat16:
@@ -152,6 +166,19 @@ class BranchAttention:
         p = self._problem(q, k, v, qb, kb, vb, ws)
         check(_abi.lib().ba_main_fwd(ctypes.byref(p), _ptr(o), _ptr(lse), _stream(stream)),
               "ba_main_fwd")
+        return o, lse
+
+    def main_fwd_ring(self, q, k, v, qb, kb, vb, stream=None):
+        """Step a2 by ring steps: partial k of every row over the visible main
+        keys of virtual rank k's zigzag chunks.  Returns (o_parts fp32
+        [R,rows,Hq,d], lse_parts fp32 [R,Hq,rows])."""
+        dev = q.device
+        o = torch.empty(self.R, self.rows, self.Hq, self.d, dtype=torch.float32, device=dev)
+        lse = torch.empty(self.R, self.Hq, self.rows, dtype=torch.float32, device=dev)
+        ws = self.workspace(BA_WS_FWD)
+        p = self._problem(q, k, v, qb, kb, vb, ws)
+        check(_abi.lib().ba_main_fwd_ring(ctypes.byref(p), _ptr(o), _ptr(lse), _stream(stream)),
+              "ba_main_fwd_ring")
         return o, lse
 
     def branch_fwd(self, q, k, v, qb, kb, vb, stream=None):

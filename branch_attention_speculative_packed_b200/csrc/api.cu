@@ -172,10 +172,12 @@ PlanCache& plan_cache() {
 
 std::string plan_key(const ba_problem* p) {
   const int32_t dims[] = {p->S, p->ndoc, p->Hq, p->Hkv, p->d, p->Nb, p->Nb > 0 ? p->B : 0,
-                          p->mode, p->R};
+                          p->mode, p->R, p->window > 0 ? p->window : 0};
   std::string key(reinterpret_cast<const char*>(dims), sizeof(dims));
   key.append(reinterpret_cast<const char*>(p->cu_seqlens_h), size_t(p->ndoc + 1) * sizeof(int32_t));
   if (p->Nb > 0) key.append(reinterpret_cast<const char*>(p->anchors_h), size_t(p->Nb) * sizeof(int32_t));
+  if (p->Nb > 0 && p->mode == BA_MASK_BITMASK)
+    key.append(reinterpret_cast<const char*>(p->branch_mask_h), size_t(p->Nb) * p->B * sizeof(uint64_t));
   return key;
 }
 
@@ -283,7 +285,7 @@ ba_status check_workspace(const void* ws, size_t bytes, const WorkspaceLayout& w
 // anything is enqueued, and the plan is uploaded from pageable memory.
 ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void* ob, float* lse,
                   cudaStream_t st, void* scratch = nullptr, size_t scratch_bytes = 0,
-                  ba_status too_big = BA_ERR_WORKSPACE) {
+                  ba_status too_big = BA_ERR_WORKSPACE, bool ring = false) {
   ba_status s = validate(p, true);
   if (s != BA_OK) return s;
   if (!lse || !aligned16(lse)) return BA_ERR_INVALID_ARG;
@@ -301,7 +303,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   } else if ((s = check_workspace(p->workspace, p->workspace_bytes, w)) != BA_OK) {
     return s;
   }
-  const int64_t items = int64_t(plan.pairs.size() / 2) * p->Hq;
+  const int64_t items = int64_t(plan.pairs.size() / 2) * p->Hq * (ring ? p->R : 1);
   if (items > 0x7fffffff) return BA_ERR_UNSUPPORTED;
   DeviceInfo di;
   if ((s = device_info(&di)) != BA_OK) return s;
@@ -329,6 +331,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   a.row_table = reinterpret_cast<const int32_t*>(ws + w.rows_off);
   a.tiles = reinterpret_cast<const TileDesc*>(ws + w.tiles_off);
   a.pairs = reinterpret_cast<const int32_t*>(ws + w.pairs_off);
+  a.bmask = (p->mode == BA_MASK_BITMASK && p->Nb > 0) ? p->branch_mask_d : nullptr;
   a.S = p->S;
   a.Nb = p->Nb;
   a.B = plan.B > 0 ? plan.B : 1;
@@ -336,11 +339,15 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   a.Hq = p->Hq;
   a.G = p->Hq / p->Hkv;
   a.d = p->d;
+  a.window = p->window > 0 ? p->window : 0;
+  a.ring = ring ? p->R : 0;
   a.n_items = static_cast<int>(items);
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.with_branch = fused && p->Nb > 0 ? 1 : 0;
   a.out_bf16 = fused ? 1 : 0;
   a.o_part = o_part;
+  a.o_part_stride = ring ? rows * p->Hq * p->d : 0;
+  a.lse_stride = ring ? rows * p->Hq : 0;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.ob = static_cast<__nv_bfloat16*>(ob);
   a.lse = lse;
@@ -348,7 +355,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   a.err = di.err;
   a.counter = reinterpret_cast<uint32_t*>(ws + w.counters_off);
   a.wait_limit = kWaitLimitCycles;
-  ProfScope prof(fused ? "fused_fwd" : "main_fwd", st);
+  ProfScope prof(fused ? "fused_fwd" : ring ? "main_fwd_ring" : "main_fwd", st);
   if (launch_fwd(maps, a, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
   return BA_OK;
 }
@@ -431,6 +438,12 @@ ba_status ba_main_fwd(const ba_problem* p, float* o_part, float* lse_part, ba_st
   return run_fwd(p, false, o_part, nullptr, nullptr, lse_part, reinterpret_cast<cudaStream_t>(stream));
 }
 
+ba_status ba_main_fwd_ring(const ba_problem* p, float* o_parts, float* lse_parts,
+                           ba_stream_t stream) {
+  return run_fwd(p, false, o_parts, nullptr, nullptr, lse_parts,
+                 reinterpret_cast<cudaStream_t>(stream), nullptr, 0, BA_ERR_WORKSPACE, true);
+}
+
 ba_status ba_fused_fwd(const ba_problem* p, void* o, void* ob, float* lse, ba_stream_t stream) {
   return run_fwd(p, true, nullptr, o, ob, lse, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -445,7 +458,8 @@ ba_status ba_branch_fwd(const ba_problem* p, float* o_part, float* lse_part, ba_
   ProfScope prof("branch_fwd", reinterpret_cast<cudaStream_t>(stream));
   if (launch_branch_fwd(static_cast<const __nv_bfloat16*>(p->qb),
                         static_cast<const __nv_bfloat16*>(p->kb),
-                        static_cast<const __nv_bfloat16*>(p->vb), p->Nb, p->B, p->mode, p->Hq,
+                        static_cast<const __nv_bfloat16*>(p->vb),
+                        p->mode == BA_MASK_BITMASK ? p->branch_mask_d : nullptr, p->Nb, p->B, p->mode, p->Hq,
                         p->Hkv, p->d, scale_of(p), o_part, lse_part,
                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return BA_ERR_CUDA;
@@ -510,8 +524,8 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   const int64_t items_q = int64_t(plan.tiles.size()) * p->Hq;
   const int64_t items_kv = int64_t(nkv) * p->Hkv;
   if (items_q > 0x7fffffff || items_kv > 0x7fffffff) return BA_ERR_UNSUPPORTED;
-  if ((s = stage_plan(p, *cp, w, p->workspace, true, st)) != BA_OK) return s;
   uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  if ((s = stage_plan(p, *cp, w, p->workspace, true, st)) != BA_OK) return s;
   const int64_t rows = int64_t(p->S) + int64_t(p->Nb) * plan.B;
   const float scale = scale_of(p);
   const int G = p->Hq / p->Hkv;
@@ -541,6 +555,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   pa.drow = reinterpret_cast<float*>(ws + w.drow_off);
   pa.meta = reinterpret_cast<SlotMeta*>(ws + w.meta_off);
   pa.lims = reinterpret_cast<int32_t*>(ws + w.lims_off);
+  const uint64_t* bmask = (nb && p->mode == BA_MASK_BITMASK) ? p->branch_mask_d : nullptr;
   {
     ProfScope prof("bwd_prep", st);
     if (launch_bwd_prep(pa, p->d, st) != cudaSuccess) return BA_ERR_CUDA;
@@ -571,6 +586,9 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   qa.meta = pa.meta;
   qa.ls = pa.ls;
   qa.ds = pa.ds;
+  qa.bmask = bmask;
+  qa.mode = p->mode;
+  qa.window = p->window > 0 ? p->window : 0;
   qa.S = p->S;
   qa.Hq = p->Hq;
   qa.G = G;
@@ -599,6 +617,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   ka.lims = pa.lims;
   ka.ls = pa.ls;
   ka.ds = pa.ds;
+  ka.window = p->window > 0 ? p->window : 0;
   ka.Hq = p->Hq;
   ka.Hkv = p->Hkv;
   ka.G = G;
@@ -627,6 +646,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
     ba_.dob = static_cast<const __nv_bfloat16*>(doutb);
     ba_.lse = lse;
     ba_.drow = pa.drow;
+    ba_.bmask = bmask;
     ba_.S = p->S;
     ba_.Nb = p->Nb;
     ba_.B = p->B;

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepArgs a) {
           const int t = (r - a.S) - b * a.B;
           m.limit = a.anchors[b];
           m.blo = b * a.B;
-          m.bhi = m.blo + (a.mode == 1 ? a.B : t + 1);
+          m.bhi = m.blo + (a.mode == 0 ? t + 1 : a.B);
         }
         a.meta[slot] = m;
         a.lims[slot] = m.limit;
@@ -99,7 +99,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepArgs a) {
 // ------------------------------------------------------------------ branch dK/dV
 // One block per (branch b, KV head g); one warp per branch key u (strided).
 // Lane l holds elements [l*E, l*E + E) of k_u, v_u and of the accumulators.
-// For every query head of the group and every row t that sees u:
+// For every query head of the group and every row t that sees u (chain:
+// t >= u; block: all; bitmask: bit u of row t's word):
 //   s = scale <q_t, k_u>, P = exp(s - L_t), dS = P (<dO_t, v_u> - D_t),
 //   dV_u += P dO_t, dK_u += scale dS q_t.
 template <int D>
@@ -123,7 +124,9 @@ __global__ void branch_bwd_kernel(const BranchBwdArgs a) {
     }
     for (int hh = 0; hh < G; ++hh) {
       const int h = g * G + hh;
-      for (int t = (a.mode == 1 ? 0 : u); t < a.B; ++t) {
+      for (int t = (a.mode == 0 ? u : 0); t < a.B; ++t) {
+        // bitmask: row t sees key u iff bit u of its word
+        if (a.mode == 2 && !((a.bmask[int64_t(b) * a.B + t] >> u) & 1ull)) continue;
         const int64_t qo = ((int64_t(b) * a.B + t) * a.Hq + h) * D + lane * E;
         float qf[E], df[E];
         float s = 0.f, dp = 0.f;

@@ -8,7 +8,8 @@
 //   S^T_i  = K Q_i^T     [128 keys x 128 rows]  -> TMEM buffer SB
 //   dP^T_i = V dO_i^T                           -> TMEM buffer DB
 //   threads (one key per thread, two warpgroups of 64 rows each):
-//       P^T = exp2(S^T*scale*log2e - L*log2e) where key <= the row's limit,
+//       P^T = exp2(S^T*scale*log2e - L*log2e) where key <= the row's limit
+//       (and, under a window W, key >= limit - W + 1),
 //       written as bf16 over the front of each warpgroup's half of SB;
 //       dS^T = P^T (dP^T - D), written as bf16 the same way into DB
 //   dV += P^T dO_i,  dK += dS^T Q_i             (A operand read from TMEM)
@@ -71,7 +72,8 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-template <int D>
+// kWin: a main-prefix window is in use (masking from below as well).
+template <int D, bool kWin>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
@@ -297,6 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t half_col = static_cast<uint32_t>(wg) * 64u;
     const float sl2 = a.scale_log2;
+    // window: a row with limit l sees keys >= l - W + 1; with no window W is
+    // huge, so that bound never bites
+    const int W = a.window > 0 ? a.window : 0x3fffffff;
     uint32_t qs = 0, qph = 0, sub = 0, acc_cnt = 0;
     bool ok = true;
     for (uint32_t rn = 0; ok; ++rn) {
@@ -311,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int g = code % a.Hkv;
       const int kp = it.key0 + row;  // this thread's key position
       const int warp_last_key = it.key0 + quarter * 32 + 31;
+      const int warp_first_key = it.key0 + quarter * 32;
       bool any = false;
       for (int ti = 0; ti < it.t_count && ok; ++ti) {
         for (int hh = 0; hh < G; ++hh) {
@@ -350,12 +356,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[c][i + 2] = __float_as_uint(x1.x);
             sv[c][i + 3] = __float_as_uint(x1.y);
           }
-          // The rows are sorted by limit (padding, limit -1, only at a tile's end), so when
-          // the warp's last key is visible to this warpgroup's first row, every pair is.
-          if (!(warp_last_key <= Lim[0])) {
+          // The rows are sorted by limit (padding, limit -1, only at a tile's end, and
+          // neutralised by its L), so when the warp's last key is visible to this
+          // warpgroup's first row, every pair is -- unless a window cuts the front of
+          // a row's range: that needs the warp's first key at or after the largest
+          // limit's window start as well.
+          bool full = warp_last_key <= Lim[0];
+          if constexpr (kWin) {
+            int mx = max(Lim[lane], Lim[lane + 32]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            full = full && warp_first_key >= mx - W + 1;
+          }
+          if (!full) {
 #pragma unroll
             for (int col = 0; col < 64; ++col)
-              if (kp > Lim[col]) sv[col >> 5][col & 31] = __float_as_uint(-INFINITY);
+              if (kp > Lim[col] || (kWin && kp < Lim[col] - W + 1)) sv[col >> 5][col & 31] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[32];
 #pragma unroll
@@ -456,24 +472,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool kWin>
 cudaError_t launch_d(const DkdvMaps& m, const DkdvArgs& a, int num_sms, cudaStream_t st) {
   using L = Smem<D>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::kAlloc));
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;
-  bwd_dkdv_kernel<D><<<grid, kThreads, L::kAlloc, st>>>(m.k, m.v, m.qg, m.dog, a);
+  bwd_dkdv_kernel<D, kWin><<<grid, kThreads, L::kAlloc, st>>>(m.k, m.v, m.qg, m.dog, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_bwd_dkdv(const DkdvMaps& m, const DkdvArgs& a, int num_sms, cudaStream_t st) {
-  if (a.d == 128) return launch_d<128>(m, a, num_sms, st);
-  if (a.d == 64) return launch_d<64>(m, a, num_sms, st);
+  const bool win = a.window > 0;
+  if (a.d == 128) return win ? launch_d<128, true>(m, a, num_sms, st) : launch_d<128, false>(m, a, num_sms, st);
+  if (a.d == 64) return win ? launch_d<64, true>(m, a, num_sms, st) : launch_d<64, false>(m, a, num_sms, st);
   return cudaErrorInvalidValue;
 }
 

@@ -54,7 +54,9 @@ struct Smem {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-template <int D>
+// kGen: a window or bitmask words are in use (per-row lower bounds and mask
+// bits); the plain instantiation keeps the original masking.
+template <int D, bool kGen>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -159,14 +161,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tma_load_2d(sbase + L::kQ + cb * 16384u, &tmQ, bar_q_full, h * D + cb * 64, td.row_base);
           ptx::tma_load_2d(sbase + L::kDO + cb * 16384u, &tmDO, bar_q_full, h * D + cb * 64, td.row_base);
         }
-        const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
+        const int nkv = ceil_div(td.kv_end - td.kv_lo, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
         for (int j = 0; j < nkv + nbr; ++j) {
           const void* mk = &tmK;
           const void* mv = &tmV;
           int y;
           if (j < nkv) {
-            y = td.doc_start + 128 * j;
+            y = td.kv_lo + 128 * j;
           } else {
             y = td.br_lo + 128 * (j - nkv);
             mk = &tmKb;
@@ -233,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(2, 1, 13))) { ok = false; break; }
         if (item >= a.n_items) break;
         const TileDesc td = a.tiles[a.order[item / Hq]];
-        const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
+        const int nkv = ceil_div(td.kv_end - td.kv_lo, 128);
         const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
         const int n = nkv + nbr;
         if (!ptx::mbar_wait(bar_q_full, q_phase, abort_flag, a.err, lim, ptx::wait_site(2, 1, 4))) { ok = false; break; }
@@ -304,13 +306,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (item >= a.n_items) break;
       const TileDesc td = a.tiles[a.order[item / Hq]];
       const int h = item % Hq;
-      const int nkv = ceil_div(td.kv_end - td.doc_start, 128);
+      const int nkv = ceil_div(td.kv_end - td.kv_lo, 128);
       const int nbr = (a.with_branch && td.br_hi > td.br_lo) ? ceil_div(td.br_hi - td.br_lo, 128) : 0;
       const int n = nkv + nbr;
       const int64_t slot = int64_t(td.row_base) + row;
       const SlotMeta m = a.meta[slot];
       const float neg_l2 = a.ls[int64_t(h) * a.n_slots + slot];
       const float dval = a.ds[int64_t(h) * a.n_slots + slot];
+      // the row's first visible main key and, for a bitmask branch row, its mask word
+      const int rlo = (kGen && a.window > 0) ? max(td.doc_start, m.limit - a.window + 1) : td.doc_start;
+      const uint64_t bits = (kGen && a.mode == 2 && m.row >= a.S) ? a.bmask[m.row - a.S] : 0ull;
       for (int j = 0; j < n; ++j) {
         const uint32_t sb = s_cnt & 1u;
         bool w = ptx::mbar_wait(bar_s_full(sb), (s_cnt >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 2, 8));
@@ -326,18 +331,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 4; ++c) ptx::tmem_regs_ready(dp[c]);
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar_dp_empty);
-        int lo, hi;
+        int lo, hi, sh = 0;
+        bool bitm = false;
         if (j < nkv) {
-          lo = 0;
-          hi = m.limit - (td.doc_start + 128 * j) + 1;
+          const int y = td.kv_lo + 128 * j;
+          lo = kGen ? rlo - y : 0;
+          hi = m.limit - y + 1;
         } else {
           const int kr0 = td.br_lo + 128 * (j - nkv);
           lo = m.blo - kr0;
           hi = m.bhi - kr0;
+          sh = lo;  // column c is branch key c - sh of the row's branch
+          bitm = kGen && a.mode == 2;
         }
         lo = max(lo, 0);
         hi = min(hi, 128);
-        const bool full = lo == 0 && hi == 128;
+        const bool full = lo == 0 && hi == 128 && !bitm;
         const float2 c2 = make_float2(sl2, sl2), nl2 = make_float2(neg_l2, neg_l2), d2 = make_float2(dval, dval);
         // dS in two halves of 64 keys: the S columns of a half are all read
         // before its 32 packed dS columns overwrite the front of the buffer.
@@ -362,7 +371,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const int col = c * 32 + i;
-                if (col < lo || col >= hi) sr[i] = __float_as_uint(-INFINITY);
+                bool out = col < lo || col >= hi;
+                if constexpr (kGen) out = out || (bitm && !((bits >> (col - sh)) & 1ull));
+                if (out) sr[i] = __float_as_uint(-INFINITY);
               }
             }
 #pragma unroll
@@ -420,24 +431,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool kGen>
 cudaError_t launch_d(const DqMaps& m, const DqArgs& a, int num_sms, cudaStream_t st) {
   using L = Smem<D>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D, kGen>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::kAlloc));
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;
-  bwd_dq_kernel<D><<<grid, kThreads, L::kAlloc, st>>>(m.qg, m.dog, m.k, m.v, m.kb, m.vb, a);
+  bwd_dq_kernel<D, kGen><<<grid, kThreads, L::kAlloc, st>>>(m.qg, m.dog, m.k, m.v, m.kb, m.vb, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_bwd_dq(const DqMaps& m, const DqArgs& a, int num_sms, cudaStream_t st) {
-  if (a.d == 128) return launch_d<128>(m, a, num_sms, st);
-  if (a.d == 64) return launch_d<64>(m, a, num_sms, st);
+  const bool gen = a.window > 0 || a.mode == 2;
+  if (a.d == 128) return gen ? launch_d<128, true>(m, a, num_sms, st) : launch_d<128, false>(m, a, num_sms, st);
+  if (a.d == 64) return gen ? launch_d<64, true>(m, a, num_sms, st) : launch_d<64, false>(m, a, num_sms, st);
   return cudaErrorInvalidValue;
 }
 

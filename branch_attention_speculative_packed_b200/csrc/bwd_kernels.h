@@ -31,6 +31,7 @@ struct BranchBwdArgs {
   const __nv_bfloat16 *qb, *kb, *vb, *dob;
   const float* lse;   // [Hq, rows]
   const float* drow;  // [Hq, rows]
+  const uint64_t* bmask;  // BA_MASK_BITMASK: [Nb*B] words
   int S, Nb, B, mode, Hq, Hkv;
   int64_t rows;
   float scale;
@@ -45,7 +46,9 @@ struct DqArgs {
   const SlotMeta* meta;
   const float* ls;  // [Hq, n_slots], -LSE * log2(e)
   const float* ds;  // [Hq, n_slots]
+  const uint64_t* bmask;  // BA_MASK_BITMASK: [Nb*B] words, else unused
   int S, Hq, G, d;
+  int mode, window;
   int64_t n_slots;
   int n_items;      // ntiles * Hq
   int with_branch;
@@ -72,6 +75,7 @@ struct DkdvArgs {
   const float* ls;  // [Hq, n_slots], -LSE * log2(e)
   const float* ds;  // [Hq, n_slots]
   int Hq, Hkv, G, d;
+  int window;   // main-prefix window (> 0), else none
   int64_t n_slots;
   int n_items;  // n_kv * Hkv
   float scale_log2, scale;

@@ -75,47 +75,128 @@ struct Bars {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// The key-tile stream of a tile pair.
+// The key-tile stream of a tile pair.  The main keys come as up to two
+// segments [sl, sh), each cut into 128-key tiles from its first key:
+//   - full rows: one segment from the first tile's first key (its document
+//     start, or later under a window) to the larger limit + 1; two segments
+//     when a window leaves a gap of at least a key tile between the tiles;
+//   - ring partial k (virtual rank k): the keys of the document's zigzag
+//     chunks k and 2R-1-k within that range.
+// Then A's branch-local key tiles, then B's.
 struct PairPlan {
   TileDesc t[2];
   bool on[2];   // tile present (the second tile of a pair may be absent)
-  int nkv[2];   // main key tiles of each tile
+  int lo[2], hi[2];  // each tile's main key range [lo, hi)
+  int nkv[2];   // plain stream: main key tiles of each tile
   int nbr[2];   // branch key tiles of each tile
-  int nmain;    // main key tiles streamed: max(nkv)
+  int sl[2], sh[2], sn[2];  // main segments and their key tiles
+  int nmain;    // main key tiles streamed: sn[0] + sn[1]
   int n;        // key tiles streamed
+  int k;        // ring partial (virtual rank) of the item, 0 for full rows
 };
 
-__device__ __forceinline__ PairPlan load_pair(const FwdArgs& a, int pair) {
+// kGen selects the general stream (window, ring partials, bitmask words); the
+// plain instantiation (full rows, chain or block masks, no window) keeps the
+// one-segment stream [doc start, larger limit] with no per-tile range checks.
+template <bool kGen>
+__device__ __forceinline__ PairPlan load_pair(const FwdArgs& a, int item) {
   PairPlan pp;
+  const int per = a.Hq * (a.ring > 0 ? a.ring : 1);
+  const int pair = item / per;
+  pp.k = a.ring > 0 ? (item / a.Hq) % a.ring : 0;
   const int2 ids = reinterpret_cast<const int2*>(a.pairs)[pair];
   const int id[2] = {ids.x, ids.y};
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     pp.on[t] = id[t] >= 0;
-    pp.nkv[t] = pp.nbr[t] = 0;
+    pp.nbr[t] = 0;
     if (pp.on[t]) {
       pp.t[t] = a.tiles[id[t]];
-      pp.nkv[t] = ceil_div(pp.t[t].kv_end - pp.t[t].doc_start, 128);
       if (a.with_branch && pp.t[t].br_hi > pp.t[t].br_lo)
         pp.nbr[t] = ceil_div(pp.t[t].br_hi - pp.t[t].br_lo, 128);
     } else {
       pp.t[t] = pp.t[0];
     }
+    pp.lo[t] = pp.t[t].kv_lo;
+    pp.hi[t] = pp.on[t] ? pp.t[t].kv_end : pp.t[t].kv_lo;
+    pp.nkv[t] = pp.on[t] ? ceil_div(pp.t[t].kv_end - pp.t[t].doc_start, 128) : 0;
   }
-  pp.nmain = max(pp.nkv[0], pp.nkv[1]);
+  if constexpr (!kGen) {
+    pp.sl[0] = pp.t[0].doc_start;
+    pp.sn[0] = max(pp.nkv[0], pp.nkv[1]);
+    pp.sh[0] = pp.sl[0] + 128 * pp.sn[0];
+    pp.sl[1] = pp.sh[1] = pp.sh[0];
+    pp.sn[1] = 0;
+    pp.nmain = pp.sn[0];
+    pp.n = pp.nmain + pp.nbr[0] + pp.nbr[1];
+    return pp;
+  }
+  const int rlo = pp.lo[0], rhi = max(pp.hi[0], pp.hi[1]);
+  if (a.ring > 0) {
+    const int s = pp.t[0].doc_start;
+    const int64_t L = pp.t[0].doc_end - s;
+    const int64_t R2 = 2 * a.ring;
+    const int c[2] = {pp.k, static_cast<int>(R2) - 1 - pp.k};
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      pp.sl[g] = max(rlo, s + static_cast<int>(c[g] * L / R2));
+      pp.sh[g] = min(rhi, s + static_cast<int>((c[g] + 1) * L / R2));
+    }
+  } else if (pp.on[1] && pp.lo[1] - pp.hi[0] >= 128) {
+    pp.sl[0] = pp.lo[0];
+    pp.sh[0] = pp.hi[0];
+    pp.sl[1] = pp.lo[1];
+    pp.sh[1] = pp.hi[1];
+  } else {
+    pp.sl[0] = rlo;
+    pp.sh[0] = rhi;
+    pp.sl[1] = pp.sh[1] = rhi;
+  }
+#pragma unroll
+  for (int g = 0; g < 2; ++g) pp.sn[g] = pp.sh[g] > pp.sl[g] ? ceil_div(pp.sh[g] - pp.sl[g], 128) : 0;
+  pp.nmain = pp.sn[0] + pp.sn[1];
   pp.n = pp.nmain + pp.nbr[0] + pp.nbr[1];
   return pp;
 }
 
+// (Fields are picked with selects, never indexed by a runtime value, so
+// PairPlan stays in registers.)
+// First key of main key tile j (< nmain) and whether it lies in segment 1.
+__device__ __forceinline__ int main_key0(const PairPlan& pp, int j, bool& s1) {
+  s1 = j >= pp.sn[0];
+  return (s1 ? pp.sl[1] : pp.sl[0]) + 128 * (j - (s1 ? pp.sn[0] : 0));
+}
+
 // Does tile t take key tile j of the stream?
+template <bool kGen>
 __device__ __forceinline__ bool takes(const PairPlan& pp, int t, int j) {
-  if (!pp.on[t]) return false;
-  if (j < pp.nmain) return j < pp.nkv[t];
+  if (!(t ? pp.on[1] : pp.on[0])) return false;
+  if (j < pp.nmain) {
+    if constexpr (!kGen) return j < (t ? pp.nkv[1] : pp.nkv[0]);
+    bool s1;
+    const int y = main_key0(pp, j, s1);
+    return max(y, t ? pp.lo[1] : pp.lo[0]) <
+           min(min(y + 128, s1 ? pp.sh[1] : pp.sh[0]), t ? pp.hi[1] : pp.hi[0]);
+  }
   j -= pp.nmain;
   return t == 0 ? j < pp.nbr[0] : j >= pp.nbr[0];
 }
 
-template <int D>
+// Index of the last key tile tile t takes (-1: none).
+template <bool kGen>
+__device__ __forceinline__ int last_taken(const PairPlan& pp, int t) {
+  if (!(t ? pp.on[1] : pp.on[0])) return -1;
+  if ((t ? pp.nbr[1] : pp.nbr[0]) > 0) return t == 0 ? pp.nmain + pp.nbr[0] - 1 : pp.n - 1;
+  if constexpr (!kGen) return (t ? pp.nkv[1] : pp.nkv[0]) - 1;
+  const int lo = t ? pp.lo[1] : pp.lo[0], hi = t ? pp.hi[1] : pp.hi[0];
+  const int e1 = min(pp.sh[1], hi);
+  if (max(pp.sl[1], lo) < e1) return pp.sn[0] + (e1 - 1 - pp.sl[1]) / 128;
+  const int e0 = min(pp.sh[0], hi);
+  if (max(pp.sl[0], lo) < e0) return (e0 - 1 - pp.sl[0]) / 128;
+  return -1;
+}
+
+template <int D, bool kGen>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
@@ -196,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t rn = 1; ok && cur < a.n_items; ++rn) {
         const int nxt = static_cast<int>(atomicAdd(a.counter, 1u));
         if (!ptx::ring_put(ring, rn, nxt, abort_flag, a.err, lim, ptx::wait_site(1, 0, 12))) { ok = false; break; }
-        const PairPlan pp = load_pair(a, cur / Hq);
+        const PairPlan pp = load_pair<kGen>(a, cur);
         const int g = (cur % Hq) / a.G;
         for (int j = 0; j < pp.n; ++j) {
           if (!ptx::mbar_wait(bar.kv_empty[kv_stage], kv_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(1, 0, 2))) {
@@ -208,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const void* mv = &tmV;
           int y;
           if (j < pp.nmain) {
-            y = pp.t[0].doc_start + 128 * j;
+            bool s1;
+            y = main_key0(pp, j, s1);
           } else {
             const int jb = j - pp.nmain;
             y = jb < pp.nbr[0] ? pp.t[0].br_lo + 128 * jb : pp.t[1].br_lo + 128 * (jb - pp.nbr[0]);
@@ -249,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int item = 0;
         if (!ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(1, 1, 13))) { ok = false; break; }
         if (item >= a.n_items) break;
-        const PairPlan pp = load_pair(a, item / Hq);
+        const PairPlan pp = load_pair<kGen>(a, item);
         bool first_s[2] = {true, true}, first_pv[2] = {true, true};
         // S_t(j) = Q_t K_j^T into tile t's S buffer (the P.V that last read it was issued before).
         auto issue_s = [&](int t, uint32_t stage) -> bool {
@@ -289,21 +371,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ptx::mbar_wait(bar.kv_full[kv_stage], kv_phase, abort_flag, a.err, lim, ptx::wait_site(1, 1, 5))) { ok = false; break; }
         ptx::tc_fence_after();
         for (int t = 0; t < 2 && ok; ++t)
-          if (takes(pp, t, 0) && !issue_s(t, kv_stage)) ok = false;
+          if (takes<kGen>(pp, t, 0) && !issue_s(t, kv_stage)) ok = false;
         for (int j = 0; j < pp.n && ok; ++j) {
           const uint32_t st_j = kv_stage;
           uint32_t st_n = kv_stage + 1, ph_n = kv_phase;
           if (st_n == kStages) { st_n = 0; ph_n ^= 1u; }
           const bool more = j + 1 < pp.n;
-          if (takes(pp, 0, j) && !issue_pv(0, st_j)) { ok = false; break; }
+          if (takes<kGen>(pp, 0, j) && !issue_pv(0, st_j)) { ok = false; break; }
           if (more) {
             if (!ptx::mbar_wait(bar.kv_full[st_n], ph_n, abort_flag, a.err, lim, ptx::wait_site(1, 1, 5))) { ok = false; break; }
             ptx::tc_fence_after();
-            if (takes(pp, 0, j + 1) && !issue_s(0, st_n)) { ok = false; break; }
+            if (takes<kGen>(pp, 0, j + 1) && !issue_s(0, st_n)) { ok = false; break; }
           }
-          if (takes(pp, 1, j) && !issue_pv(1, st_j)) { ok = false; break; }
+          if (takes<kGen>(pp, 1, j) && !issue_pv(1, st_j)) { ok = false; break; }
           ptx::umma_commit(bar.kv_empty[st_j]);
-          if (more && takes(pp, 1, j + 1) && !issue_s(1, st_n)) { ok = false; break; }
+          if (more && takes<kGen>(pp, 1, j + 1) && !issue_s(1, st_n)) { ok = false; break; }
           kv_stage = st_n;
           kv_phase = ph_n;
         }
@@ -333,7 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // This thread's row of the warpgroup's tile in a work item.
     struct RowItem {
       bool valid, on;
-      int h, n, nmain, nkv, nbr0, last, doc_start, br_lo, r, limit, blo, bhi;
+      int h, k, n, nmain, nkv, sn0, nbr0, last;
+      int sl0, sh0, sl1, sh1, tlo, thi;  // main segments and the tile's main key range
+      int br_lo, r, limit, rlo, blo, bhi;  // the row: main keys [rlo, limit], branch [blo, bhi)
+      uint64_t bits;                        // the row's branch mask word (BA_MASK_BITMASK)
     };
     auto get_item = [&](uint32_t rn, int& item) -> bool {
       return __all_sync(0xffffffffu, ptx::ring_get(ring, rn, &item, abort_flag, a.err, lim, ptx::wait_site(1, 2, 14)));
@@ -342,21 +427,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       it.valid = item < a.n_items;
       it.on = false;
       if (!it.valid) return;
-      const PairPlan pp = load_pair(a, item / Hq);
+      const PairPlan pp = load_pair<kGen>(a, item);
       it.on = t ? pp.on[1] : pp.on[0];
       if (!it.on) return;
       const TileDesc td = t ? pp.t[1] : pp.t[0];
       it.h = item % Hq;
+      it.k = pp.k;
       it.n = pp.n;
       it.nmain = pp.nmain;
       it.nkv = t ? pp.nkv[1] : pp.nkv[0];
+      it.sn0 = pp.sn[0];
       it.nbr0 = pp.nbr[0];
-      it.last = (t ? pp.nbr[1] : pp.nbr[0]) > 0 ? (t == 0 ? pp.nmain + pp.nbr[0] - 1 : pp.n - 1) : it.nkv - 1;
-      it.doc_start = td.doc_start;
+      it.last = last_taken<kGen>(pp, t);
+      it.sl0 = pp.sl[0];
+      it.sh0 = pp.sh[0];
+      it.sl1 = pp.sl[1];
+      it.sh1 = pp.sh[1];
+      it.tlo = t ? pp.lo[1] : pp.lo[0];
+      it.thi = t ? pp.hi[1] : pp.hi[0];
       it.br_lo = td.br_lo;
       it.r = a.row_table[td.row_base + row];
-      it.limit = td.doc_start;  // padding rows see one key: keeps their math finite
+      it.limit = td.doc_start;  // padding rows see at most one key: keeps their math finite
+      it.rlo = td.doc_start;
       it.blo = it.bhi = 0;      // visible branch key rows [blo, bhi)
+      it.bits = 0;
       if (it.r >= 0 && it.r < a.S) {
         it.limit = it.r;
       } else if (it.r >= a.S) {
@@ -364,16 +458,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tt = (it.r - a.S) - b * a.B;
         it.limit = a.anchors[b];
         it.blo = b * a.B;
-        it.bhi = it.blo + (a.mode == 1 ? a.B : tt + 1);
+        it.bhi = it.blo + (a.mode == 0 ? tt + 1 : a.B);
+        if (kGen && a.mode == 2) it.bits = a.bmask[it.r - a.S];
       }
+      if (kGen && a.window > 0 && it.r >= 0) it.rlo = max(td.doc_start, it.limit - a.window + 1);
     };
-    // Where this thread's query row of `item` lives (false: the tile is absent).
+    // Where this thread's query row of `item` lives (false: the tile is absent
+    // or takes no key tile of the item, so no S MMA reads its Q).
     auto q_src = [&](int item, const __nv_bfloat16*& src, uint32_t& bytes) -> bool {
       if (item >= a.n_items) return false;
-      const int2 ids = reinterpret_cast<const int2*>(a.pairs)[item / Hq];
-      const int id = t == 0 ? ids.x : ids.y;
-      if (id < 0) return false;
-      const int r = a.row_table[a.tiles[id].row_base + row];
+      int row_base;
+      if constexpr (kGen) {
+        const PairPlan pp = load_pair<kGen>(a, item);
+        if (last_taken<kGen>(pp, t) < 0) return false;
+        row_base = (t ? pp.t[1] : pp.t[0]).row_base;
+      } else {  // every present tile takes at least its first main key tile
+        const int2 ids = reinterpret_cast<const int2*>(a.pairs)[item / Hq];
+        const int id = t == 0 ? ids.x : ids.y;
+        if (id < 0) return false;
+        row_base = a.tiles[id].row_base;
+      }
+      const int r = a.row_table[row_base + row];
       const int h = item % Hq;
       src = a.q;  // padding row: zero-filled
       bytes = 0;
@@ -388,7 +493,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // Does this warpgroup's tile take key tile j of the item's stream?
     auto takes_own = [&](const RowItem& it, int j) -> bool {
-      if (j < it.nmain) return j < it.nkv;
+      if (j < it.nmain) {
+        if constexpr (!kGen) return j < it.nkv;  // the plain stream: a prefix of the main tiles
+        const bool s1 = j >= it.sn0;
+        const int y = (s1 ? it.sl1 : it.sl0) + 128 * (j - (s1 ? it.sn0 : 0));
+        return max(y, it.tlo) < min(min(y + 128, s1 ? it.sh1 : it.sh0), it.thi);
+      }
       return t == 0 ? j - it.nmain < it.nbr0 : j - it.nmain >= it.nbr0;
     };
     // Copy this thread's query row (bf16, D values) into row `row` of the
@@ -430,6 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (cur.on) {
         const int h = cur.h, nmain = cur.nmain, r = cur.r;
         const int limit = cur.limit, blo = cur.blo, bhi = cur.bhi;
+        const bool use_bits = kGen && a.mode == 2;
         float m_used = -INFINITY;
         float l = 0.f;
         bool first = true;
@@ -451,20 +562,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tc_fence_after();
           // The tile's last S MMA has finished: the next item's rows may overwrite Q.
           if (j == cur.last && nxt_on) copy_q(nsrc, nbytes);
-          // visible columns [lo, hi) of this key tile
-          int lo, hi;
+          // visible columns [lo, hi) of this key tile (and, for a bitmask
+          // branch tile, those whose bit is set: column c is branch key c - sh)
+          int lo, hi, sh = 0;
+          bool bitm = false;
           if (j < nmain) {
-            lo = 0;
-            hi = limit - (cur.doc_start + 128 * j) + 1;
+            if constexpr (kGen) {
+              const bool s1 = j >= cur.sn0;
+              const int y = (s1 ? cur.sl1 : cur.sl0) + 128 * (j - (s1 ? cur.sn0 : 0));
+              lo = max(cur.rlo, s1 ? cur.sl1 : cur.sl0) - y;
+              hi = min(limit + 1, s1 ? cur.sh1 : cur.sh0) - y;
+            } else {
+              lo = 0;
+              hi = limit - (cur.sl0 + 128 * j) + 1;
+            }
           } else {
             const int kb = t == 0 ? j - nmain : j - nmain - cur.nbr0;
             const int kr0 = cur.br_lo + 128 * kb;
             lo = blo - kr0;
             hi = bhi - kr0;
+            sh = lo;
+            bitm = use_bits;
           }
           lo = max(lo, 0);
           hi = min(hi, 128);
-          const bool full = lo == 0 && hi == 128;
+          const bool full = lo == 0 && hi == 128 && !bitm;
+          const uint64_t bits = cur.bits;
+          auto masked = [&](int col) -> bool {
+            if constexpr (!kGen) return col < lo || col >= hi;
+            return col < lo || col >= hi || (bitm && !((bits >> (col - sh)) & 1ull));
+          };
           // Pass 1: row max, 32 columns at a time, 8 independent accumulators.
           float mx8[8];
 #pragma unroll
@@ -478,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!full) {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (c * 32 + i < lo || c * 32 + i >= hi) sr[i] = __float_as_uint(-INFINITY);
+                if (masked(c * 32 + i)) sr[i] = __float_as_uint(-INFINITY);
             }
 #pragma unroll
             for (int i = 0; i < 32; i += 2)
@@ -518,7 +645,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // Pass 2: P = exp2(S * scale*log2(e) - m) as bf16 pairs over the first
           // 64 columns of S, row sum over 4 paired accumulators.
           const float2 c2 = make_float2(sl2, sl2);
-          const float2 nm2 = make_float2(-m_used, -m_used);
+          // a row with no visible key so far keeps m = -inf; subtract 0 then, so P = 0 exactly
+          const float mref = (kGen && m_used == -INFINITY) ? 0.f : m_used;
+          const float2 nm2 = make_float2(-mref, -mref);
           float2 rs4[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) rs4[u] = make_float2(0.f, 0.f);
@@ -531,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!full) {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (c * 32 + i < lo || c * 32 + i >= hi) sr[i] = __float_as_uint(-INFINITY);
+                if (masked(c * 32 + i)) sr[i] = __float_as_uint(-INFINITY);
             }
             uint32_t pw[16];
 #pragma unroll
@@ -563,13 +692,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-        const float inv_l = 1.f / l;
+        // l == 0: the row saw no key of this item (a ring partial may be
+        // empty): O = 0, LSE = -inf, whatever TMEM holds
+        const bool empty = kGen && !(l > 0.f);
+        const float inv_l = empty ? 0.f : 1.f / l;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
           ptx::tmem_ld32(tl + colO + c * 32u, ov);
           ptx::tmem_wait_ld();
           ptx::tmem_regs_ready(ov);
+          if (empty) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = 0u;
+          }
           if (r >= 0) {
             if (a.out_bf16) {
               __nv_bfloat16* dst = (r < a.S ? a.o + (int64_t(r) * Hq + h) * D
@@ -584,7 +720,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 reinterpret_cast<uint4*>(dst)[q4] = w;
               }
             } else {
-              float* dst = a.o_part + (int64_t(r) * Hq + h) * D + c * 32;
+              float* dst = a.o_part + (kGen ? int64_t(cur.k) * a.o_part_stride : 0) +
+                           (int64_t(r) * Hq + h) * D + c * 32;
 #pragma unroll
               for (int q4 = 0; q4 < 8; ++q4) {
                 float4 w;
@@ -597,7 +734,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (r >= 0) a.lse[int64_t(h) * a.lse_ld + r] = (m_used + __log2f(l)) * 0.69314718055994531f;
+        if (r >= 0)
+          a.lse[(kGen ? int64_t(cur.k) * a.lse_stride : 0) + int64_t(h) * a.lse_ld + r] =
+              empty ? -INFINITY : (m_used + __log2f(l)) * 0.69314718055994531f;
         ptx::tc_fence_before();
       }
       if (!fetched) {
@@ -626,24 +765,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool kGen>
 cudaError_t launch_fwd_d(const FwdMaps& m, const FwdArgs& a, int num_sms, cudaStream_t stream) {
   using L = Smem<D>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, kGen>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::kAlloc));
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;
-  fwd_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(m.k, m.v, m.kb, m.vb, a);
+  fwd_kernel<D, kGen><<<grid, kThreads, L::kAlloc, stream>>>(m.k, m.v, m.kb, m.vb, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd(const FwdMaps& maps, const FwdArgs& a, int num_sms, cudaStream_t stream) {
-  if (a.d == 128) return launch_fwd_d<128>(maps, a, num_sms, stream);
-  if (a.d == 64) return launch_fwd_d<64>(maps, a, num_sms, stream);
+  // the general stream only where a window, ring partials or mask words need it
+  const bool gen = a.window > 0 || a.ring > 0 || a.mode == 2;
+  if (a.d == 128) return gen ? launch_fwd_d<128, true>(maps, a, num_sms, stream)
+                             : launch_fwd_d<128, false>(maps, a, num_sms, stream);
+  if (a.d == 64) return gen ? launch_fwd_d<64, true>(maps, a, num_sms, stream)
+                            : launch_fwd_d<64, false>(maps, a, num_sms, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -19,12 +19,17 @@ struct FwdArgs {
   const int32_t* row_table;  // [ntiles * 128], -1 = padding
   const TileDesc* tiles;     // [ntiles]
   const int32_t* pairs;      // [n_pairs][2] tile indices (second -1: single), longest first
+  const uint64_t* bmask;     // BA_MASK_BITMASK: [Nb*B] words (row (b,t) sees branch key u iff bit u)
   int S, Nb, B, mode, Hq, G, d;
-  int n_items;               // n_pairs * Hq
+  int window;                // main-prefix window (> 0), else none
+  int ring;                  // R > 0: one partial per virtual rank's zigzag keys; 0: full rows
+  int n_items;               // n_pairs * Hq (* ring when ring > 0)
   float scale_log2;          // softmax scale * log2(e)
   int with_branch;           // also visit the branch key tiles (fused forward)
   int out_bf16;              // 1: bf16 o / ob; 0: fp32 o_part
-  float* o_part;             // [rows, Hq, d]
+  float* o_part;             // [rows, Hq, d] (ring: [ring, rows, Hq, d])
+  int64_t o_part_stride;     // elements between ring partials of o_part
+  int64_t lse_stride;        // elements between ring partials of lse
   __nv_bfloat16* o;          // [S, Hq, d]
   __nv_bfloat16* ob;         // [Nb*B, Hq, d]
   float* lse;                // element (h, r) at lse[h * lse_ld + r]
@@ -47,9 +52,9 @@ cudaError_t launch_plan_rows(const int32_t* cu_seqlens, int ndoc, const int32_t*
 
 // ---------------------------------------------------------------- branch part / merge
 cudaError_t launch_branch_fwd(const __nv_bfloat16* qb, const __nv_bfloat16* kb,
-                              const __nv_bfloat16* vb, int Nb, int B, int mode, int Hq, int Hkv,
-                              int d, float scale, float* o_part, float* lse_part,
-                              cudaStream_t stream);
+                              const __nv_bfloat16* vb, const uint64_t* bmask, int Nb, int B,
+                              int mode, int Hq, int Hkv, int d, float scale, float* o_part,
+                              float* lse_part, cudaStream_t stream);
 
 struct MergeArgs {
   int nparts, rows, H, d;

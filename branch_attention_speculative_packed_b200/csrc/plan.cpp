@@ -22,12 +22,27 @@ int lower_bound_i(const int32_t* a, int lo, int hi, int64_t x) {
 
 }  // namespace
 
+int64_t pair_main_tiles(const TileDesc& a, const TileDesc& b) {
+  // One stream [a.kv_lo, b.kv_end) unless a gap of at least a whole key tile
+  // separates the two tiles' ranges; then two streams.
+  const int64_t K = kKeysPerTile;
+  if (int64_t(b.kv_lo) - a.kv_end >= K)
+    return (int64_t(a.kv_end) - a.kv_lo + K - 1) / K + (int64_t(b.kv_end) - b.kv_lo + K - 1) / K;
+  const int64_t hi = std::max(a.kv_end, b.kv_end);
+  return (hi - a.kv_lo + K - 1) / K;
+}
+
 ba_status validate(const ba_problem* p, bool need_tensors) {
   if (!p) return BA_ERR_INVALID_ARG;
   if (p->S < 1 || p->ndoc < 1 || p->ndoc > p->S) return BA_ERR_INVALID_ARG;
   if (p->Hq < 1 || p->Hkv < 1 || p->Hq % p->Hkv != 0) return BA_ERR_INVALID_ARG;
   if (p->d < 1 || p->Nb < 0 || p->R < 1 || p->R > 64) return BA_ERR_INVALID_ARG;
-  if (p->mode != BA_MASK_CHAIN && p->mode != BA_MASK_BLOCK) return BA_ERR_INVALID_ARG;
+  if (p->mode != BA_MASK_CHAIN && p->mode != BA_MASK_BLOCK && p->mode != BA_MASK_BITMASK)
+    return BA_ERR_INVALID_ARG;
+  if (p->mode == BA_MASK_BITMASK && p->Nb > 0) {
+    if (!p->branch_mask_h || !p->branch_mask_d || !aligned16(p->branch_mask_d))
+      return BA_ERR_INVALID_ARG;
+  }
   if (p->Nb > 0 && (p->B < 1 || p->B > 64)) return BA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return BA_ERR_UNSUPPORTED;
   // Row indices and head-major LSE offsets must fit the kernels' int32 row math.
@@ -73,16 +88,29 @@ void build_plan(const ba_problem* p, Plan* plan) {
   plan->n_tile_pairs = plan->n_branch_tile_pairs = plan->n_visible_pairs = 0;
   plan->rank_pairs.assign(R, 0);
 
-  // Exact visible pairs per head (counting rule of the definition).
+  const int64_t W = p->window > 0 ? p->window : 0;
+  // Exact visible pairs per head (counting rule of the definition): a prefix
+  // of n main keys counts min(n, W) under a window.
   int64_t vis = 0;
   for (int i = 0; i < p->ndoc; ++i) {
     const int64_t L = cu[i + 1] - cu[i];
-    vis += L * (L + 1) / 2;
+    if (W > 0 && L > W)
+      vis += W * (W + 1) / 2 + (L - W) * W;
+    else
+      vis += L * (L + 1) / 2;
   }
   for (int b = 0; b < Nb; ++b) {
     const int di = static_cast<int>(std::upper_bound(cu, cu + p->ndoc + 1, anc[b]) - cu) - 1;
-    vis += int64_t(B) * (anc[b] - cu[di] + 1);
-    vis += (p->mode == BA_MASK_CHAIN) ? int64_t(B) * (B + 1) / 2 : int64_t(B) * B;
+    const int64_t n = anc[b] - cu[di] + 1;
+    vis += int64_t(B) * (W > 0 ? std::min(n, W) : n);
+    if (p->mode == BA_MASK_CHAIN) {
+      vis += int64_t(B) * (B + 1) / 2;
+    } else if (p->mode == BA_MASK_BLOCK) {
+      vis += int64_t(B) * B;
+    } else {
+      const uint64_t keep = B >= 64 ? ~uint64_t(0) : ((uint64_t(1) << B) - 1);
+      for (int t = 0; t < B; ++t) vis += __builtin_popcountll(p->branch_mask_h[int64_t(b) * B + t] & keep);
+    }
   }
   plan->n_visible_pairs = vis;
 
@@ -145,6 +173,9 @@ void build_plan(const ba_problem* p, Plan* plan) {
       td.doc_start = s;
       td.min_limit = limit_at(m0);
       td.kv_end = limit_at(m1 - 1) + 1;
+      td.kv_lo = W > 0 ? static_cast<int32_t>(std::max<int64_t>(s, td.min_limit - W + 1)) : s;
+      td.doc_end = e;
+      td.pad0 = td.pad1 = 0;
       td.rank = 0;
       for (int k = 0; k < 2 * R; ++k) {
         const Chunk& c = plan->chunks[chunk0 + k];
@@ -171,7 +202,7 @@ void build_plan(const ba_problem* p, Plan* plan) {
           td.br_hi = bhi * B;
         }
       }
-      const int64_t nkv = (int64_t(td.kv_end) - td.doc_start + kKeysPerTile - 1) / kKeysPerTile;
+      const int64_t nkv = (int64_t(td.kv_end) - td.kv_lo + kKeysPerTile - 1) / kKeysPerTile;
       const int64_t nbr = (int64_t(td.br_hi) - td.br_lo + kKeysPerTile - 1) / kKeysPerTile;
       plan->n_tile_pairs += nkv;
       plan->n_branch_tile_pairs += std::max<int64_t>(0, nbr);
@@ -188,7 +219,7 @@ void build_plan(const ba_problem* p, Plan* plan) {
   std::vector<int64_t> cost(nt);
   for (int i = 0; i < nt; ++i) {
     const TileDesc& td = plan->tiles[i];
-    cost[i] = (int64_t(td.kv_end) - td.doc_start + kKeysPerTile - 1) / kKeysPerTile +
+    cost[i] = (int64_t(td.kv_end) - td.kv_lo + kKeysPerTile - 1) / kKeysPerTile +
               (int64_t(td.br_hi) - td.br_lo + kKeysPerTile - 1) / kKeysPerTile;
   }
   std::stable_sort(plan->order.begin(), plan->order.end(),
@@ -202,10 +233,11 @@ void build_plan(const ba_problem* p, Plan* plan) {
     const TileDesc& ta = plan->tiles[i];
     int64_t c = cost[i];
     if (two) {
+      // the pair streams its main key tiles once (see pair_main_tiles)
       const TileDesc& tb = plan->tiles[i + 1];
-      const int64_t ma = (int64_t(ta.kv_end) - ta.doc_start + kKeysPerTile - 1) / kKeysPerTile;
-      const int64_t mb = (int64_t(tb.kv_end) - tb.doc_start + kKeysPerTile - 1) / kKeysPerTile;
-      c = cost[i] + cost[i + 1] - std::min(ma, mb);
+      const int64_t ma = (int64_t(ta.kv_end) - ta.kv_lo + kKeysPerTile - 1) / kKeysPerTile;
+      const int64_t mb = (int64_t(tb.kv_end) - tb.kv_lo + kKeysPerTile - 1) / kKeysPerTile;
+      c = cost[i] + cost[i + 1] - ma - mb + pair_main_tiles(ta, tb);
     }
     prs.emplace_back(i, two ? i + 1 : -1);
     pcost.push_back(c);
@@ -243,7 +275,18 @@ void build_kv_plan(const ba_problem* p, Plan* plan) {
       it.key0 = k0;
       it.key_end = std::min(e, k0 + kKeysPerTile);
       it.t_first = lo;
-      it.t_count = t_hi - lo;
+      int t_end = t_hi;
+      if (p->window > 0) {
+        // rows see this tile only while limit - W + 1 <= key_end - 1
+        int a = lo, c = t_hi;  // first tile whose smallest limit is beyond that
+        while (a < c) {
+          const int mid = (a + c) / 2;
+          if (int64_t(plan->tiles[mid].min_limit) - p->window + 1 > int64_t(it.key_end) - 1) c = mid;
+          else a = mid + 1;
+        }
+        t_end = a;
+      }
+      it.t_count = t_end - lo;
       plan->n_kv_pairs += it.t_count;
       plan->kv_items.push_back(it);
     }

@@ -56,6 +56,9 @@ ba_status validate(const ba_problem* p, bool need_tensors);
 // Precondition: validate(p, ...) == BA_OK.
 void build_plan(const ba_problem* p, Plan* plan);
 
+// Main key tiles a forward tile pair streams (the device kernel's rule).
+int64_t pair_main_tiles(const TileDesc& a, const TileDesc& b);
+
 // Builds the key-tile list of the dK/dV pass (after build_plan).
 void build_kv_plan(const ba_problem* p, Plan* plan);
 

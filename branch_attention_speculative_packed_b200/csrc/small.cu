@@ -61,11 +61,13 @@ __global__ void plan_rows_kernel(const int32_t* __restrict__ cu, int ndoc,
 // One block per (branch b, KV head g), one warp per query head of the group.
 // The branch's B keys and values of head g are staged in shared memory; each
 // warp walks the B rows of its head: scores against the visible branch keys
-// (chain: u <= t; block: all), softmax, O = P V.  Output fp32 O and LSE.
+// (chain: u <= t; block: all; bitmask: the row's bits), softmax, O = P V.
+// Output fp32 O and LSE.
 template <int D>
 __global__ void branch_fwd_kernel(const __nv_bfloat16* __restrict__ qb,
                                   const __nv_bfloat16* __restrict__ kb,
-                                  const __nv_bfloat16* __restrict__ vb, int Nb, int B, int mode,
+                                  const __nv_bfloat16* __restrict__ vb,
+                                  const uint64_t* __restrict__ bmask, int Nb, int B, int mode,
                                   int Hq, int Hkv, float scale, float* __restrict__ o_part,
                                   float* __restrict__ lse_part) {
   constexpr int E = D / 32;  // elements per lane
@@ -91,12 +93,14 @@ __global__ void branch_fwd_kernel(const __nv_bfloat16* __restrict__ qb,
     float qv[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) qv[e] = __bfloat162float(qb[(row * Hq + h) * D + lane * E + e]);
-    const int nvis = mode == 1 ? B : t + 1;
+    const int nvis = mode == 0 ? t + 1 : B;
+    const uint64_t bits = mode == 2 ? bmask[row] : ~0ull;
     float mx = -INFINITY, l = 0.f;
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
     for (int u = 0; u < nvis; ++u) {
+      if (!((bits >> u) & 1ull)) continue;  // bitmask: row t sees key u iff bit u is set
       float s = 0.f;
 #pragma unroll
       for (int e = 0; e < E; ++e) s = fmaf(qv[e], sk[u * D + lane * E + e], s);
@@ -111,10 +115,11 @@ __global__ void branch_fwd_kernel(const __nv_bfloat16* __restrict__ qb,
       for (int e = 0; e < E; ++e) acc[e] = acc[e] * c + p * sv[u * D + lane * E + e];
       mx = mn;
     }
-    const float inv = 1.f / l;
+    // a bitmask row may see no branch key at all: the empty partial (0, -inf)
+    const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) o_part[(row * Hq + h) * D + lane * E + e] = acc[e] * inv;
-    if (lane == 0) lse_part[int64_t(h) * nbr + row] = mx + logf(l);
+    if (lane == 0) lse_part[int64_t(h) * nbr + row] = l > 0.f ? mx + logf(l) : -INFINITY;
   }
 }
 
@@ -226,9 +231,9 @@ cudaError_t launch_plan_rows(const int32_t* cu_seqlens, int ndoc, const int32_t*
 }
 
 cudaError_t launch_branch_fwd(const __nv_bfloat16* qb, const __nv_bfloat16* kb,
-                              const __nv_bfloat16* vb, int Nb, int B, int mode, int Hq, int Hkv,
-                              int d, float scale, float* o_part, float* lse_part,
-                              cudaStream_t stream) {
+                              const __nv_bfloat16* vb, const uint64_t* bmask, int Nb, int B,
+                              int mode, int Hq, int Hkv, int d, float scale, float* o_part,
+                              float* lse_part, cudaStream_t stream) {
   if (Nb == 0) return cudaSuccess;
   const int G = Hq / Hkv;
   const int threads = G * 32 < 64 ? 64 : G * 32;
@@ -240,13 +245,13 @@ cudaError_t launch_branch_fwd(const __nv_bfloat16* qb, const __nv_bfloat16* kb,
       cudaFuncSetAttribute(branch_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
     branch_fwd_kernel<128><<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
-        qb, kb, vb, Nb, B, mode, Hq, Hkv, scale, o_part, lse_part);
+        qb, kb, vb, bmask, Nb, B, mode, Hq, Hkv, scale, o_part, lse_part);
   } else {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(branch_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
     branch_fwd_kernel<64><<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
-        qb, kb, vb, Nb, B, mode, Hq, Hkv, scale, o_part, lse_part);
+        qb, kb, vb, bmask, Nb, B, mode, Hq, Hkv, scale, o_part, lse_part);
   }
   return cudaGetLastError();
 }

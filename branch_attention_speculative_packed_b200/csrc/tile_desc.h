@@ -17,8 +17,12 @@ struct TileDesc {
   int32_t br_lo;      // branch key rows (flattened b*B+u) the tile's branch
   int32_t br_hi;      //   rows can see: [br_lo, br_hi); empty if br_lo >= br_hi
   int32_t rank;       // owning virtual rank
+  int32_t kv_lo;      // first main key any row of the tile sees (doc_start
+                      //   unless a window cuts the prefix)
+  int32_t doc_end;    // one past the last main key of the tile's document
+  int32_t pad0, pad1;
 };
-static_assert(sizeof(TileDesc) == 32, "TileDesc must stay 32 bytes");
+static_assert(sizeof(TileDesc) == 48, "TileDesc must stay 48 bytes");
 
 // Per-document data the device row scatter needs.
 struct ChunkDev {

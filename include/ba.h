@@ -78,8 +78,11 @@ typedef enum {
 } ba_status;
 
 typedef enum {
-  BA_MASK_CHAIN = 0, /* EAGLE-3 training-time test: depth t sees branch keys u <= t */
-  BA_MASK_BLOCK = 1  /* DFlash-style block draft: all B keys of its own block */
+  BA_MASK_CHAIN = 0,  /* EAGLE-3 training-time test: depth t sees branch keys u <= t */
+  BA_MASK_BLOCK = 1,  /* DFlash-style block draft: all B keys of its own block */
+  BA_MASK_BITMASK = 2 /* any per-branch pattern, e.g. for DSpark's Markov head (the
+                         pages do not spell that mask out): row (b, t) sees branch
+                         key (b, u) iff bit u of branch_mask[b * B + t] is set */
 } ba_mask_mode;
 
 enum { BA_WS_FWD = 0, BA_WS_BWD = 1 };
@@ -103,6 +106,11 @@ typedef struct {
   const void* qb; const void* kb; const void* vb;  /* device, bf16 (ignored if Nb == 0) */
   void* workspace;        /* device, 256-byte aligned, caller-owned */
   size_t workspace_bytes; /* its size */
+  int window;             /* main-prefix window W: if > 0, a row whose last main key is l
+                             sees only main keys [max(s(l), l - W + 1), l]; branch keys
+                             are not affected; <= 0: no window */
+  const uint64_t* branch_mask_h; /* BA_MASK_BITMASK only: host copy, [Nb * B] words */
+  const uint64_t* branch_mask_d; /* device copy of the same (16-byte aligned) */
 } ba_problem;
 
 /* Bytes of workspace that ba_main_fwd / ba_fused_fwd (which = BA_WS_FWD) or
@@ -121,6 +129,23 @@ BA_API size_t ba_workspace_size(const ba_problem* p, int which);
  * Paper: §3.2 (rcap.io post: the main-sequence part is computed by the
  * existing packed, load-balanced zigzag ring attention). */
 BA_API ba_status ba_main_fwd(const ba_problem* p, float* o_part, float* lse_part, ba_stream_t stream);
+
+/* Step a2 as the ring computes it: per-virtual-rank partials of the main
+ * component.  The zigzag split gives virtual rank k the keys of chunks k and
+ * 2R-1-k of every document; partial k of a row is its attention over the
+ * visible main keys among those, i.e. what the row's rank computes at the
+ * ring step where rank k's K/V visit it.  Merging the R partials of a row
+ * with ba_lse_merge (Eq. 2; R <= 16 there) gives ba_main_fwd's result.
+ *   o_parts   device fp32 [R, S + Nb*B, Hq, d]
+ *   lse_parts device fp32 [R, Hq, S + Nb*B]
+ * A row with no visible key in rank k's chunks gets the empty partial
+ * (O = 0, LSE = -inf).  Needs ba_workspace_size(p, BA_WS_FWD) bytes of
+ * workspace.  Paper: §3.2 (rcap.io post: the main-sequence part rides the
+ * packed, load-balanced zigzag ring attention, whose ring steps are merged
+ * with the log-sum-exp rule); the zigzag chunk rule itself is this library's
+ * reading: a document [s, s+L) is cut at s + floor(kL/2R). */
+BA_API ba_status ba_main_fwd_ring(const ba_problem* p, float* o_parts, float* lse_parts,
+                                  ba_stream_t stream);
 
 /* Step a3: the rank-local branch component: each branch row against its own
  * branch keys only (chain: u <= t; block: all B).  Needs no workspace.
@@ -208,7 +233,8 @@ BA_API ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, cons
  * work list).  Every entry point plans on the host from cu_seqlens_h and
  * anchors_h: the zigzag split, row tiles, their order and the key tiles of the
  * backward.  Plans are cached, keyed by the problem's sizes (S, ndoc, Hq,
- * Hkv, d, Nb, B, mode, R) and the contents of cu_seqlens_h and anchors_h, so
+ * Hkv, d, Nb, B, mode, R, window) and the contents of cu_seqlens_h, anchors_h
+ * and (bitmask mode) branch_mask_h, so
  * the forward and backward of one packing, and later steps over the same
  * packing, plan once.  The cache keeps the 16 most recently used plans.  A
  * cached plan also keeps a page-locked copy of the bytes a device call

@@ -49,10 +49,11 @@ def make_case(case, seed=7, device="cpu"):
                           device=device, R=R, cfg_name=name)
 
 
-def attn_for(problem, ba, R=None):
+def attn_for(problem, ba, R=None, **kw):
+    """The library's handle for a problem; ``kw``: window, branch_mask."""
     c = problem.cfg
     return ba.BranchAttention(problem.cu_seqlens, problem.anchors, Hq=c.Hq, Hkv=c.Hkv, d=c.d,
-                              B=c.B, mode=c.mode, R=c.R if R is None else R)
+                              B=c.B, mode=c.mode, R=c.R if R is None else R, **kw)
 
 
 def to_device(problem, device="cuda"):
@@ -63,12 +64,13 @@ def to_device(problem, device="cuda"):
     return problem
 
 
-def oracle_fwd(problem, rows=None, heads=None):
-    """(rows, O [n,Hq,d], LSE [Hq,n]) from the fp64 row-set oracle."""
+def oracle_fwd(problem, rows=None, heads=None, **kw):
+    """(rows, O [n,Hq,d], LSE [Hq,n]) from the fp64 row-set oracle; ``kw``:
+    window, branch_mask."""
     c = problem.cfg
     return orc.forward_rows(problem.q, problem.k, problem.v, problem.qb, problem.kb, problem.vb,
                             problem.cu_seqlens.numpy(), problem.anchors.numpy(), c.B, c.mode,
-                            rows=rows, heads=heads)
+                            rows=rows, heads=heads, **kw)
 
 
 def gather_rows(o, ob, rows, S):
@@ -112,7 +114,7 @@ def sub_heads(problem, groups):
     return p, heads
 
 
-def oracle_rows_by_group(problem, rows=None, groups=None, backward=False):
+def oracle_rows_by_group(problem, rows=None, groups=None, backward=False, **kw):
     """The row-set oracle over the given concatenated rows (default: all) for
     the query heads of every listed KV group (default: all), one thread per
     group.
@@ -144,11 +146,11 @@ def oracle_rows_by_group(problem, rows=None, groups=None, backward=False):
     def one(g):
         sub, _ = sub_heads(problem, [g])
         args = (sub.q, sub.k, sub.v, sub.qb, sub.kb, sub.vb)
-        _, O, L = orc.forward_rows(*args, cu, anc, c.B, c.mode, rows=rows)
+        _, O, L = orc.forward_rows(*args, cu, anc, c.B, c.mode, rows=rows, **kw)
         if not backward:
             return O, L
         _, dQ, dk, dv, dkb, dvb = orc.backward_rows(*args, sub.do, sub.dob, cu, anc, c.B, c.mode,
-                                                    rows=rows)
+                                                    rows=rows, **kw)
         return O, L, dQ, dk, dv, dkb, dvb
 
     workers = max(1, min(len(groups), os.cpu_count() or 1))

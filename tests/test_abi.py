@@ -250,3 +250,30 @@ def test_plan_cache_keeps_the_16_most_recent(ba):
     probs[0].plan_stats()    # least recent: evicted, plans again
     assert ba.plan_cache_stats()["misses"] == before["misses"] + 1
     ba.clear_cache()
+
+
+def test_visible_pairs_with_window_and_bitmask_match_oracle_count(ba):
+    """The planner's exact pair count under a main-prefix window and under
+    per-branch mask words equals the oracle's counting rule."""
+    rs = np.random.default_rng(0)
+    for trial in range(40):
+        S = int(rs.integers(1, 400))
+        nd = int(rs.integers(1, min(S, 6) + 1))
+        cuts = sorted(rs.choice(np.arange(1, S), nd - 1, replace=False).tolist()) if nd > 1 else []
+        cu = [0] + cuts + [S]
+        anc = sorted(rs.integers(0, S, int(rs.integers(0, S + 1))).tolist())
+        B = int(rs.integers(1, 9))
+        mode = int(rs.integers(0, 3))
+        W = int(rs.choice([0, 1, 3, 17, 500]))
+        bm = rs.integers(0, 2 ** B, size=(len(anc), B), dtype=np.uint64) if mode == 2 else None
+        a = ba.BranchAttention(cu, anc, Hq=2, Hkv=1, d=64, B=B, mode=mode, R=int(rs.integers(1, 9)),
+                               device="cpu", window=W, branch_mask=bm)
+        exp = orc.visible_pair_count(np.array(cu), np.array(anc, dtype=np.int64), B, mode, window=W,
+                                     branch_mask=bm)
+        assert a.plan_stats()["visible_pairs"] == exp, (trial, mode, W)
+
+
+def test_bitmask_mode_needs_its_words(ba):
+    a = ba.BranchAttention([0, 10], [3], Hq=2, Hkv=1, d=64, B=2, mode=2, device="cpu")
+    with pytest.raises(ba.BAError):
+        a.plan_stats()

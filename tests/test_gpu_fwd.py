@@ -102,15 +102,26 @@ def test_lse_merge_rejects_bad_args(ba):
         ba.lse_merge([torch.zeros(10, 2, 96, device="cuda")], [l])
 
 
-@pytest.mark.parametrize("R", [1, 2, 5, 8])
-def test_result_independent_of_R(ba, R):
-    case = ("R_sweep", [700, 301, 5], "rand60", 4, 2, 128, 3, wl.CHAIN, R)
+def test_full_rows_bit_identical_across_R(ba):
+    """R labels the row tiles with their virtual ranks (the zigzag split) but
+    does not change what the full-row forward computes: the tile list, the
+    pairs and their order are the same for every R, so the outputs are
+    bit-identical.  (The zigzag split itself is checked by the per-rank ring
+    partials in test_gpu_variants.py.)"""
+    case = ("R_sweep", [700, 301, 5], "rand60", 4, 2, 128, 3, wl.CHAIN, 1)
     cpu = make_case(case)
     rows, O, L = oracle_fwd(cpu)
     prob = to_device(make_case(case))
-    o, ob, lse = _fused(ba, prob)
-    assert max_abs(gather_rows(o, ob, rows, prob.S), O) <= TOL_O
-    assert max_abs(lse.cpu().numpy(), L) <= TOL_LSE
+    ref = None
+    for R in (1, 2, 5, 8):
+        o, ob, lse = _fused(ba, prob, R)
+        if ref is None:
+            assert max_abs(gather_rows(o, ob, rows, prob.S), O) <= TOL_O
+            assert max_abs(lse.cpu().numpy(), L) <= TOL_LSE
+            ref = (o, ob, lse)
+        else:
+            for x, y in zip((o, ob, lse), ref):
+                assert torch.equal(x, y)
 
 
 def test_fused_fwd_config_tiny(ba):
