@@ -32,7 +32,7 @@ EXPORTED = (
     "ba_bwd", "ba_status_string", "ba_sync_status", "ba_plan_stats", "ba_profile_enable",
     "ba_profile_collect", "ba_last_error_word", "ba_fused_fwd_noalloc", "ba_plan_rank_work",
     "ba_plan_fwd_pairs", "ba_plan_prepare", "ba_clear_cache", "ba_plan_cache_stats",
-    "ba_main_fwd_ring",
+    "ba_main_fwd_ring", "ba_set_wait_limit", "ba_check_bounded_wait",
 )
 
 
@@ -100,6 +100,10 @@ def lib() -> ctypes.CDLL:
         L.ba_clear_cache.restype = None
         L.ba_plan_cache_stats.argtypes = [i64p, i64p, i64p]
         L.ba_plan_cache_stats.restype = None
+        L.ba_set_wait_limit.argtypes = [ctypes.c_longlong]
+        L.ba_set_wait_limit.restype = None
+        L.ba_check_bounded_wait.argtypes = [vp]
+        L.ba_check_bounded_wait.restype = ctypes.c_int
         L.ba_last_error_word.argtypes = []
         L.ba_last_error_word.restype = ctypes.c_uint32
         L.ba_profile_enable.argtypes = [i32]
@@ -113,6 +117,18 @@ def lib() -> ctypes.CDLL:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
+
+
+def set_wait_limit(cycles: int) -> None:
+    """Bound of every device-side wait of later launches, in SM cycles (<= 0:
+    the default, about 2 s).  For testing the failure path."""
+    lib().ba_set_wait_limit(int(cycles))
+
+
+def error_word_fields(word: int) -> dict:
+    """Decode a device error word (see ba_last_error_word in include/ba.h)."""
+    return {"expired": bool(word >> 31), "kernel": (word >> 24) & 0x7f, "role": (word >> 16) & 0xff,
+            "site": (word >> 8) & 0xff, "parity": word & 1}
 
 
 def clear_cache() -> None:

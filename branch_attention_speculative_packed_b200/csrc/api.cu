@@ -2,6 +2,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <chrono>
 #include <cmath>
 #include <cstring>
@@ -28,6 +29,8 @@ __device__ uint32_t g_error_word;
 namespace {
 
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at B200 clocks
+// The limit every launch passes to its bounded waits (ba_set_wait_limit).
+std::atomic<long long> g_wait_limit{kWaitLimitCycles};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -354,7 +357,7 @@ ba_status run_fwd(const ba_problem* p, bool fused, float* o_part, void* o, void*
   a.lse_ld = rows;
   a.err = di.err;
   a.counter = reinterpret_cast<uint32_t*>(ws + w.counters_off);
-  a.wait_limit = kWaitLimitCycles;
+  a.wait_limit = g_wait_limit.load();
   ProfScope prof(fused ? "fused_fwd" : ring ? "main_fwd_ring" : "main_fwd", st);
   if (launch_fwd(maps, a, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
   return BA_OK;
@@ -602,7 +605,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   qa.dqb = static_cast<__nv_bfloat16*>(nb ? dqb : dq);
   qa.err = di.err;
   qa.counter = reinterpret_cast<uint32_t*>(ws + w.counters_off) + 1;
-  qa.wait_limit = kWaitLimitCycles;
+  qa.wait_limit = g_wait_limit.load();
   {
     ProfScope prof("bwd_dq", st);
     if (launch_bwd_dq(dm, qa, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
@@ -630,7 +633,7 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
   ka.dv = static_cast<__nv_bfloat16*>(dv);
   ka.err = di.err;
   ka.counter = reinterpret_cast<uint32_t*>(ws + w.counters_off) + 2;
-  ka.wait_limit = kWaitLimitCycles;
+  ka.wait_limit = g_wait_limit.load();
   {
     ProfScope prof("bwd_dkdv", st);
     if (launch_bwd_dkdv(km, ka, di.num_sms, st) != cudaSuccess) return BA_ERR_CUDA;
@@ -713,6 +716,20 @@ int ba_profile_collect(const char** names, double* total_ms, int* launches, int 
     ++i;
   }
   return ok ? i : -1;
+}
+
+void ba_set_wait_limit(long long cycles) {
+  g_wait_limit.store(cycles > 0 ? cycles : kWaitLimitCycles);
+}
+
+ba_status ba_check_bounded_wait(ba_stream_t stream) {
+  DeviceInfo di;
+  ba_status s = device_info(&di);
+  if (s != BA_OK) return s;
+  if (launch_bounded_wait_probe(di.err, g_wait_limit.load(), reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return BA_ERR_CUDA;
+  return BA_OK;
 }
 
 static uint32_t g_last_error_word = 0;

@@ -192,13 +192,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (*abort_flag) {
+      {
+        // our own copies land before the CTA exits (immediate on a normal exit)
         volatile int never = 0;
+        const long long dl = ptx::kDrainCycles;
         for (uint32_t i = 0; i < kSlots; ++i) {
-          if (qpend & (1u << i)) ptx::mbar_wait(bar_q_full(i), (qpar >> i) & 1u, &never, a.err, lim / 8);
-          if (opend & (1u << i)) ptx::mbar_wait(bar_o_full(i), (opar >> i) & 1u, &never, a.err, lim / 8);
+          if (qpend & (1u << i)) ptx::mbar_wait(bar_q_full(i), (qpar >> i) & 1u, &never, a.err, dl);
+          if (opend & (1u << i)) ptx::mbar_wait(bar_o_full(i), (opar >> i) & 1u, &never, a.err, dl);
         }
-        if (kv_fills) ptx::mbar_wait(bar_kv_full, (kv_fills - 1) & 1u, &never, a.err, lim / 8);
+        if (kv_fills) ptx::mbar_wait(bar_kv_full, (kv_fills - 1) & 1u, &never, a.err, dl);
       }
     }
   } else if (warp == 1) {
@@ -289,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::umma_commit(bar_drain);
       volatile int never = 0;
-      ptx::mbar_wait(bar_drain, 0, &never, a.err, lim);
+      ptx::mbar_wait(bar_drain, 0, &never, a.err, ptx::kDrainCycles);
     }
   } else {
     // ------------------------------------------------------------ P^T, dS^T / epilogue

@@ -194,13 +194,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         item = nxt;
         td = td_next;
       }
-      if (*abort_flag) {
+      {
+        // our own copies land before the CTA exits (immediate on a normal exit)
         volatile int never = 0;
+        const long long dl = ptx::kDrainCycles;
         for (uint32_t i = 0; i < kKStages; ++i)
-          if (kpend & (1u << i)) ptx::mbar_wait(bar_k_full(i), (kpar >> i) & 1u, &never, a.err, lim / 8);
+          if (kpend & (1u << i)) ptx::mbar_wait(bar_k_full(i), (kpar >> i) & 1u, &never, a.err, dl);
         for (uint32_t i = 0; i < kVStages; ++i)
-          if (vpend & (1u << i)) ptx::mbar_wait(bar_v_full(i), (vpar >> i) & 1u, &never, a.err, lim / 8);
-        if (q_fills) ptx::mbar_wait(bar_q_full, (q_fills - 1) & 1u, &never, a.err, lim / 8);
+          if (vpend & (1u << i)) ptx::mbar_wait(bar_v_full(i), (vpar >> i) & 1u, &never, a.err, dl);
+        if (q_fills) ptx::mbar_wait(bar_q_full, (q_fills - 1) & 1u, &never, a.err, dl);
       }
     }
   } else if (warp == 1) {
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::umma_commit(bar_drain);
       volatile int never = 0;
-      ptx::mbar_wait(bar_drain, 0, &never, a.err, lim);
+      ptx::mbar_wait(bar_drain, 0, &never, a.err, ptx::kDrainCycles);
     }
   } else {
     // ------------------------------------------------------------ dS / epilogue

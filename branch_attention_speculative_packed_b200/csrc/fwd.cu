@@ -310,12 +310,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cur = nxt;
       }
-      if (*abort_flag) {
-        // Let our own copies in flight land before the CTA exits (bounded).
+      {
+        // Our own copies land before the CTA exits (on a normal exit every
+        // fill was consumed, so these waits return at once).
         volatile int never = 0;
         for (int i = 0; i < kStages; ++i)
           if (pend_mask & (1u << i))
-            ptx::mbar_wait(bar.kv_full[i], (pend_par >> i) & 1u, &never, a.err, lim / 8);
+            ptx::mbar_wait(bar.kv_full[i], (pend_par >> i) & 1u, &never, a.err, ptx::kDrainCycles);
       }
     }
   } else if (warp == kWarpMma) {
@@ -393,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Drain: every MMA this thread issued completes before TMEM is freed.
       ptx::umma_commit(bar.drain);
       volatile int never = 0;
-      ptx::mbar_wait(bar.drain, 0, &never, a.err, lim);
+      ptx::mbar_wait(bar.drain, 0, &never, a.err, ptx::kDrainCycles);
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue

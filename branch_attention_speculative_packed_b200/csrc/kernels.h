@@ -56,6 +56,11 @@ cudaError_t launch_branch_fwd(const __nv_bfloat16* qb, const __nv_bfloat16* kb,
                               int mode, int Hq, int Hkv, int d, float scale, float* o_part,
                               float* lse_part, cudaStream_t stream);
 
+// One thread waits, with the bounded wait every kernel uses, on a barrier no
+// one arrives on: it gives up after `limit` cycles and records wait site
+// (kernel 4, role 0, site 1) in the device error word.
+cudaError_t launch_bounded_wait_probe(uint32_t* err, long long limit, cudaStream_t stream);
+
 struct MergeArgs {
   int nparts, rows, H, d;
   const float* o[16];

@@ -46,6 +46,12 @@ __host__ __device__ constexpr uint32_t wait_site(uint32_t kernel, uint32_t role,
   return kErrTimeout | (kernel << 24) | (role << 16) | (site << 8);
 }
 
+// Bound of the waits a CTA makes on its way out (its own TMA copies and MMAs
+// still in flight), independent of the configurable wait limit, so a short
+// limit can never let a CTA free TMEM or leave shared memory under work it
+// issued itself: about 2 s at B200 clocks.
+constexpr long long kDrainCycles = 4000000000LL;
+
 // Bounded wait on an mbarrier phase.  Gives up after ~`limit_cycles` SM
 // cycles or when another role of the CTA has raised `abort`; on expiry it
 // records where it gave up in the device error word, raises `abort` and

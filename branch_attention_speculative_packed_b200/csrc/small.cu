@@ -212,6 +212,20 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const MergeArgs a) {
   }
 }
 
+// ------------------------------------------------------------------ bounded-wait probe
+__global__ void bounded_wait_probe_kernel(uint32_t* err, long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    const uint32_t b = ptx::smem_u32(&bar);
+    ptx::mbar_init(b, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+    // nothing ever arrives: the wait gives up after `limit` cycles and reports
+    ptx::mbar_wait(b, 0, &abort_flag, err, limit, ptx::wait_site(4, 0, 1));
+  }
+}
+
 int grid_for(int64_t work, int per_block, int cap) {
   int64_t g = (work + per_block - 1) / per_block;
   if (g < 1) g = 1;
@@ -253,6 +267,11 @@ cudaError_t launch_branch_fwd(const __nv_bfloat16* qb, const __nv_bfloat16* kb,
     branch_fwd_kernel<64><<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
         qb, kb, vb, bmask, Nb, B, mode, Hq, Hkv, scale, o_part, lse_part);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bounded_wait_probe(uint32_t* err, long long limit, cudaStream_t stream) {
+  bounded_wait_probe_kernel<<<1, 32, 0, stream>>>(err, limit);
   return cudaGetLastError();
 }
 

@@ -265,9 +265,28 @@ BA_API const char* ba_status_string(ba_status s);
  * if the synchronisation failed, else BA_OK. */
 BA_API ba_status ba_sync_status(ba_stream_t stream);
 
+/* Failure detection (no counterpart on the pages).  Every wait inside the
+ * library's kernels is bounded: when it expires the kernel records where it
+ * gave up in the device error word, lets its own copies and tensor-core work
+ * in flight finish (a separate, fixed bound of about 2 s), frees its tensor
+ * memory and returns; the CUDA context stays usable.
+ * ba_set_wait_limit sets the bound, in SM clock cycles, that later launches
+ * use for their waits (<= 0 restores the default, about 2 s).  Shortening it
+ * to a few hundred cycles makes ordinary waits expire, which is how the
+ * failure path is tested; results of launches that expired are garbage.  Not
+ * thread-safe with respect to concurrent calls of the library. */
+BA_API void ba_set_wait_limit(long long cycles);
+
+/* Launches a one-thread check of the bounded wait on `stream`: it waits, with
+ * the current limit, on a barrier that nothing arrives on.  After it,
+ * ba_sync_status() must report BA_ERR_TIMEOUT with an error word naming
+ * kernel 4, role 0, wait site 1.  Returns BA_OK if the check was enqueued. */
+BA_API ba_status ba_check_bounded_wait(ba_stream_t stream);
+
 /* The device error word that the last failing ba_sync_status() reported
  * (0 if none): bit 31 set for an expired bounded wait, bits 24-30 the kernel
- * (1 forward, 2 dQ pass, 3 dK/dV pass), bits 16-23 the role (0 TMA producer,
+ * (1 forward, 2 dQ pass, 3 dK/dV pass, 4 the check above), bits 16-23 the
+ * role (0 TMA producer,
  * 1 MMA issuer, 2 softmax / gradient threads), bits 8-15 the wait site in that
  * role, bit 0 the phase parity waited for.  For diagnosing a timeout. */
 BA_API uint32_t ba_last_error_word(void);
