@@ -48,6 +48,7 @@ class BaProblem(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("window", ctypes.c_int),
         ("branch_mask_h", ctypes.c_void_p), ("branch_mask_d", ctypes.c_void_p),
+        ("cp_select", ctypes.c_int), ("cp_rank", ctypes.c_int),
     ]
 
 

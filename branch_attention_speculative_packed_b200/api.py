@@ -32,10 +32,11 @@ class BranchAttention:
     1 block (DFlash-style), 2 bitmask (``branch_mask``: [Nb, B] 64-bit words,
     row (b, t) sees branch key u iff bit u of branch_mask[b, t]); R: virtual
     zigzag ranks; scale: softmax scale (None: 1/sqrt(d)); window: main-prefix
-    window W (0: none)."""
+    window W (0: none); cp_rank: compute only virtual rank cp_rank's rows (its
+    share under context parallelism; see include/ba.h)."""
 
     def __init__(self, cu_seqlens, anchors, *, Hq, Hkv, d, B, mode, R=1, scale=None,
-                 device="cuda", window=0, branch_mask=None):
+                 device="cuda", window=0, branch_mask=None, cp_rank=None):
         self.cu_h = torch.as_tensor(cu_seqlens, dtype=torch.int32).cpu().contiguous()
         self.anc_h = torch.as_tensor(anchors, dtype=torch.int32).cpu().contiguous()
         self.device = torch.device(device)
@@ -52,6 +53,8 @@ class BranchAttention:
         self.Hq, self.Hkv, self.d, self.B, self.mode, self.R = Hq, Hkv, d, B, mode, R
         self.scale = -1.0 if scale is None else float(scale)
         self.window = int(window)
+        # None: every row; r: only the rows the zigzag split gives virtual rank r
+        self.cp_rank = None if cp_rank is None else int(cp_rank)
         self.bm_h = self.bm_d = None
         if branch_mask is not None:
             bm = torch.as_tensor(branch_mask)
@@ -74,6 +77,8 @@ class BranchAttention:
         p.anchors_h = self.anc_h.data_ptr() if self.Nb else None
         p.anchors_d = self.anc_d.data_ptr() if self.Nb else None
         p.window = self.window
+        if self.cp_rank is not None:
+            p.cp_select, p.cp_rank = 1, self.cp_rank
         if self.bm_h is not None:
             p.branch_mask_h = self.bm_h.data_ptr()
             p.branch_mask_d = self.bm_d.data_ptr()

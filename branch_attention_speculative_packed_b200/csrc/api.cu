@@ -175,7 +175,8 @@ PlanCache& plan_cache() {
 
 std::string plan_key(const ba_problem* p) {
   const int32_t dims[] = {p->S, p->ndoc, p->Hq, p->Hkv, p->d, p->Nb, p->Nb > 0 ? p->B : 0,
-                          p->mode, p->R, p->window > 0 ? p->window : 0};
+                          p->mode, p->R, p->window > 0 ? p->window : 0, p->cp_select,
+                          p->cp_select ? p->cp_rank : 0};
   std::string key(reinterpret_cast<const char*>(dims), sizeof(dims));
   key.append(reinterpret_cast<const char*>(p->cu_seqlens_h), size_t(p->ndoc + 1) * sizeof(int32_t));
   if (p->Nb > 0) key.append(reinterpret_cast<const char*>(p->anchors_h), size_t(p->Nb) * sizeof(int32_t));
@@ -268,9 +269,9 @@ ba_status stage_plan(const ba_problem* p, CachedPlan& e, const WorkspaceLayout& 
       cudaMemsetAsync(ws + w.counters_off, 0, 4 * sizeof(uint32_t), st) != cudaSuccess)
     return BA_ERR_CUDA;
   ProfScope prof("plan_rows", st);
-  if (launch_plan_rows(p->cu_seqlens_d, p->ndoc, p->anchors_d, p->S, p->Nb, e.plan.B,
-                       reinterpret_cast<const ChunkDev*>(ws + w.chunks_off),
-                       reinterpret_cast<int32_t*>(ws + w.rows_off), w.n_slots,
+  if (launch_plan_rows(reinterpret_cast<const ChunkDev*>(ws + w.chunks_off),
+                       static_cast<int>(e.plan.chunks_dev.size()), p->anchors_d, p->S, p->Nb,
+                       e.plan.B, reinterpret_cast<int32_t*>(ws + w.rows_off), w.n_slots,
                        st) != cudaSuccess)
     return BA_ERR_CUDA;
   return BA_OK;
@@ -650,6 +651,11 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
     ba_.lse = lse;
     ba_.drow = pa.drow;
     ba_.bmask = bmask;
+    ba_.cu = p->cu_seqlens_d;
+    ba_.anchors = p->anchors_d;
+    ba_.ndoc = p->ndoc;
+    ba_.R = p->R;
+    ba_.cp_rank = p->cp_select ? p->cp_rank : -1;
     ba_.S = p->S;
     ba_.Nb = p->Nb;
     ba_.B = p->B;

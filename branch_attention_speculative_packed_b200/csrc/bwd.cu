@@ -97,17 +97,36 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepArgs a) {
 }
 
 // ------------------------------------------------------------------ branch dK/dV
+// Virtual rank owning main position p: the zigzag chunk k of its document
+// [s, s + L) with s + floor(kL/2R) <= p < s + floor((k+1)L/2R) belongs to
+// rank k (k < R) or 2R-1-k.
+__device__ __forceinline__ int zigzag_owner(const int32_t* cu, int ndoc, int R, int p) {
+  int lo = 0, hi = ndoc - 1;  // last document with start <= p
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu[mid] <= p) lo = mid; else hi = mid - 1;
+  }
+  const int64_t s = cu[lo], L = cu[lo + 1] - cu[lo], R2 = 2 * R;
+  int64_t k = (int64_t(p) - s) * R2 / L;  // floor(kL/2R) <= p - s for this k
+  while (k + 1 < R2 && s + (k + 1) * L / R2 <= p) ++k;
+  return static_cast<int>(k < R ? k : R2 - 1 - k);
+}
+
 // One block per (branch b, KV head g); one warp per branch key u (strided).
 // Lane l holds elements [l*E, l*E + E) of k_u, v_u and of the accumulators.
 // For every query head of the group and every row t that sees u (chain:
 // t >= u; block: all; bitmask: bit u of row t's word):
 //   s = scale <q_t, k_u>, P = exp(s - L_t), dS = P (<dO_t, v_u> - D_t),
 //   dV_u += P dO_t, dK_u += scale dS q_t.
+// (Batching several rows' loads per warp was tried: the extra registers cost
+// more occupancy than the loads in flight gained.)
 template <int D>
 __global__ void branch_bwd_kernel(const BranchBwdArgs a) {
   constexpr int E = D / 32;
   const int b = blockIdx.x / a.Hkv;
   const int g = blockIdx.x % a.Hkv;
+  // one rank's rows: the branch belongs to the rank owning its anchor
+  if (a.cp_rank >= 0 && zigzag_owner(a.cu, a.ndoc, a.R, a.anchors[b]) != a.cp_rank) return;
   const int G = a.Hq / a.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = blockDim.x >> 5;

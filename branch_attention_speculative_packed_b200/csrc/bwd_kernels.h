@@ -32,6 +32,10 @@ struct BranchBwdArgs {
   const float* lse;   // [Hq, rows]
   const float* drow;  // [Hq, rows]
   const uint64_t* bmask;  // BA_MASK_BITMASK: [Nb*B] words
+  const int32_t* cu;      // [ndoc + 1] (one rank's rows: to find a branch's owner)
+  const int32_t* anchors; // [Nb]
+  int ndoc, R;
+  int cp_rank;            // >= 0: only the branches whose anchor virtual rank cp_rank owns
   int S, Nb, B, mode, Hq, Hkv;
   int64_t rows;
   float scale;

@@ -46,9 +46,8 @@ struct FwdMaps {
 cudaError_t launch_fwd(const FwdMaps& maps, const FwdArgs& a, int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- planning
-cudaError_t launch_plan_rows(const int32_t* cu_seqlens, int ndoc, const int32_t* anchors, int S,
-                             int Nb, int B, const ChunkDev* docs, int32_t* row_table,
-                             int64_t n_slots, cudaStream_t stream);
+cudaError_t launch_plan_rows(const ChunkDev* segs, int nseg, const int32_t* anchors, int S, int Nb,
+                             int B, int32_t* row_table, int64_t n_slots, cudaStream_t stream);
 
 // ---------------------------------------------------------------- branch part / merge
 cudaError_t launch_branch_fwd(const __nv_bfloat16* qb, const __nv_bfloat16* kb,

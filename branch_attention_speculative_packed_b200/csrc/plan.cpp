@@ -45,6 +45,8 @@ ba_status validate(const ba_problem* p, bool need_tensors) {
   }
   if (p->Nb > 0 && (p->B < 1 || p->B > 64)) return BA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return BA_ERR_UNSUPPORTED;
+  if (p->cp_select != 0 && (p->cp_select != 1 || p->cp_rank < 0 || p->cp_rank >= p->R))
+    return BA_ERR_INVALID_ARG;
   // Row indices and head-major LSE offsets must fit the kernels' int32 row math.
   const int64_t rows = (int64_t)p->S + (int64_t)p->Nb * (p->Nb > 0 ? p->B : 0);
   if (rows >= (int64_t(1) << 31) - kRowsPerTile * 4) return BA_ERR_UNSUPPORTED;
@@ -89,30 +91,17 @@ void build_plan(const ba_problem* p, Plan* plan) {
   plan->rank_pairs.assign(R, 0);
 
   const int64_t W = p->window > 0 ? p->window : 0;
-  // Exact visible pairs per head (counting rule of the definition): a prefix
-  // of n main keys counts min(n, W) under a window.
-  int64_t vis = 0;
-  for (int i = 0; i < p->ndoc; ++i) {
-    const int64_t L = cu[i + 1] - cu[i];
-    if (W > 0 && L > W)
-      vis += W * (W + 1) / 2 + (L - W) * W;
-    else
-      vis += L * (L + 1) / 2;
-  }
-  for (int b = 0; b < Nb; ++b) {
-    const int di = static_cast<int>(std::upper_bound(cu, cu + p->ndoc + 1, anc[b]) - cu) - 1;
-    const int64_t n = anc[b] - cu[di] + 1;
-    vis += int64_t(B) * (W > 0 ? std::min(n, W) : n);
-    if (p->mode == BA_MASK_CHAIN) {
-      vis += int64_t(B) * (B + 1) / 2;
-    } else if (p->mode == BA_MASK_BLOCK) {
-      vis += int64_t(B) * B;
-    } else {
-      const uint64_t keep = B >= 64 ? ~uint64_t(0) : ((uint64_t(1) << B) - 1);
-      for (int t = 0; t < B; ++t) vis += __builtin_popcountll(p->branch_mask_h[int64_t(b) * B + t] & keep);
-    }
-  }
-  plan->n_visible_pairs = vis;
+  const bool one_rank = p->cp_select != 0;
+  // sum over n in [n0, n1] of min(n, W) (W = 0: no window)
+  auto prefix_sum = [&](int64_t n0, int64_t n1) -> int64_t {
+    if (n1 < n0) return 0;
+    auto upto = [&](int64_t n) -> int64_t {  // sum over [1, n]
+      if (W > 0 && n > W) return W * (W + 1) / 2 + (n - W) * W;
+      return n * (n + 1) / 2;
+    };
+    return upto(n1) - upto(n0 - 1);
+  };
+  int64_t vis = 0;  // exact visible pairs per head of the rows this plan covers
 
   int tile_count = 0;
   for (int di = 0; di < p->ndoc; ++di) {
@@ -133,85 +122,115 @@ void build_plan(const ba_problem* p, Plan* plan) {
       c.tile0 = c.ntiles = 0;
       plan->chunks.push_back(c);
     }
-    // Row tiles over the document's rows in limit order (main row p, then the
-    // branch rows anchored at p).  A tile may cross a zigzag chunk edge; it is
-    // owned by the virtual rank whose chunk holds its first row.
-    const int b0 = Nb ? lower_bound_i(anc, 0, Nb, s) : 0;
-    const int b1 = Nb ? lower_bound_i(anc, b0, Nb, e) : 0;
-    const int64_t n_rows = L + int64_t(B) * (b1 - b0);
-    const int ntiles = static_cast<int>((n_rows + kRowsPerTile - 1) / kRowsPerTile);
-    ChunkDev cd;
-    cd.c0 = s;
-    cd.b0 = b0;
-    cd.slot_base = tile_count * kRowsPerTile;
-    cd.pad = 0;
-    plan->chunks_dev.push_back(cd);
-    // merged index of main position q within the document
-    auto main_index = [&](int q) -> int64_t {
-      const int lb = Nb ? lower_bound_i(anc, b0, b1, q) : 0;
-      return int64_t(q - s) + int64_t(B) * (lb - b0);
-    };
-    // limit of the row at merged index m: largest q in [s, e) with main_index(q) <= m
-    auto limit_at = [&](int64_t m) -> int {
-      int lo = s, hi = e - 1;
-      while (lo < hi) {
-        const int mid = lo + (hi - lo + 1) / 2;
-        if (main_index(mid) <= m) lo = mid; else hi = mid - 1;
-      }
-      return lo;
-    };
-    // first merged index of branch b's rows
-    auto branch_start = [&](int b) -> int64_t {
-      return int64_t(anc[b] - s) + 1 + int64_t(B) * (b - b0);
-    };
-    for (int t = 0; t < ntiles; ++t) {
-      const int64_t m0 = int64_t(t) * kRowsPerTile;
-      const int64_t m1 = std::min<int64_t>(n_rows, m0 + kRowsPerTile);
-      TileDesc td;
-      td.row_base = (tile_count + t) * kRowsPerTile;
-      td.n_rows = static_cast<int32_t>(m1 - m0);
-      td.doc_start = s;
-      td.min_limit = limit_at(m0);
-      td.kv_end = limit_at(m1 - 1) + 1;
-      td.kv_lo = W > 0 ? static_cast<int32_t>(std::max<int64_t>(s, td.min_limit - W + 1)) : s;
-      td.doc_end = e;
-      td.pad0 = td.pad1 = 0;
-      td.rank = 0;
-      for (int k = 0; k < 2 * R; ++k) {
-        const Chunk& c = plan->chunks[chunk0 + k];
-        if (c.c0 <= td.min_limit && td.min_limit < c.c1) td.rank = c.rank;
-      }
-      td.br_lo = td.br_hi = 0;
-      if (b1 > b0) {
-        // branches whose rows [start, start + B) meet [m0, m1)
-        int lo = b0, hi = b1;  // first b with start(b) + B > m0
-        while (lo < hi) {
-          const int mid = (lo + hi) / 2;
-          if (branch_start(mid) + B > m0) hi = mid; else lo = mid + 1;
-        }
-        const int blo = lo;
-        lo = b0;
-        hi = b1;  // first b with start(b) >= m1
-        while (lo < hi) {
-          const int mid = (lo + hi) / 2;
-          if (branch_start(mid) >= m1) hi = mid; else lo = mid + 1;
-        }
-        const int bhi = lo;  // exclusive
-        if (bhi > blo) {
-          td.br_lo = blo * B;
-          td.br_hi = bhi * B;
-        }
-      }
-      const int64_t nkv = (int64_t(td.kv_end) - td.kv_lo + kKeysPerTile - 1) / kKeysPerTile;
-      const int64_t nbr = (int64_t(td.br_hi) - td.br_lo + kKeysPerTile - 1) / kKeysPerTile;
-      plan->n_tile_pairs += nkv;
-      plan->n_branch_tile_pairs += std::max<int64_t>(0, nbr);
-      plan->rank_pairs.resize(R, 0);
-      plan->rank_pairs[td.rank] += nkv;
-      plan->tiles.push_back(td);
+    // The row segments of this document the plan covers: the whole document,
+    // or (one rank's rows) the rank's two zigzag chunks, positions [c0, c1)
+    // with the branches anchored there.
+    int seg_lo[2], seg_hi[2], nseg = 0;
+    if (!one_rank) {
+      seg_lo[0] = s;
+      seg_hi[0] = e;
+      nseg = 1;
+    } else {
+      const Chunk& ca = plan->chunks[chunk0 + p->cp_rank];
+      const Chunk& cb = plan->chunks[chunk0 + 2 * R - 1 - p->cp_rank];
+      if (ca.c1 > ca.c0) { seg_lo[nseg] = ca.c0; seg_hi[nseg] = ca.c1; ++nseg; }
+      if (cb.c1 > cb.c0) { seg_lo[nseg] = cb.c0; seg_hi[nseg] = cb.c1; ++nseg; }
     }
-    tile_count += ntiles;
+    for (int sg = 0; sg < nseg; ++sg) {
+      // Row tiles over the segment's rows in limit order (main row p, then
+      // the branch rows anchored at p).  A tile may cross a zigzag chunk edge
+      // (whole documents); it is owned by the virtual rank whose chunk holds
+      // its first row.
+      const int c0 = seg_lo[sg], c1 = seg_hi[sg];
+      const int b0 = Nb ? lower_bound_i(anc, 0, Nb, c0) : 0;
+      const int b1 = Nb ? lower_bound_i(anc, b0, Nb, c1) : 0;
+      const int64_t n_rows = int64_t(c1 - c0) + int64_t(B) * (b1 - b0);
+      const int ntiles = static_cast<int>((n_rows + kRowsPerTile - 1) / kRowsPerTile);
+      vis += prefix_sum(c0 - s + 1, c1 - s);
+      for (int b = b0; b < b1; ++b) {
+        vis += int64_t(B) * prefix_sum(anc[b] - s + 1, anc[b] - s + 1);
+        if (p->mode == BA_MASK_CHAIN) {
+          vis += int64_t(B) * (B + 1) / 2;
+        } else if (p->mode == BA_MASK_BLOCK) {
+          vis += int64_t(B) * B;
+        } else {
+          const uint64_t keep = B >= 64 ? ~uint64_t(0) : ((uint64_t(1) << B) - 1);
+          for (int t = 0; t < B; ++t) vis += __builtin_popcountll(p->branch_mask_h[int64_t(b) * B + t] & keep);
+        }
+      }
+      ChunkDev cd;
+      cd.c0 = c0;
+      cd.b0 = b0;
+      cd.slot_base = tile_count * kRowsPerTile;
+      cd.pad = c1;
+      plan->chunks_dev.push_back(cd);
+      // merged index of main position q within the segment
+      auto main_index = [&](int q) -> int64_t {
+        const int lb = Nb ? lower_bound_i(anc, b0, b1, q) : 0;
+        return int64_t(q - c0) + int64_t(B) * (lb - b0);
+      };
+      // limit of the row at merged index m: largest q in [c0, c1) with main_index(q) <= m
+      auto limit_at = [&](int64_t m) -> int {
+        int lo = c0, hi = c1 - 1;
+        while (lo < hi) {
+          const int mid = lo + (hi - lo + 1) / 2;
+          if (main_index(mid) <= m) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+      };
+      // first merged index of branch b's rows
+      auto branch_start = [&](int b) -> int64_t {
+        return int64_t(anc[b] - c0) + 1 + int64_t(B) * (b - b0);
+      };
+      for (int t = 0; t < ntiles; ++t) {
+        const int64_t m0 = int64_t(t) * kRowsPerTile;
+        const int64_t m1 = std::min<int64_t>(n_rows, m0 + kRowsPerTile);
+        TileDesc td;
+        td.row_base = (tile_count + t) * kRowsPerTile;
+        td.n_rows = static_cast<int32_t>(m1 - m0);
+        td.doc_start = s;
+        td.min_limit = limit_at(m0);
+        td.kv_end = limit_at(m1 - 1) + 1;
+        td.kv_lo = W > 0 ? static_cast<int32_t>(std::max<int64_t>(s, td.min_limit - W + 1)) : s;
+        td.doc_end = e;
+        td.pad0 = td.pad1 = 0;
+        td.rank = 0;
+        for (int k = 0; k < 2 * R; ++k) {
+          const Chunk& c = plan->chunks[chunk0 + k];
+          if (c.c0 <= td.min_limit && td.min_limit < c.c1) td.rank = c.rank;
+        }
+        td.br_lo = td.br_hi = 0;
+        if (b1 > b0) {
+          // branches whose rows [start, start + B) meet [m0, m1)
+          int lo = b0, hi = b1;  // first b with start(b) + B > m0
+          while (lo < hi) {
+            const int mid = (lo + hi) / 2;
+            if (branch_start(mid) + B > m0) hi = mid; else lo = mid + 1;
+          }
+          const int blo = lo;
+          lo = b0;
+          hi = b1;  // first b with start(b) >= m1
+          while (lo < hi) {
+            const int mid = (lo + hi) / 2;
+            if (branch_start(mid) >= m1) hi = mid; else lo = mid + 1;
+          }
+          const int bhi = lo;  // exclusive
+          if (bhi > blo) {
+            td.br_lo = blo * B;
+            td.br_hi = bhi * B;
+          }
+        }
+        const int64_t nkv = (int64_t(td.kv_end) - td.kv_lo + kKeysPerTile - 1) / kKeysPerTile;
+        const int64_t nbr = (int64_t(td.br_hi) - td.br_lo + kKeysPerTile - 1) / kKeysPerTile;
+        plan->n_tile_pairs += nkv;
+        plan->n_branch_tile_pairs += std::max<int64_t>(0, nbr);
+        plan->rank_pairs[td.rank] += nkv;
+        plan->tiles.push_back(td);
+      }
+      tile_count += ntiles;
+    }
   }
+  plan->n_visible_pairs = vis;
   // Longest-processing-time-first order over the key tiles each row tile visits.
   const int nt = static_cast<int>(plan->tiles.size());
   plan->order.resize(nt);

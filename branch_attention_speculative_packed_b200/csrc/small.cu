@@ -11,17 +11,20 @@ namespace ba {
 namespace {
 
 // ------------------------------------------------------------------ plan rows
-// Writes every concatenated row index r (main rows 0..S-1, then branch rows
-// S + b*B + t) into its slot of the row table.  Within a document starting at
-// s the rows are ordered by limit (main row p: p; branch row: its anchor),
-// main row first on ties, then branches in index order, depth-minor:
-//   main p:       m = (p - s) + B * (#anchors in [s, p))
-//   branch (b,t): m = (a_b - s) + 1 + B * (b - b0) + t
-// where b0 is the document's first branch.
-__global__ void plan_rows_kernel(const int32_t* __restrict__ cu, int ndoc,
+// Writes every covered concatenated row index r (main rows 0..S-1, then
+// branch rows S + b*B + t) into its slot of the row table.  The plan covers
+// row segments (whole documents, or one virtual rank's zigzag chunks): main
+// positions [c0, c1) and the branches anchored there, in position order.
+// Within a segment the rows are ordered by limit (main row p: p; branch row:
+// its anchor), main row first on ties, then branches in index order,
+// depth-minor:
+//   main p:       m = (p - c0) + B * (#anchors in [c0, p))
+//   branch (b,t): m = (a_b - c0) + 1 + B * (b - b0) + t
+// where b0 is the segment's first branch.  Rows outside every segment are
+// skipped.
+__global__ void plan_rows_kernel(const ChunkDev* __restrict__ segs, int nseg,
                                  const int32_t* __restrict__ anchors, int S, int Nb, int B,
-                                 const ChunkDev* __restrict__ docs, int32_t* __restrict__ rows,
-                                 int64_t n_slots) {
+                                 int32_t* __restrict__ rows, int64_t n_slots) {
   const int64_t total = int64_t(S) + int64_t(Nb) * B;
   for (int64_t r = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; r < total;
        r += int64_t(gridDim.x) * blockDim.x) {
@@ -35,12 +38,13 @@ __global__ void plan_rows_kernel(const int32_t* __restrict__ cu, int ndoc,
       t = static_cast<int>(q - int64_t(b) * B);
       lim = anchors[b];
     }
-    int lo = 0, hi = ndoc - 1;  // last document with start <= lim
+    int lo = 0, hi = nseg - 1;  // last segment with c0 <= lim
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (cu[mid] <= lim) lo = mid; else hi = mid - 1;
+      if (segs[mid].c0 <= lim) lo = mid; else hi = mid - 1;
     }
-    const ChunkDev c = docs[lo];
+    const ChunkDev c = segs[lo];
+    if (lim < c.c0 || lim >= c.pad) continue;  // not a covered row
     int64_t m;
     if (!br) {
       int a0 = 0, a1 = Nb;  // first anchor >= lim
@@ -235,12 +239,12 @@ int grid_for(int64_t work, int per_block, int cap) {
 
 }  // namespace
 
-cudaError_t launch_plan_rows(const int32_t* cu_seqlens, int ndoc, const int32_t* anchors, int S,
-                             int Nb, int B, const ChunkDev* docs, int32_t* row_table,
-                             int64_t n_slots, cudaStream_t stream) {
+cudaError_t launch_plan_rows(const ChunkDev* segs, int nseg, const int32_t* anchors, int S, int Nb,
+                             int B, int32_t* row_table, int64_t n_slots, cudaStream_t stream) {
   const int64_t total = int64_t(S) + int64_t(Nb) * B;
+  if (nseg <= 0) return cudaSuccess;
   plan_rows_kernel<<<grid_for(total, 256, 148 * 16), 256, 0, stream>>>(
-      cu_seqlens, ndoc, anchors, S, Nb, B, docs, row_table, n_slots);
+      segs, nseg, anchors, S, Nb, B, row_table, n_slots);
   return cudaGetLastError();
 }
 

@@ -24,12 +24,14 @@ struct TileDesc {
 };
 static_assert(sizeof(TileDesc) == 48, "TileDesc must stay 48 bytes");
 
-// Per-document data the device row scatter needs.
+// A row segment of the plan (a whole document, or one zigzag chunk of it
+// when the plan covers one virtual rank's rows): what the device row scatter
+// needs.
 struct ChunkDev {
-  int32_t c0;        // first main position of the document
-  int32_t b0;        // first branch anchored in the document
+  int32_t c0;        // first main position of the segment
+  int32_t b0;        // first branch anchored in the segment
   int32_t slot_base; // row-table slot of merged index 0
-  int32_t pad;
+  int32_t pad;       // one past the last main position of the segment
 };
 static_assert(sizeof(ChunkDev) == 16, "ChunkDev must stay 16 bytes");
 

@@ -111,7 +111,22 @@ typedef struct {
                              are not affected; <= 0: no window */
   const uint64_t* branch_mask_h; /* BA_MASK_BITMASK only: host copy, [Nb * B] words */
   const uint64_t* branch_mask_d; /* device copy of the same (16-byte aligned) */
+  int cp_select;          /* 0: every row; 1: only the rows the zigzag split gives
+                             virtual rank cp_rank (its two chunks of every document
+                             and the branches anchored there) -- one rank's share
+                             under context parallelism; see the notes below */
+  int cp_rank;            /* 0 <= cp_rank < R when cp_select = 1 */
 } ba_problem;
+
+/* One rank's rows (cp_select = 1).  Every entry point then computes only the
+ * rows of virtual rank cp_rank, against the full main K/V (which a context-
+ * parallel caller all-gathers first): the forward writes O / LSE of those rows
+ * alone; ba_bwd writes dQ of those rows, dK / dV of the branches anchored in
+ * the rank's chunks, and a partial dK / dV of every main key -- the
+ * contributions of this rank's rows only, zero for keys none of them sees --
+ * which the ranks then sum.  Rows, keys and branches outside stay untouched
+ * except for those partial main-key gradients.  ba_plan_stats counts the
+ * rank's rows. */
 
 /* Bytes of workspace that ba_main_fwd / ba_fused_fwd (which = BA_WS_FWD) or
  * ba_bwd (which = BA_WS_BWD) need for this problem.  Returns 0 if the problem

@@ -277,3 +277,29 @@ def test_bitmask_mode_needs_its_words(ba):
     a = ba.BranchAttention([0, 10], [3], Hq=2, Hkv=1, d=64, B=2, mode=2, device="cpu")
     with pytest.raises(ba.BAError):
         a.plan_stats()
+
+
+def test_one_rank_plans_partition_the_rows(ba):
+    """The plans of the R virtual ranks' rows (cp_rank) split the work: their
+    visible-pair counts add up to the whole problem's, each rank's pairs are
+    within a few percent of the mean for long documents (the zigzag balance),
+    and an out-of-range rank is refused."""
+    rs = np.random.default_rng(3)
+    for trial in range(12):
+        S = int(rs.integers(2, 3000))
+        nd = int(rs.integers(1, min(S, 5) + 1))
+        cuts = sorted(rs.choice(np.arange(1, S), nd - 1, replace=False).tolist()) if nd > 1 else []
+        cu = [0] + cuts + [S]
+        anc = sorted(rs.integers(0, S, int(rs.integers(0, S + 1))).tolist())
+        R = int(rs.integers(1, 9))
+        W = int(rs.choice([0, 50]))
+        kw = dict(Hq=2, Hkv=1, d=64, B=3, mode=0, R=R, device="cpu", window=W)
+        whole = ba.BranchAttention(cu, anc, **kw).plan_stats()["visible_pairs"]
+        parts = [ba.BranchAttention(cu, anc, cp_rank=r, **kw).plan_stats()["visible_pairs"] for r in range(R)]
+        assert sum(parts) == whole, (trial, parts, whole)
+    big = [ba.BranchAttention([0, 65536], list(range(65536)), Hq=1, Hkv=1, d=64, B=3, mode=0, R=8,
+                              device="cpu", cp_rank=r).plan_stats()["visible_pairs"] for r in range(8)]
+    assert max(big) / min(big) < 1.01
+    with pytest.raises(ba.BAError):
+        ba.BranchAttention([0, 10], [1], Hq=1, Hkv=1, d=64, B=1, mode=0, R=2, device="cpu",
+                           cp_rank=2).plan_stats()

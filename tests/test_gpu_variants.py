@@ -173,3 +173,54 @@ def test_ring_partials_match_oracle_and_merge(ba, idx, R, W):
     ba.sync_status()
     assert max_abs(mo.double().cpu().numpy(), Om) <= TOL_O
     assert max_abs(ml.cpu().numpy(), Lm) <= TOL_LSE
+
+
+# --------------------------------------------------------------------------- one rank's rows
+
+CP_CASES = [(1, 3), (2, 4), (4, 8), (9, 2), (7, 5)]
+
+
+@pytest.mark.parametrize("idx,R", CP_CASES, ids=[f"{SMALL_CASES[i][0]}-R{R}" for i, R in CP_CASES])
+def test_one_rank_rows_assemble_the_whole_problem(ba, idx, R):
+    """Context parallelism emulated on one GPU: each virtual rank r computes
+    only its zigzag rows (cp_rank = r) against the full K/V; the union of the
+    ranks' rows and the sum of their partial main-key gradients must equal the
+    oracle's forward and backward of the whole problem.  The ranks run one
+    after another: no kernel waits on another."""
+    from branch_attention_speculative_packed_b200.cp import zigzag_rows
+    cpu = make_case(SMALL_CASES[idx])
+    c = cpu.cfg
+    cu, anc = cpu.cu_seqlens.numpy(), cpu.anchors.numpy()
+    prob = to_device(make_case(SMALL_CASES[idx]))
+    S, Nb, B = prob.S, prob.Nb, c.B
+    nan = float("nan")
+    o_all = torch.full_like(prob.q, nan)
+    ob_all = torch.full((Nb, B, c.Hq, c.d), nan, dtype=torch.bfloat16, device="cuda")
+    lse_all = torch.full((c.Hq, S + Nb * B), nan, dtype=torch.float32, device="cuda")
+    dq_all, dqb_all = torch.full_like(prob.q, nan), torch.full_like(prob.qb, nan)
+    dkb_all, dvb_all = torch.full_like(prob.kb, nan), torch.full_like(prob.vb, nan)
+    dk_sum = torch.zeros(prob.k.shape, dtype=torch.float32, device="cuda")
+    dv_sum = torch.zeros_like(dk_sum)
+    for r in range(R):
+        m, b = (t.cuda() for t in zigzag_rows(cu, anc, R, r))
+        rows = torch.cat([m, (S + b[:, None] * B + torch.arange(B, device="cuda")).reshape(-1)])
+        a = attn_for(prob, ba, R=R, cp_rank=r)
+        o, ob, lse = a.fused_fwd(prob.q, prob.k, prob.v, prob.qb, prob.kb, prob.vb)
+        g = a.bwd(prob.q, prob.k, prob.v, prob.qb, prob.kb, prob.vb, o, ob, lse, prob.do, prob.dob)
+        ba.sync_status()
+        o_all[m], ob_all[b], lse_all[:, rows] = o[m], ob[b], lse[:, rows]
+        dq_all[m], dqb_all[b], dkb_all[b], dvb_all[b] = g[0][m], g[3][b], g[4][b], g[5][b]
+        dk_sum += g[1].float()
+        dv_sum += g[2].float()
+    rows, O, L = oracle_fwd(cpu)
+    assert max_abs(gather_rows(o_all, ob_all, rows, S), O) <= TOL_O
+    assert max_abs(lse_all.cpu().numpy(), L) <= TOL_LSE
+    _, dQ, dk, dv, dkb, dvb = orc.backward_rows(cpu.q, cpu.k, cpu.v, cpu.qb, cpu.kb, cpu.vb, cpu.do,
+                                                cpu.dob, cu, anc, B, c.mode)
+    assert max_abs(_np(dq_all), dQ[:S]) <= TOL_GRAD
+    assert max_abs(dk_sum.double().cpu().numpy(), dk) <= TOL_GRAD
+    assert max_abs(dv_sum.double().cpu().numpy(), dv) <= TOL_GRAD
+    if Nb:
+        assert max_abs(_np(dqb_all).reshape(-1, c.Hq, c.d), dQ[S:]) <= TOL_GRAD
+        assert max_abs(_np(dkb_all), dkb) <= TOL_GRAD
+        assert max_abs(_np(dvb_all), dvb) <= TOL_GRAD
