@@ -248,15 +248,18 @@ def kernel_flops(kind: str, d: int, pairs: int, Hq: int) -> float:
     return 2.0 * g * d * pairs * Hq
 
 
-def merge_bandwidth(ba, cfg, rows: int, dev, world: int, hbm_gbs: float, parts: int = 2) -> dict:
+def merge_bandwidth(ba, cfg, rows: int, dev, world: int, hbm_gbs: float, parts: int = 2,
+                    d: int = None) -> dict:
     """HBM bandwidth of the k-way Eq. 2 merge (`ba_lse_merge`) over `rows`
-    rows of the workload's head layout: k fp32 partials in, bf16 O and fp32
-    LSE out; inputs far larger than L2, timed with CUDA events."""
+    rows of the workload's head layout (head dim `d`, default the
+    workload's): k fp32 partials in, bf16 O and fp32 LSE out; inputs far
+    larger than L2, timed with CUDA events."""
     import torch
+    d = cfg.d if d is None else d
     g = torch.Generator(device=dev).manual_seed(2024)
-    o_parts = [torch.randn(rows, cfg.Hq, cfg.d, device=dev, generator=g) for _ in range(parts)]
+    o_parts = [torch.randn(rows, cfg.Hq, d, device=dev, generator=g) for _ in range(parts)]
     lse_parts = [torch.randn(cfg.Hq, rows, device=dev, generator=g) * 4.0 for _ in range(parts)]
-    o = torch.empty(rows, cfg.Hq, cfg.d, dtype=torch.bfloat16, device=dev)
+    o = torch.empty(rows, cfg.Hq, d, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(cfg.Hq, rows, dtype=torch.float32, device=dev)
     for _ in range(2):
         ba.lse_merge(o_parts, lse_parts, out=(o, lse))
@@ -270,10 +273,10 @@ def merge_bandwidth(ba, cfg, rows: int, dev, world: int, hbm_gbs: float, parts: 
     e1.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
-    nbytes = rows * cfg.Hq * (parts * (4 * cfg.d + 4) + 2 * cfg.d + 4)
+    nbytes = rows * cfg.Hq * (parts * (4 * d + 4) + 2 * d + 4)
     gbs = nbytes / (ms / 1e3) / 1e9
     del o_parts, lse_parts, o, lse
-    return {"kernel": "lse_merge", "parts": parts, "rows": rows, "bytes_per_launch": nbytes,
+    return {"kernel": "lse_merge", "parts": parts, "rows": rows, "d": d, "bytes_per_launch": nbytes,
             "ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "peak_gbs": hbm_gbs,
             "frac": round(gbs / hbm_gbs, 4)}
 
@@ -432,8 +435,30 @@ def run_gpu(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = total_useful * e2e_steps / (e2e_ms / 1e3) / 1e12
 
-    merge = merge_bandwidth(ba, cfg, Nb * cfg.B if Nb else S, dev, world,
-                            float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    merge = merge_bandwidth(ba, cfg, Nb * cfg.B if Nb else S, dev, world, hbm)
+    merge_d64 = merge_bandwidth(ba, cfg, Nb * cfg.B if Nb else S, dev, world, hbm, d=64)
+
+    # The literal three-step forward of the decomposition: main component over
+    # every row (fp32 partial), branch-local component, Eq. 2 merge of the
+    # branch rows (k = 2) and the main rows' conversion (k = 1), against the
+    # fused kernel that does all three in one pass.
+    def three_step():
+        om, lm = a.main_fwd(prob.q, prob.k, prob.v, prob.qb, prob.kb, prob.vb)
+        obr, lbr = a.branch_fwd(prob.q, prob.k, prob.v, prob.qb, prob.kb, prob.vb)
+        ba.lse_merge([om[S:], obr], [lm[:, S:], lbr],
+                     out=(ob.view(-1, cfg.Hq, cfg.d), lse[:, S:]))
+        ba.lse_merge([om[:S]], [lm[:, :S]], out=(o, lse[:, :S]))
+    three_step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(3):
+        three_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ba.sync_status()
+    three_ms = max_over_ranks(t0.elapsed_time(t1) / 3, world, dev)
 
     result = {
         "metric": METRIC,
@@ -467,6 +492,9 @@ def run_gpu(args):
         "host_plan_ms": dict(host_plan_ms, note="cold host planning per packing; every step "
                                                 "reuses the cached plan"),
         "merge": merge,
+        "merge_d64": merge_d64,
+        "three_step_fwd": {"ms": round(three_ms, 3), "fused_fwd_ms": round(per_kernel["fused_fwd"]["ms_per_launch"], 3),
+                           "steps": "ba_main_fwd + ba_branch_fwd + ba_lse_merge (branch rows k=2, main rows k=1)"},
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline and widx == WORKLOAD_INDEX:

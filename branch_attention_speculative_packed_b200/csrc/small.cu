@@ -129,15 +129,18 @@ __global__ void branch_fwd_kernel(const __nv_bfloat16* __restrict__ qb,
 
 // ------------------------------------------------------------------ LSE merge
 // One warp per (head h, group of 32 rows).  Lane j first merges the LSEs of
-// row r0 + j (coalesced over rows), then the warp walks the 32 rows and each
-// lane rescales-and-adds a 16-byte slice of every part's O row (coalesced
-// over d), writing bf16 O and fp32 LSE.
+// row r0 + j (coalesced over rows); then D/8 lanes cover one row, each lane 8
+// consecutive elements: two 16-byte fp32 loads per part and one 16-byte bf16
+// store, 32/(D/8) rows per warp instruction and two such row sets in flight.
 template <int D>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const MergeArgs a) {
-  constexpr int E = D / 32;  // 4 (float4) for D=128, 2 (float2) for D=64
+  constexpr int TPR = D / 8;      // lanes per row
+  constexpr int RPI = 32 / TPR;   // rows per warp instruction
+  constexpr int U = 2;            // row sets per iteration
   const int64_t groups = (int64_t(a.rows) + 31) / 32;
   const int64_t nwarps = groups * a.H;
   const int lane = threadIdx.x & 31;
+  const int sub = lane % TPR, rsel = lane / TPR;
   for (int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32; w < nwarps;
        w += (int64_t(gridDim.x) * blockDim.x) / 32) {
     const int h = static_cast<int>(w % a.H);
@@ -165,52 +168,49 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const MergeArgs a) {
     if (live) a.lse_out[int64_t(h) * a.lse_out_ld + my] = Lr;
     const int64_t left = int64_t(a.rows) - r0;
     const int nr = left < 32 ? static_cast<int>(left) : 32;
-    // Four rows at a time, so each warp keeps 4 x nparts row loads in flight.
-    for (int i0 = 0; i0 < nr; i0 += 4) {
-      float acc[4][E];
+    for (int i0 = 0; i0 < nr; i0 += RPI * U) {
+      float acc[U][8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < U; ++u)
 #pragma unroll
-        for (int e = 0; e < E; ++e) acc[u][e] = 0.f;
+        for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
 #pragma unroll
       for (int p = 0; p < 16; ++p) {
         if (p >= a.nparts) break;
-        float v[4][E];
+        float4 v[U][2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t base = ((r0 + i0 + u) * a.H + h) * D + lane * E;
-          if (i0 + u < nr) {
-            if constexpr (E == 4) {
-              const float4 x = *reinterpret_cast<const float4*>(a.o[p] + base);
-              v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
-            } else {
-              const float2 x = *reinterpret_cast<const float2*>(a.o[p] + base);
-              v[u][0] = x.x; v[u][1] = x.y;
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < E; ++e) v[u][e] = 0.f;
+        for (int u = 0; u < U; ++u) {
+          const int i = i0 + u * RPI + rsel;
+          v[u][0] = v[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (i < nr) {
+            const float4* src = reinterpret_cast<const float4*>(a.o[p] + ((r0 + i) * a.H + h) * D + sub * 8);
+            v[u][0] = src[0];
+            v[u][1] = src[1];
           }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float wp = __shfl_sync(0xffffffffu, wt[p], (i0 + u) & 31);
-#pragma unroll
-          for (int e = 0; e < E; ++e) acc[u][e] = fmaf(wp, v[u][e], acc[u][e]);
+        for (int u = 0; u < U; ++u) {
+          const float wp = __shfl_sync(0xffffffffu, wt[p], (i0 + u * RPI + rsel) & 31);
+          acc[u][0] = fmaf(wp, v[u][0].x, acc[u][0]);
+          acc[u][1] = fmaf(wp, v[u][0].y, acc[u][1]);
+          acc[u][2] = fmaf(wp, v[u][0].z, acc[u][2]);
+          acc[u][3] = fmaf(wp, v[u][0].w, acc[u][3]);
+          acc[u][4] = fmaf(wp, v[u][1].x, acc[u][4]);
+          acc[u][5] = fmaf(wp, v[u][1].y, acc[u][5]);
+          acc[u][6] = fmaf(wp, v[u][1].z, acc[u][6]);
+          acc[u][7] = fmaf(wp, v[u][1].w, acc[u][7]);
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (i0 + u >= nr) break;
-        const int64_t base = ((r0 + i0 + u) * a.H + h) * D + lane * E;
-        if constexpr (E == 4) {
-          uint2 o;
-          o.x = ptx::pack_bf16x2(acc[u][0], acc[u][1]);
-          o.y = ptx::pack_bf16x2(acc[u][2], acc[u][3]);
-          *reinterpret_cast<uint2*>(a.o_out + base) = o;
-        } else {
-          *reinterpret_cast<uint32_t*>(a.o_out + base) = ptx::pack_bf16x2(acc[u][0], acc[u][1]);
-        }
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * RPI + rsel;
+        if (i >= nr) continue;
+        uint4 o;
+        o.x = ptx::pack_bf16x2(acc[u][0], acc[u][1]);
+        o.y = ptx::pack_bf16x2(acc[u][2], acc[u][3]);
+        o.z = ptx::pack_bf16x2(acc[u][4], acc[u][5]);
+        o.w = ptx::pack_bf16x2(acc[u][6], acc[u][7]);
+        *reinterpret_cast<uint4*>(a.o_out + ((r0 + i) * a.H + h) * D + sub * 8) = o;
       }
     }
   }
