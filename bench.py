@@ -378,63 +378,68 @@ def run_gpu(args):
     # host-to-device copies on one stream, compute on another, device-to-host
     # copies on a third, with two device buffer sets so step k+1's inputs and
     # step k-1's outputs move while step k computes.
-    names = ("q", "k", "v", "qb", "kb", "vb", "do", "dob")
-    host = {name: getattr(prob, name).cpu().pin_memory() for name in names}
-    dev_in = [{name: torch.empty_like(getattr(prob, name)) for name in names} for _ in range(2)]
-    dev_out = [(o, ob, lse) + grads,
-               tuple(torch.empty_like(t) for t in (o, ob, lse) + grads)]
-    outs_h = [t.new_empty(t.shape, device="cpu").pin_memory() for t in dev_out[0]]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs_h)
-    s_h2d, s_comp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev = {kind: [torch.cuda.Event() for _ in range(2)]
-          for kind in ("in_ready", "in_free", "out_ready", "out_free")}
+    e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 6))
+    e2e = None
+    if e2e_steps:
+        names = ("q", "k", "v", "qb", "kb", "vb", "do", "dob")
+        host = {name: getattr(prob, name).cpu().pin_memory() for name in names}
+        dev_in = [{name: torch.empty_like(getattr(prob, name)) for name in names} for _ in range(2)]
+        dev_out = [(o, ob, lse) + grads,
+                   tuple(torch.empty_like(t) for t in (o, ob, lse) + grads)]
+        outs_h = [t.new_empty(t.shape, device="cpu").pin_memory() for t in dev_out[0]]
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs_h)
+        s_h2d, s_comp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = {kind: [torch.cuda.Event() for _ in range(2)]
+              for kind in ("in_ready", "in_free", "out_ready", "out_free")}
 
-    def e2e_step(k: int):
-        b = k % 2
-        if k >= 2:
-            s_h2d.wait_event(ev["in_free"][b])
-        with torch.cuda.stream(s_h2d):
-            for name, t in host.items():
-                dev_in[b][name].copy_(t, non_blocking=True)
-        ev["in_ready"][b].record(s_h2d)
-        s_comp.wait_event(ev["in_ready"][b])
-        if k >= 2:
-            s_comp.wait_event(ev["out_free"][b])
-        x = dev_in[b]
-        oo, oob, olse = dev_out[b][:3]
-        with torch.cuda.stream(s_comp):
-            a.fused_fwd(x["q"], x["k"], x["v"], x["qb"], x["kb"], x["vb"], out=(oo, oob, olse))
-            a.bwd(x["q"], x["k"], x["v"], x["qb"], x["kb"], x["vb"], oo, oob, olse, x["do"], x["dob"],
-                  out=dev_out[b][3:])
-        ev["in_free"][b].record(s_comp)
-        ev["out_ready"][b].record(s_comp)
-        s_d2h.wait_event(ev["out_ready"][b])
-        with torch.cuda.stream(s_d2h):
-            for dst, src in zip(outs_h, dev_out[b]):
-                dst.copy_(src, non_blocking=True)
-        ev["out_free"][b].record(s_d2h)
+        def e2e_step(k: int):
+            b = k % 2
+            if k >= 2:
+                s_h2d.wait_event(ev["in_free"][b])
+            with torch.cuda.stream(s_h2d):
+                for name, t in host.items():
+                    dev_in[b][name].copy_(t, non_blocking=True)
+            ev["in_ready"][b].record(s_h2d)
+            s_comp.wait_event(ev["in_ready"][b])
+            if k >= 2:
+                s_comp.wait_event(ev["out_free"][b])
+            x = dev_in[b]
+            oo, oob, olse = dev_out[b][:3]
+            with torch.cuda.stream(s_comp):
+                a.fused_fwd(x["q"], x["k"], x["v"], x["qb"], x["kb"], x["vb"], out=(oo, oob, olse))
+                a.bwd(x["q"], x["k"], x["v"], x["qb"], x["kb"], x["vb"], oo, oob, olse, x["do"], x["dob"],
+                      out=dev_out[b][3:])
+            ev["in_free"][b].record(s_comp)
+            ev["out_ready"][b].record(s_comp)
+            s_d2h.wait_event(ev["out_ready"][b])
+            with torch.cuda.stream(s_d2h):
+                for dst, src in zip(outs_h, dev_out[b]):
+                    dst.copy_(src, non_blocking=True)
+            ev["out_free"][b].record(s_d2h)
 
-    e2e_steps = max(3, min(args.steps, 6))
-    for k in range(2):  # warm-up of the pipeline
-        e2e_step(k)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s_h2d)
-    s_comp.wait_event(e0)
-    s_d2h.wait_event(e0)
-    for k in range(2, 2 + e2e_steps):
-        e2e_step(k)
-    s_d2h.wait_event(ev["out_ready"][(1 + e2e_steps) % 2])
-    e1.record(s_d2h)
-    torch.cuda.synchronize()
-    ba.sync_status()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e_value = total_useful * e2e_steps / (e2e_ms / 1e3) / 1e12
+        for k in range(2):  # warm-up of the pipeline
+            e2e_step(k)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s_h2d)
+        s_comp.wait_event(e0)
+        s_d2h.wait_event(e0)
+        for k in range(2, 2 + e2e_steps):
+            e2e_step(k)
+        s_d2h.wait_event(ev["out_ready"][(1 + e2e_steps) % 2])
+        e1.record(s_d2h)
+        torch.cuda.synchronize()
+        ba.sync_status()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e_value = total_useful * e2e_steps / (e2e_ms / 1e3) / 1e12
 
+        e2e = {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "pipelined": "h2d / compute / d2h on three streams, two buffer sets"}
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     merge = merge_bandwidth(ba, cfg, Nb * cfg.B if Nb else S, dev, world, hbm)
     merge_d64 = merge_bandwidth(ba, cfg, Nb * cfg.B if Nb else S, dev, world, hbm, d=64)
@@ -485,9 +490,7 @@ def run_gpu(args):
                      "peak_source": f"{peak_src} bf16_tflops_sustained"},
         "kernels": {k: {"ms": round(v["ms_per_launch"], 4), "launches": v["launches"],
                         "share": round(v["share"], 4)} for k, v in per_kernel.items()},
-        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "pipelined": "h2d / compute / d2h on three streams, two buffer sets"},
+        "e2e": e2e,
         "gpu_launches": launches,
         "host_plan_ms": dict(host_plan_ms, note="cold host planning per packing; every step "
                                                 "reuses the cached plan"),
@@ -545,6 +548,8 @@ def main():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffers) leg, for lines of the other workloads")
     ap.add_argument("--workload", default="eagle3_64k",
                     help="configuration name (default: the 64K headline); others are parity-test "
                          "sizes, useful for small profiling captures")
