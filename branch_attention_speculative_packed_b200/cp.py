@@ -81,10 +81,12 @@ class ContextParallelBranchAttention:
     # ------------------------------------------------------------------ exchange
     def gather_main(self, x_local):
         """All-gather of a main-row tensor [n_main, ...] of every rank into the
-        full packed tensor [S, ...] (one collective; bf16 moves as its bits)."""
+        full packed tensor [S, ...] (one collective; 16-bit floats move as their
+        bytes, which every backend carries)."""
         n = x_local.shape[0]
-        tail = x_local.shape[1:]
-        wire = x_local.view(torch.int16) if x_local.dtype == torch.bfloat16 else x_local
+        raw = x_local.element_size() == 2
+        wire = x_local.contiguous().view(torch.uint8) if raw else x_local
+        tail = wire.shape[1:]
         buf = wire.new_zeros((self.n_max,) + tuple(tail))
         buf[:n] = wire
         parts = [torch.empty_like(buf) for _ in range(self.world)]
@@ -92,7 +94,7 @@ class ContextParallelBranchAttention:
         full = wire.new_empty((self.S,) + tuple(tail))
         for j, (m, _) in enumerate(self.shares):
             full[m] = parts[j][: m.numel()]
-        return full.view(x_local.dtype) if x_local.dtype == torch.bfloat16 else full
+        return full.view(x_local.dtype) if raw else full
 
     def _full(self, x_local, n_rows, is_branch):
         """Place this rank's rows into a zero-filled full-size buffer."""

@@ -224,3 +224,64 @@ def test_one_rank_rows_assemble_the_whole_problem(ba, idx, R):
         assert max_abs(_np(dqb_all).reshape(-1, c.Hq, c.d), dQ[S:]) <= TOL_GRAD
         assert max_abs(_np(dkb_all), dkb) <= TOL_GRAD
         assert max_abs(_np(dvb_all), dvb) <= TOL_GRAD
+
+
+# --------------------------------------------------------------------------- context parallelism over NCCL
+
+def _cp_worker(port, out):
+    import os
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.join(root, "tests"))
+    import torch.distributed as dist
+    try:
+        torch.cuda.set_device(0)
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+        from branch_attention_speculative_packed_b200.cp import ContextParallelBranchAttention
+        cpu = make_case(SMALL_CASES[1])
+        c = cpu.cfg
+        prob = to_device(make_case(SMALL_CASES[1]))
+        cp = ContextParallelBranchAttention(prob.cu_seqlens, prob.anchors, Hq=c.Hq, Hkv=c.Hkv, d=c.d, B=c.B,
+                                            mode=c.mode, device="cuda")
+        m, b = cp.main_pos, cp.branch_ids
+        o, ob, lse = cp.forward(prob.q[m], prob.k[m], prob.v[m], prob.qb[b], prob.kb[b], prob.vb[b])
+        g = cp.backward(prob.do[m], prob.dob[b])
+        torch.cuda.synchronize()
+        rows, O, L = oracle_fwd(cpu)
+        S = prob.S
+        err_o = max_abs(gather_rows(o, ob, rows, S), O)
+        err_l = max_abs(lse.cpu().numpy(), L)
+        _, dQ, dk, dv, dkb, dvb = orc.backward_rows(cpu.q, cpu.k, cpu.v, cpu.qb, cpu.kb, cpu.vb, cpu.do,
+                                                    cpu.dob, cpu.cu_seqlens.numpy(), cpu.anchors.numpy(),
+                                                    c.B, c.mode)
+        err_g = max(max_abs(_np(g[0]), dQ[:S]), max_abs(_np(g[1]), dk), max_abs(_np(g[2]), dv),
+                    max_abs(_np(g[3]).reshape(-1, c.Hq, c.d), dQ[S:]), max_abs(_np(g[4]), dkb),
+                    max_abs(_np(g[5]), dvb))
+        dist.destroy_process_group()
+        out.put((err_o, err_l, err_g))
+    except Exception as e:
+        out.put(repr(e))
+
+
+def test_context_parallel_driver_over_nccl_one_rank():
+    """The context-parallel driver end to end with NCCL and the CUDA kernels on
+    a one-rank group (this pool gives one GPU per call): the all-gather and the
+    all-reduce run through NCCL, the kernels through cp_rank = 0, and the
+    result matches the oracle.  Multi-rank runs are covered by the gloo tests
+    on CPU."""
+    import socket
+    import torch.multiprocessing as mp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    p = ctx.Process(target=_cp_worker, args=(port, out))
+    p.start()
+    res = out.get(timeout=300)
+    p.join(timeout=60)
+    assert not isinstance(res, str), res
+    err_o, err_l, err_g = res
+    assert err_o <= TOL_O and err_l <= TOL_LSE and err_g <= TOL_GRAD, res

@@ -29,6 +29,7 @@ def _source(handle, src, device, errq):
         w = TapWriter(handle, src)
         for mb in range(1, N_MB + 1):
             w.write(_tap(src, mb, device), mb, timeout_s=60)
+        del w, handle  # drop the mapped slots before telling the owner we are done
         errq.put((src, None))
     except Exception as e:  # reported to the owner
         errq.put((src, repr(e)))
