@@ -40,7 +40,16 @@
 namespace ba {
 namespace {
 
-constexpr int kThreads = 320;
+// Gradient warpgroups: each takes 128 / NWG of a sub-tile's query rows for
+// its keys (one key per thread).  Four of them (d = 128) halve every thread's
+// share of the S^T / dP^T work and put four gradient warps on each scheduler.
+template <int D>
+struct Roles {
+  static constexpr int kNWG = D == 128 ? 4 : 2;
+  static constexpr int kCW = 128 / kNWG;              // query rows (columns of S^T) per warpgroup
+  static constexpr int kGrad = 128 * kNWG;            // gradient threads
+  static constexpr int kThreads = 64 + kGrad;         // + TMA producer warp, MMA warp
+};
 constexpr int kSlots = 2;  // Q and dO ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;
@@ -74,11 +83,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 
 // kWin: a main-prefix window is in use (masking from below as well).
 template <int D, bool kWin>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<D>::kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const DkdvArgs a) {
   using L = Smem<D>;
+  constexpr int kNWG = Roles<D>::kNWG, kCW = Roles<D>::kCW, kGrad = Roles<D>::kGrad;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -111,15 +121,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(bar_o_empty(i), 1);
     }
     ptx::mbar_init(bar_s_full, 1);
-    ptx::mbar_init(bar_p_ready, 256);
+    ptx::mbar_init(bar_p_ready, kGrad);
     ptx::mbar_init(bar_dp_full, 1);
-    ptx::mbar_init(bar_ds_ready, 256);
+    ptx::mbar_init(bar_ds_ready, kGrad);
     ptx::mbar_init(bar_acc_full, 1);
-    ptx::mbar_init(bar_acc_free, 256);
+    ptx::mbar_init(bar_acc_free, kGrad);
     ptx::mbar_init(bar_drain, 1);
     for (uint32_t i = 0; i < ptx::kItemSlots; ++i) {
       ptx::mbar_init(ring.full + 8 * i, 1);
-      ptx::mbar_init(ring.empty + 8 * i, 257);  // MMA issuer + 256 gradient threads
+      ptx::mbar_init(ring.empty + 8 * i, 1 + kGrad);  // MMA issuer + the gradient threads
     }
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -229,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t qd0 = ptx::sdesc_sw128(sbase + L::kQ0 + qslot * L::kQSlot, 16384u, 1024u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            ptx::umma_ts(tmem + kColDK, tmem + kColDP + (kk >> 2) * 64u + (kk & 3) * 8u,
+            ptx::umma_ts(tmem + kColDK, tmem + kColDP + (kk / (kCW / 16)) * kCW + (kk % (kCW / 16)) * 8u,
                          ptx::sdesc_add(qd0, kk * 2048u), kIdG, (!first_dk || kk > 0) ? 1u : 0u);
           first_dk = false;
           ptx::umma_commit(bar_q_empty(qslot));
@@ -269,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t ogd0 = ptx::sdesc_sw128(so, 16384u, 1024u);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              ptx::umma_ts(tmem + kColDV, tmem + kColS + (kk >> 2) * 64u + (kk & 3) * 8u,
+              ptx::umma_ts(tmem + kColDV, tmem + kColS + (kk / (kCW / 16)) * kCW + (kk % (kCW / 16)) * 8u,
                            ptx::sdesc_add(ogd0, kk * 2048u), kIdG, (!first_dv || kk > 0) ? 1u : 0u);
             first_dv = false;
             ptx::umma_commit(bar_o_empty(os));
@@ -295,11 +305,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ P^T, dS^T / epilogue
+    constexpr int kNC = kCW / 32;          // 32-column chunks per warpgroup
     const int quarter = warp & 3;
-    const int wg = (warp - 2) >> 2;        // which 64 query rows of a sub-tile
+    const int wg = (warp - 2) >> 2;        // which kCW query rows of a sub-tile
     const int row = quarter * 32 + lane;   // key row within the tile
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t half_col = static_cast<uint32_t>(wg) * 64u;
+    const uint32_t wg_col = static_cast<uint32_t>(wg) * kCW;
     const float sl2 = a.scale_log2;
     // window: a row with limit l sees keys >= l - W + 1; with no window W is
     // huge, so that bound never bites
@@ -333,20 +344,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           ptx::tc_fence_after();
-          uint32_t sv[2][32];
-          ptx::tmem_ld32(tl + kColS + half_col, sv[0]);
-          ptx::tmem_ld32(tl + kColS + half_col + 32u, sv[1]);
+          uint32_t sv[kNC][32];
+#pragma unroll
+          for (int c = 0; c < kNC; ++c) ptx::tmem_ld32(tl + kColS + wg_col + c * 32u, sv[c]);
           ptx::tmem_wait_ld();
-          ptx::tmem_regs_ready(sv[0]);
-          ptx::tmem_regs_ready(sv[1]);
+#pragma unroll
+          for (int c = 0; c < kNC; ++c) ptx::tmem_regs_ready(sv[c]);
           const uint8_t* sq = smem + L::kQ0 + qs * L::kQSlot;
-          const float4* L4 = reinterpret_cast<const float4*>(sq + L::kSL) + wg * 16;  // -L * log2(e)
-          const float4* D4 = reinterpret_cast<const float4*>(sq + L::kSD) + wg * 16;
-          const int* Lim = reinterpret_cast<const int*>(sq + L::kSLim) + wg * 64;
+          const float4* L4 = reinterpret_cast<const float4*>(sq + L::kSL) + wg * (kCW / 4);  // -L * log2(e)
+          const float4* D4 = reinterpret_cast<const float4*>(sq + L::kSD) + wg * (kCW / 4);
+          const int* Lim = reinterpret_cast<const int*>(sq + L::kSLim) + wg * kCW;
           // exponent arguments S^T * scale*log2(e) - L*log2(e), two rows per instruction
           const float2 c2 = make_float2(sl2, sl2);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
+          for (int q = 0; q < kCW / 4; ++q) {
             const float4 l = L4[q];
             const int c = q >> 3, i = (q & 7) * 4;
             const float2 x0 = ptx::fma2(make_float2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])), c2,
@@ -365,19 +376,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           // limit's window start as well.
           bool full = warp_last_key <= Lim[0];
           if constexpr (kWin) {
-            int mx = max(Lim[lane], Lim[lane + 32]);
+            int mx = Lim[lane];
+#pragma unroll
+            for (int c = 1; c < kNC; ++c) mx = max(mx, Lim[c * 32 + lane]);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             full = full && warp_first_key >= mx - W + 1;
           }
           if (!full) {
 #pragma unroll
-            for (int col = 0; col < 64; ++col)
+            for (int col = 0; col < kCW; ++col)
               if (kp > Lim[col] || (kWin && kp < Lim[col] - W + 1)) sv[col >> 5][col & 31] = __float_as_uint(-INFINITY);
           }
-          uint32_t pk[32];
+          uint32_t pk[kCW / 2];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < kCW / 2; ++j) {
             const int c = j >> 4, i = (j & 15) * 2;
             // every other pair on the FMA pipe, the rest on the special-function unit
             const float2 xx = make_float2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
@@ -386,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[c][i + 1] = __float_as_uint(pp.y);
             pk[j] = ptx::pack_bf16x2(pp.x, pp.y);  // lower row in the low half
           }
-          ptx::tmem_st32(tl + kColS + half_col, pk);
+          if constexpr (kCW == 64) ptx::tmem_st32(tl + kColS + wg_col, pk); else ptx::tmem_st16(tl + kColS + wg_col, pk);
           ptx::tmem_wait_st();
           ptx::tc_fence_before();
           ptx::mbar_arrive(bar_p_ready);
@@ -396,14 +409,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           ptx::tc_fence_after();
-          uint32_t pv[2][32];
-          ptx::tmem_ld32(tl + kColDP + half_col, pv[0]);
-          ptx::tmem_ld32(tl + kColDP + half_col + 32u, pv[1]);
-          ptx::tmem_wait_ld();
-          ptx::tmem_regs_ready(pv[0]);
-          ptx::tmem_regs_ready(pv[1]);
+          uint32_t pv[kNC][32];
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
+          for (int c = 0; c < kNC; ++c) ptx::tmem_ld32(tl + kColDP + wg_col + c * 32u, pv[c]);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < kNC; ++c) ptx::tmem_regs_ready(pv[c]);
+#pragma unroll
+          for (int q = 0; q < kCW / 4; ++q) {
             const float4 dd = D4[q];
             const int c = q >> 3, i = (q & 7) * 4;
             const float2 g0 = ptx::mul2(make_float2(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])),
@@ -415,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[q * 2] = ptx::pack_bf16x2(g0.x, g0.y);
             pk[q * 2 + 1] = ptx::pack_bf16x2(g1.x, g1.y);
           }
-          ptx::tmem_st32(tl + kColDP + half_col, pk);
+          if constexpr (kCW == 64) ptx::tmem_st32(tl + kColDP + wg_col, pk); else ptx::tmem_st16(tl + kColDP + wg_col, pk);
           ptx::tmem_wait_st();
           ptx::tc_fence_before();
           ptx::mbar_arrive(bar_ds_ready);
@@ -434,20 +447,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
       const bool own = kp < it.key_end && any;
       const bool zero = kp < it.key_end && !any;
-      // each warpgroup writes half of the D columns of dK and of dV
+      // each warpgroup writes D / kNWG (= 32) of the D columns of dK and of dV
+      static_assert(D / kNWG == 32, "one 32-column chunk per warpgroup");
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         __nv_bfloat16* out = which == 0 ? a.dk : a.dv;
         const float mul = which == 0 ? a.scale : 1.f;
-        const uint32_t col0 = (which == 0 ? kColDK : kColDV) + static_cast<uint32_t>(wg) * (D / 2);
+        const uint32_t col0 = (which == 0 ? kColDK : kColDV) + static_cast<uint32_t>(wg) * (D / kNWG);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / kNWG / 32; ++c) {
           uint32_t v[32];
           ptx::tmem_ld32(tl + col0 + c * 32u, v);
           ptx::tmem_wait_ld();
           ptx::tmem_regs_ready(v);
           if (own || zero) {
-            __nv_bfloat16* dst = out + (int64_t(kp) * a.Hkv + g) * D + wg * (D / 2) + c * 32;
+            __nv_bfloat16* dst = out + (int64_t(kp) * a.Hkv + g) * D + wg * (D / kNWG) + c * 32;
             const float z = zero ? 0.f : mul;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
@@ -483,7 +497,7 @@ cudaError_t launch_d(const DkdvMaps& m, const DkdvArgs& a, int num_sms, cudaStre
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;
-  bwd_dkdv_kernel<D, kWin><<<grid, kThreads, L::kAlloc, st>>>(m.k, m.v, m.qg, m.dog, a);
+  bwd_dkdv_kernel<D, kWin><<<grid, Roles<D>::kThreads, L::kAlloc, st>>>(m.k, m.v, m.qg, m.dog, a);
   return cudaGetLastError();
 }
 

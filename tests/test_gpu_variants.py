@@ -144,6 +144,17 @@ def test_bitmask_fwd_bwd_and_branch_part(ba, case):
     assert np.abs(got[fin] - exp[fin]).max() <= TOL_LSE
 
 
+def test_bitmask_with_window(ba):
+    """Both variants at once: mask words on the branch keys, a window on the
+    main prefix."""
+    case = BITMASK_CASES[1]
+    cpu = make_case(case)
+    words = _mask_words(7, cpu.Nb, cpu.cfg.B)
+    prob = to_device(make_case(case))
+    fwd, grads = _fwd_bwd(ba, prob, branch_mask=words, window=45)
+    _check_against_oracle(cpu, prob, fwd, grads, branch_mask=words, window=45)
+
+
 # --------------------------------------------------------------------------- ring partials
 
 RING_CASES = [(0, 1, 0), (0, 2, 0), (1, 3, 0), (2, 4, 0), (4, 8, 0), (9, 5, 0), (9, 2, 200),
@@ -177,11 +188,11 @@ def test_ring_partials_match_oracle_and_merge(ba, idx, R, W):
 
 # --------------------------------------------------------------------------- one rank's rows
 
-CP_CASES = [(1, 3), (2, 4), (4, 8), (9, 2), (7, 5)]
+CP_CASES = [(1, 3, 0), (2, 4, 0), (4, 8, 0), (9, 2, 0), (7, 5, 0), (9, 3, 150)]
 
 
-@pytest.mark.parametrize("idx,R", CP_CASES, ids=[f"{SMALL_CASES[i][0]}-R{R}" for i, R in CP_CASES])
-def test_one_rank_rows_assemble_the_whole_problem(ba, idx, R):
+@pytest.mark.parametrize("idx,R,W", CP_CASES, ids=[f"{SMALL_CASES[i][0]}-R{R}-W{W}" for i, R, W in CP_CASES])
+def test_one_rank_rows_assemble_the_whole_problem(ba, idx, R, W):
     """Context parallelism emulated on one GPU: each virtual rank r computes
     only its zigzag rows (cp_rank = r) against the full K/V; the union of the
     ranks' rows and the sum of their partial main-key gradients must equal the
@@ -204,7 +215,7 @@ def test_one_rank_rows_assemble_the_whole_problem(ba, idx, R):
     for r in range(R):
         m, b = (t.cuda() for t in zigzag_rows(cu, anc, R, r))
         rows = torch.cat([m, (S + b[:, None] * B + torch.arange(B, device="cuda")).reshape(-1)])
-        a = attn_for(prob, ba, R=R, cp_rank=r)
+        a = attn_for(prob, ba, R=R, cp_rank=r, window=W)
         o, ob, lse = a.fused_fwd(prob.q, prob.k, prob.v, prob.qb, prob.kb, prob.vb)
         g = a.bwd(prob.q, prob.k, prob.v, prob.qb, prob.kb, prob.vb, o, ob, lse, prob.do, prob.dob)
         ba.sync_status()
@@ -212,11 +223,11 @@ def test_one_rank_rows_assemble_the_whole_problem(ba, idx, R):
         dq_all[m], dqb_all[b], dkb_all[b], dvb_all[b] = g[0][m], g[3][b], g[4][b], g[5][b]
         dk_sum += g[1].float()
         dv_sum += g[2].float()
-    rows, O, L = oracle_fwd(cpu)
+    rows, O, L = oracle_fwd(cpu, window=W)
     assert max_abs(gather_rows(o_all, ob_all, rows, S), O) <= TOL_O
     assert max_abs(lse_all.cpu().numpy(), L) <= TOL_LSE
     _, dQ, dk, dv, dkb, dvb = orc.backward_rows(cpu.q, cpu.k, cpu.v, cpu.qb, cpu.kb, cpu.vb, cpu.do,
-                                                cpu.dob, cu, anc, B, c.mode)
+                                                cpu.dob, cu, anc, B, c.mode, window=W)
     assert max_abs(_np(dq_all), dQ[:S]) <= TOL_GRAD
     assert max_abs(dk_sum.double().cpu().numpy(), dk) <= TOL_GRAD
     assert max_abs(dv_sum.double().cpu().numpy(), dv) <= TOL_GRAD
