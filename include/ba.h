@@ -212,7 +212,7 @@ BA_API ba_status ba_fused_fwd(const ba_problem* p, void* o, void* ob, float* lse
  * table and row table) from a file-scope device array inside the library instead of
  * p->workspace, which is ignored along with p->workspace_bytes.
  *   - Capacity: BA_STATIC_SCRATCH_BYTES (8 MiB), enough for problems of up to
- *     about 1.9 million rows (S + Nb*B).  Every GPU that loads the library
+ *     about 1.8 million rows (S + Nb*B).  Every GPU that loads the library
  *     holds this array until the process exits.  A problem whose plan needs
  *     more returns BA_ERR_SCRATCH_LIMIT before anything is enqueued.
  *   - The first call on a device looks up the array's device address
