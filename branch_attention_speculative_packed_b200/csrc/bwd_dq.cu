@@ -19,8 +19,12 @@
 // separate rings: V_j is released as soon as dP_j has run, K_j only after
 // dQ_j, so K gets the deeper ring.
 //
-// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-5
-// one query row per thread.  Shared memory (D = head dim): Q | dO | 3 x K |
+// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer X (S_j,
+// dQ_j), warps 2-5 one query row per thread, warp 6 MMA issuer Y (dP_j).  Two
+// issuers because a thread that waits on a barrier stops feeding the tensor
+// pipe until its queued MMAs drain; the S/dQ chain and the dP chain wait on
+// different events (K fills and dS from the threads; V fills and the threads
+// freeing dP), so each keeps the pipe busy while the other waits.  Shared memory (D = head dim): Q | dO | 3 x K |
 // 2 x V.  TMEM: S/dS buffers at columns 0 and 128, dP at 256, dQ at 384.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -31,7 +35,8 @@
 namespace ba {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
+constexpr int kWarpY = 6;  // the second MMA issuer (dP)
 constexpr uint32_t kKStages = 3, kVStages = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColDP = 256, kColDQ = 384;
@@ -45,8 +50,8 @@ struct Smem {
   static constexpr uint32_t kV0 = kK0 + kKStages * kTileBytes;
   static constexpr uint32_t kBar = kV0 + kVStages * kTileBytes;
   // q_full, q_empty, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], dp_full,
-  // dp_empty, ds_full[2], dq_done, drain, item_full[4], item_empty[4]
-  static constexpr uint32_t kNumBars = 28;
+  // dp_empty, ds_full[2], dq_done, drain, item_full[4], item_empty[4], drain_y
+  static constexpr uint32_t kNumBars = 29;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8u;  // tmem base, abort, item slots[4]
   static constexpr uint32_t kTotal = kMisc + 32u;
   static constexpr uint32_t kAlloc = kTotal + 1024u;
@@ -86,10 +91,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   ring.slot = reinterpret_cast<volatile int*>(smem + L::kMisc + 16);
   ring.full = bar_drain + 8;
   ring.empty = ring.full + 8 * ptx::kItemSlots;
+  const uint32_t bar_drain_y = ring.empty + 8 * ptx::kItemSlots;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_q_full, 1);
-    ptx::mbar_init(bar_q_empty, 1);
+    ptx::mbar_init(bar_q_empty, 2);  // Q read by issuer X's S MMAs, dO by issuer Y's dP MMAs
     for (uint32_t i = 0; i < kKStages; ++i) {
       ptx::mbar_init(bar_k_full(i), 1);
       ptx::mbar_init(bar_k_empty(i), 1);
@@ -106,9 +112,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bar_dp_empty, 128);
     ptx::mbar_init(bar_dq_done, 1);
     ptx::mbar_init(bar_drain, 1);
+    ptx::mbar_init(bar_drain_y, 1);
     for (uint32_t i = 0; i < ptx::kItemSlots; ++i) {
       ptx::mbar_init(ring.full + 8 * i, 1);
-      ptx::mbar_init(ring.empty + 8 * i, 129);  // MMA issuer + 128 gradient threads
+      ptx::mbar_init(ring.empty + 8 * i, 130);  // two MMA issuers + 128 gradient threads
     }
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -205,29 +212,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (q_fills) ptx::mbar_wait(bar_q_full, (q_fills - 1) & 1u, &never, a.err, dl);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == kWarpY) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two issuing threads: X (warp 1) runs S_j and dQ_j, the users of the two
+    // S/dS buffers, the K stages and dQ; Y (warp 6) runs dP_j, the user of the
+    // dP buffer and the V stages.  Neither touches the other's TMEM columns; a
+    // thread that waits on a barrier stops feeding the tensor pipe while the
+    // other keeps it busy.  The item's Q / dO slot is released by both.
     if (lane == 0) {
+      const bool X = warp == 1;
       constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdDQ = ptx::idesc_bf16_f32(128, D, false, true);
       uint32_t ks = 0, kph = 0, vs = 0, vph = 0, q_phase = 0, dp_phase = 0;
       uint32_t s_cnt = 0, ds_cnt = 0;  // S tiles issued, dQ MMAs issued
       bool ok = true;
-      const uint32_t sQ = sbase + L::kQ, sDO = sbase + L::kDO;
+      // Shared-memory descriptors of every tile and stage, built once.
+      const uint64_t qd0 = ptx::sdesc_sw128(sbase + L::kQ, 16u, 1024u);
+      const uint64_t od0 = ptx::sdesc_sw128(sbase + L::kDO, 16u, 1024u);
+      static_assert(kKStages == 3 && kVStages == 2, "descriptor selects");
+      const uint64_t kd0 = ptx::sdesc_sw128(sbase + L::kK0, 16u, 1024u);
+      const uint64_t kd1 = ptx::sdesc_sw128(sbase + L::kK0 + L::kTileBytes, 16u, 1024u);
+      const uint64_t kd2 = ptx::sdesc_sw128(sbase + L::kK0 + 2u * L::kTileBytes, 16u, 1024u);
+      const uint64_t kg0 = ptx::sdesc_sw128(sbase + L::kK0, 16384u, 1024u);
+      const uint64_t kg1 = ptx::sdesc_sw128(sbase + L::kK0 + L::kTileBytes, 16384u, 1024u);
+      const uint64_t kg2 = ptx::sdesc_sw128(sbase + L::kK0 + 2u * L::kTileBytes, 16384u, 1024u);
+      const uint64_t vd0 = ptx::sdesc_sw128(sbase + L::kV0, 16u, 1024u);
+      const uint64_t vd1 = ptx::sdesc_sw128(sbase + L::kV0 + L::kTileBytes, 16u, 1024u);
+      const uint32_t b_drain = X ? bar_drain : bar_drain_y;
       // dQ += dS K for the tile whose S went to buffer ds_cnt % 2 and whose K
       // sits in K stage `kstage`.
       auto issue_dq = [&](int jj, uint32_t kstage) -> bool {
         const uint32_t b = ds_cnt & 1u;
         if (!ptx::mbar_wait(bar_ds_full(b), (ds_cnt >> 1) & 1u, abort_flag, a.err, lim, ptx::wait_site(2, 1, 3))) return false;
         ptx::tc_fence_after();
-        const uint32_t sk = sbase + L::kK0 + kstage * L::kTileBytes;
-        const uint64_t bd0 = ptx::sdesc_sw128(sk, 16384u, 1024u);
+        const uint64_t bd0 = kstage == 0 ? kg0 : (kstage == 1 ? kg1 : kg2);
+        const uint32_t acc0 = jj > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = ptx::sdesc_add(bd0, kk * 2048u);
-          ptx::umma_ts(tmem + kColDQ, tmem + kColS0 + b * 128u + kk * 8u, bd, kIdDQ,
-                       (jj > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::umma_ts(tmem + kColDQ, tmem + kColS0 + b * 128u + kk * 8u, ptx::sdesc_add(bd0, kk * 2048u), kIdDQ,
+                       kk > 0 ? 1u : acc0);
         ptx::umma_commit(bar_k_empty(kstage));
         ++ds_cnt;
         return true;
@@ -243,53 +266,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ptx::mbar_wait(bar_q_full, q_phase, abort_flag, a.err, lim, ptx::wait_site(2, 1, 4))) { ok = false; break; }
         q_phase ^= 1u;
         ptx::tc_fence_after();
-        uint32_t prev_ks = 0;
-        for (int j = 0; j < n; ++j) {
-          // S_j = Q K_j^T.  Its buffer last held S/dS of tile j-2, whose dQ MMA
-          // was issued before this point, so the in-order pipe keeps them apart.
-          if (!ptx::mbar_wait(bar_k_full(ks), kph, abort_flag, a.err, lim, ptx::wait_site(2, 1, 5))) { ok = false; break; }
-          ptx::tc_fence_after();
-          const uint32_t sb = s_cnt & 1u;
-          const uint32_t sk = sbase + L::kK0 + ks * L::kTileBytes;
-          const uint64_t qd0 = ptx::sdesc_sw128(sQ, 16u, 1024u);
-          const uint64_t kd0 = ptx::sdesc_sw128(sk, 16u, 1024u);
+        if (X) {
+          uint32_t prev_ks = 0;
+          for (int j = 0; j < n; ++j) {
+            // S_j = Q K_j^T.  Its buffer last held S/dS of tile j-2, whose dQ MMA
+            // was issued before this point, so the in-order pipe keeps them apart.
+            if (!ptx::mbar_wait(bar_k_full(ks), kph, abort_flag, a.err, lim, ptx::wait_site(2, 1, 5))) { ok = false; break; }
+            ptx::tc_fence_after();
+            const uint32_t sb = s_cnt & 1u;
+            const uint64_t bk0 = ks == 0 ? kd0 : (ks == 1 ? kd1 : kd2);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-            ptx::umma_ss(tmem + kColS0 + sb * 128u, ptx::sdesc_add(qd0, off), ptx::sdesc_add(kd0, off),
-                         kIdS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+              ptx::umma_ss(tmem + kColS0 + sb * 128u, ptx::sdesc_add(qd0, off), ptx::sdesc_add(bk0, off), kIdS,
+                           kk > 0 ? 1u : 0u);
+            }
+            ptx::umma_commit(bar_s_full(sb));
+            ++s_cnt;
+            if (j == n - 1) ptx::umma_commit(bar_q_empty);
+            if (j > 0 && !issue_dq(j - 1, prev_ks)) { ok = false; break; }
+            prev_ks = ks;
+            if (++ks == kKStages) { ks = 0; kph ^= 1u; }
           }
-          ptx::umma_commit(bar_s_full(sb));
-          ++s_cnt;
-          // dP_j = dO V_j^T once the threads hold dP_{j-1} in registers
-          if (!ptx::mbar_wait(bar_v_full(vs), vph, abort_flag, a.err, lim, ptx::wait_site(2, 1, 6))) { ok = false; break; }
-          if (!ptx::mbar_wait(bar_dp_empty, dp_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 1, 7))) { ok = false; break; }
-          dp_phase ^= 1u;
-          ptx::tc_fence_after();
-          const uint32_t sv = sbase + L::kV0 + vs * L::kTileBytes;
-          const uint64_t od0 = ptx::sdesc_sw128(sDO, 16u, 1024u);
-          const uint64_t vd0 = ptx::sdesc_sw128(sv, 16u, 1024u);
+          if (!ok) break;
+          if (!issue_dq(n - 1, prev_ks)) { ok = false; break; }
+          ptx::umma_commit(bar_dq_done);
+        } else {
+          for (int j = 0; j < n; ++j) {
+            // dP_j = dO V_j^T once the threads hold dP_{j-1} in registers
+            if (!ptx::mbar_wait(bar_v_full(vs), vph, abort_flag, a.err, lim, ptx::wait_site(2, 1, 6))) { ok = false; break; }
+            if (!ptx::mbar_wait(bar_dp_empty, dp_phase ^ 1u, abort_flag, a.err, lim, ptx::wait_site(2, 1, 7))) { ok = false; break; }
+            dp_phase ^= 1u;
+            ptx::tc_fence_after();
+            const uint64_t bv0 = vs ? vd1 : vd0;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-            ptx::umma_ss(tmem + kColDP, ptx::sdesc_add(od0, off), ptx::sdesc_add(vd0, off), kIdS,
-                         kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+              ptx::umma_ss(tmem + kColDP, ptx::sdesc_add(od0, off), ptx::sdesc_add(bv0, off), kIdS, kk > 0 ? 1u : 0u);
+            }
+            ptx::umma_commit(bar_dp_full);
+            ptx::umma_commit(bar_v_empty(vs));
+            if (++vs == kVStages) { vs = 0; vph ^= 1u; }
+            if (j == n - 1) ptx::umma_commit(bar_q_empty);
           }
-          ptx::umma_commit(bar_dp_full);
-          ptx::umma_commit(bar_v_empty(vs));
-          if (++vs == kVStages) { vs = 0; vph ^= 1u; }
-          if (j == n - 1) ptx::umma_commit(bar_q_empty);
-          if (j > 0 && !issue_dq(j - 1, prev_ks)) { ok = false; break; }
-          prev_ks = ks;
-          if (++ks == kKStages) { ks = 0; kph ^= 1u; }
+          if (!ok) break;
         }
-        if (!ok) break;
-        if (!issue_dq(n - 1, prev_ks)) { ok = false; break; }
-        ptx::umma_commit(bar_dq_done);
       }
-      ptx::umma_commit(bar_drain);
+      ptx::umma_commit(b_drain);
       volatile int never = 0;
-      ptx::mbar_wait(bar_drain, 0, &never, a.err, ptx::kDrainCycles);
+      ptx::mbar_wait(b_drain, 0, &never, a.err, ptx::kDrainCycles);
     }
   } else {
     // ------------------------------------------------------------ dS / epilogue

@@ -327,6 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kv_stage = 0, kv_phase = 0;
       uint32_t q_phase[2] = {0u, 0u};
       uint32_t p_cnt[2] = {0u, 0u};  // P tiles consumed per tile slot (p_full parity)
+      // Shared-memory descriptors of every tile and stage, built once: rebuilding
+      // them per MMA group costs the issuing thread more than an MMA takes.
+      const uint64_t dq0 = ptx::sdesc_sw128(sbase + L::kQ0, 16u, 1024u);
+      const uint64_t dq1 = ptx::sdesc_sw128(sbase + L::kQ0 + L::kTileBytes, 16u, 1024u);
+      const uint64_t dk0 = ptx::sdesc_sw128(sbase + L::kK0, 16u, 1024u);
+      const uint64_t dk1 = ptx::sdesc_sw128(sbase + L::kK0 + L::kStageBytes, 16u, 1024u);
+      const uint64_t dv0 = ptx::sdesc_sw128(sbase + L::kK0 + L::kTileBytes, 16384u, 1024u);
+      const uint64_t dv1 = ptx::sdesc_sw128(sbase + L::kK0 + L::kStageBytes + L::kTileBytes, 16384u, 1024u);
       bool ok = true;
       for (uint32_t rn = 0; ok; ++rn) {
         int item = 0;
@@ -342,8 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             first_s[t] = false;
           }
-          const uint64_t ad0 = ptx::sdesc_sw128(sbase + L::kQ0 + t * L::kTileBytes, 16u, 1024u);
-          const uint64_t bd0 = ptx::sdesc_sw128(sbase + L::kK0 + stage * L::kStageBytes, 16u, 1024u);
+          const uint64_t ad0 = t ? dq1 : dq0;
+          const uint64_t bd0 = stage ? dk1 : dk0;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
@@ -358,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ptx::mbar_wait(bar.p_full[t], p_cnt[t] & 1u, abort_flag, a.err, lim, ptx::wait_site(1, 1, 3))) return false;
           ++p_cnt[t];
           ptx::tc_fence_after();
-          const uint64_t bd0 = ptx::sdesc_sw128(sbase + L::kK0 + stage * L::kStageBytes + L::kTileBytes, 16384u, 1024u);
+          const uint64_t bd0 = stage ? dv1 : dv0;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             ptx::umma_ts(tmem + kColO + t * 128u, tmem + kColS + t * 128u + kk * 8u, ptx::sdesc_add(bd0, kk * 2048u),
