@@ -666,6 +666,8 @@ ba_status ba_bwd(const ba_problem* p, const void* o, const void* ob, const float
     ba_.scale = scale;
     ba_.dkb = static_cast<__nv_bfloat16*>(dkb);
     ba_.dvb = static_cast<__nv_bfloat16*>(dvb);
+    ba_.err = di.err;
+    ba_.wait_limit = g_wait_limit.load();
     ProfScope prof("branch_bwd", st);
     if (launch_branch_bwd(ba_, p->d, st) != cudaSuccess) return BA_ERR_CUDA;
   }

@@ -24,6 +24,7 @@
 #include "../../include/ba.h"
 #include "bwd_kernels.h"
 #include "plan.h"
+#include "ptx.cuh"
 
 namespace ba {
 namespace {
@@ -113,46 +114,102 @@ __device__ __forceinline__ int zigzag_owner(const int32_t* cu, int ndoc, int R, 
 }
 
 // One block per (branch b, KV head g); one warp per branch key u (strided).
-// Lane l holds elements [l*E, l*E + E) of k_u, v_u and of the accumulators.
-// For every query head of the group and every row t that sees u (chain:
-// t >= u; block: all; bitmask: bit u of row t's word):
+// The block's inputs are contiguous runs of the input layouts: for each of the
+// B rows, the G query heads of q and of dO (G * D values), and for each of the
+// B keys, k and v (D values).  Thread 0 moves them into shared memory with
+// 4B bulk copies (the TMA engine, completion counted on one mbarrier), so all
+// of a block's bytes are in flight at once instead of one row per warp at a
+// time; the warps then work from shared memory.  Lane l holds elements
+// [l*E, l*E + E) of k_u, v_u and of the accumulators.  For every query head of
+// the group and every row t that sees u (chain: t >= u; block: all; bitmask:
+// bit u of row t's word):
 //   s = scale <q_t, k_u>, P = exp(s - L_t), dS = P (<dO_t, v_u> - D_t),
 //   dV_u += P dO_t, dK_u += scale dS q_t.
-// (Batching several rows' loads per warp was tried: the extra registers cost
-// more occupancy than the loads in flight gained.)
+// E consecutive bf16 values of shared memory (8 or 4 bytes, aligned) as floats.
+template <int E>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float (&f)[E]) {
+  static_assert(E == 4 || E == 2, "4 or 2 values per lane");
+  if constexpr (E == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+    f[0] = lo.x; f[1] = lo.y; f[2] = hi.x; f[3] = hi.y;
+  } else {
+    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    f[0] = v.x; f[1] = v.y;
+  }
+}
+
 template <int D>
-__global__ void branch_bwd_kernel(const BranchBwdArgs a) {
+__global__ void __launch_bounds__(256) branch_bwd_kernel(const BranchBwdArgs a) {
   constexpr int E = D / 32;
   const int b = blockIdx.x / a.Hkv;
   const int g = blockIdx.x % a.Hkv;
   // one rank's rows: the branch belongs to the rank owning its anchor
   if (a.cp_rank >= 0 && zigzag_owner(a.cu, a.ndoc, a.R, a.anchors[b]) != a.cp_rank) return;
   const int G = a.Hq / a.Hkv;
+  const int B = a.B;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = blockDim.x >> 5;
-  const int64_t base_row = int64_t(a.S) + int64_t(b) * a.B;  // concatenated row of (b, 0)
-  for (int u = warp; u < a.B; u += nw) {
-    const int64_t ku = ((int64_t(b) * a.B + u) * a.Hkv + g) * D + lane * E;
+  extern __shared__ __align__(128) uint8_t sm[];
+  __nv_bfloat16* sq = reinterpret_cast<__nv_bfloat16*>(sm);  // [B][G][D]
+  __nv_bfloat16* sdo = sq + B * G * D;                        // [B][G][D]
+  __nv_bfloat16* sk = sdo + B * G * D;                        // [B][D]
+  __nv_bfloat16* sv = sk + B * D;                             // [B][D]
+  float* sL = reinterpret_cast<float*>(sv + B * D);           // [B][G] natural-log LSE
+  float* sD = sL + B * G;                                     // [B][G]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sL + ((2 * B * G + 1) & ~1));  // after L, D; 8-byte aligned
+  const uint32_t bar_a = ptx::smem_u32(bar);
+  const int64_t row0 = int64_t(b) * B;  // flattened branch row / key of (b, 0)
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar_a, 1);
+    ptx::fence_mbar_init();
+    const uint32_t rowb = static_cast<uint32_t>(G * D * 2), keyb = static_cast<uint32_t>(D * 2);
+    ptx::mbar_expect_tx(bar_a, 2u * B * (rowb + keyb));
+    for (int t = 0; t < B; ++t) {
+      const int64_t qo = ((row0 + t) * a.Hq + int64_t(g) * G) * D;
+      const int64_t ko = ((row0 + t) * a.Hkv + g) * D;
+      ptx::bulk_g2s(ptx::smem_u32(sq + t * G * D), a.qb + qo, rowb, bar_a);
+      ptx::bulk_g2s(ptx::smem_u32(sdo + t * G * D), a.dob + qo, rowb, bar_a);
+      ptx::bulk_g2s(ptx::smem_u32(sk + t * D), a.kb + ko, keyb, bar_a);
+      ptx::bulk_g2s(ptx::smem_u32(sv + t * D), a.vb + ko, keyb, bar_a);
+    }
+  }
+  for (int i = threadIdx.x; i < B * G; i += blockDim.x) {
+    const int64_t row = int64_t(a.S) + row0 + i / G;
+    const int64_t h = int64_t(g) * G + i % G;
+    sL[i] = a.lse[h * a.rows + row];
+    sD[i] = a.drow[h * a.rows + row];
+  }
+  __syncthreads();  // the barrier's initialisation and L, D
+  {
+    volatile int never = 0;
+    if (!ptx::mbar_wait(bar_a, 0, &never, a.err, a.wait_limit, ptx::wait_site(5, 2, 1))) {
+      // the copies still land before the block's shared memory goes away
+      ptx::mbar_wait(bar_a, 0, &never, a.err, ptx::kDrainCycles);
+      return;
+    }
+  }
+  for (int u = warp; u < B; u += nw) {
     float kf[E], vf[E], dk[E], dv[E];
+    load_bf16<E>(sk + u * D + lane * E, kf);
+    load_bf16<E>(sv + u * D + lane * E, vf);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      kf[e] = __bfloat162float(a.kb[ku + e]);
-      vf[e] = __bfloat162float(a.vb[ku + e]);
       dk[e] = 0.f;
       dv[e] = 0.f;
     }
     for (int hh = 0; hh < G; ++hh) {
-      const int h = g * G + hh;
-      for (int t = (a.mode == 0 ? u : 0); t < a.B; ++t) {
+      for (int t = (a.mode == 0 ? u : 0); t < B; ++t) {
         // bitmask: row t sees key u iff bit u of its word
-        if (a.mode == 2 && !((a.bmask[int64_t(b) * a.B + t] >> u) & 1ull)) continue;
-        const int64_t qo = ((int64_t(b) * a.B + t) * a.Hq + h) * D + lane * E;
+        if (a.mode == 2 && !((a.bmask[row0 + t] >> u) & 1ull)) continue;
+        const int o = (t * G + hh) * D + lane * E;
         float qf[E], df[E];
+        load_bf16<E>(sq + o, qf);
+        load_bf16<E>(sdo + o, df);
         float s = 0.f, dp = 0.f;
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-          qf[e] = __bfloat162float(a.qb[qo + e]);
-          df[e] = __bfloat162float(a.dob[qo + e]);
           s = fmaf(qf[e], kf[e], s);
           dp = fmaf(df[e], vf[e], dp);
         }
@@ -161,9 +218,8 @@ __global__ void branch_bwd_kernel(const BranchBwdArgs a) {
           s += __shfl_xor_sync(0xffffffffu, s, off);
           dp += __shfl_xor_sync(0xffffffffu, dp, off);
         }
-        const int64_t row = base_row + t;
-        const float P = expf(s * a.scale - a.lse[int64_t(h) * a.rows + row]);
-        const float dS = P * (dp - a.drow[int64_t(h) * a.rows + row]);
+        const float P = expf(s * a.scale - sL[t * G + hh]);
+        const float dS = P * (dp - sD[t * G + hh]);
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           dv[e] = fmaf(P, df[e], dv[e]);
@@ -171,12 +227,19 @@ __global__ void branch_bwd_kernel(const BranchBwdArgs a) {
         }
       }
     }
+    const int64_t ku = ((row0 + u) * a.Hkv + g) * D + lane * E;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       a.dkb[ku + e] = __float2bfloat16_rn(dk[e] * a.scale);
       a.dvb[ku + e] = __float2bfloat16_rn(dv[e]);
     }
   }
+}
+
+// Shared memory of one branch-key block: q, dO [B][G][D], k, v [B][D] (bf16),
+// L, D [B][G] (fp32, padded to 8 bytes) and the copy barrier.
+size_t branch_bwd_smem(int B, int G, int d) {
+  return size_t(2) * B * G * d * 2 + size_t(2) * B * d * 2 + size_t((2 * B * G + 1) & ~1) * 4 + 8;
 }
 
 int grid_cap(int64_t work, int per_block, int cap) {
@@ -204,10 +267,15 @@ cudaError_t launch_branch_bwd(const BranchBwdArgs& a, int d, cudaStream_t st) {
   const int64_t blocks = int64_t(a.Nb) * a.Hkv;
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
   const int warps = a.B < 8 ? a.B : 8;
+  const size_t smem = branch_bwd_smem(a.B, a.Hq / a.Hkv, d);
+  if (smem > 232448) return cudaErrorInvalidValue;  // B x G too large for one block's rows
+  cudaError_t e = d == 128 ? cudaFuncSetAttribute(branch_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))
+                           : cudaFuncSetAttribute(branch_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
   if (d == 128)
-    branch_bwd_kernel<128><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(a);
+    branch_bwd_kernel<128><<<static_cast<unsigned>(blocks), warps * 32, smem, st>>>(a);
   else
-    branch_bwd_kernel<64><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(a);
+    branch_bwd_kernel<64><<<static_cast<unsigned>(blocks), warps * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -40,6 +40,8 @@ struct BranchBwdArgs {
   int64_t rows;
   float scale;
   __nv_bfloat16 *dkb, *dvb;
+  uint32_t* err;          // device error word
+  long long wait_limit;   // bound of the copy wait, in cycles
 };
 cudaError_t launch_branch_bwd(const BranchBwdArgs& a, int d, cudaStream_t st);
 

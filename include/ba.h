@@ -300,7 +300,8 @@ BA_API ba_status ba_check_bounded_wait(ba_stream_t stream);
 
 /* The device error word that the last failing ba_sync_status() reported
  * (0 if none): bit 31 set for an expired bounded wait, bits 24-30 the kernel
- * (1 forward, 2 dQ pass, 3 dK/dV pass, 4 the check above), bits 16-23 the
+ * (1 forward, 2 dQ pass, 3 dK/dV pass, 4 the check above, 5 the branch-key
+ * backward), bits 16-23 the
  * role (0 TMA producer,
  * 1 MMA issuer, 2 softmax / gradient threads), bits 8-15 the wait site in that
  * role, bit 0 the phase parity waited for.  For diagnosing a timeout. */
