@@ -236,6 +236,68 @@ __global__ void __launch_bounds__(256) branch_bwd_kernel(const BranchBwdArgs a) 
   }
 }
 
+// The same computation for shapes whose rows do not fit in one block's shared
+// memory (large B x G): each warp loads its rows from global memory one at a
+// time.
+template <int D>
+__global__ void branch_bwd_rows_kernel(const BranchBwdArgs a) {
+  constexpr int E = D / 32;
+  const int b = blockIdx.x / a.Hkv;
+  const int g = blockIdx.x % a.Hkv;
+  // one rank's rows: the branch belongs to the rank owning its anchor
+  if (a.cp_rank >= 0 && zigzag_owner(a.cu, a.ndoc, a.R, a.anchors[b]) != a.cp_rank) return;
+  const int G = a.Hq / a.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  const int64_t base_row = int64_t(a.S) + int64_t(b) * a.B;  // concatenated row of (b, 0)
+  for (int u = warp; u < a.B; u += nw) {
+    const int64_t ku = ((int64_t(b) * a.B + u) * a.Hkv + g) * D + lane * E;
+    float kf[E], vf[E], dk[E], dv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      kf[e] = __bfloat162float(a.kb[ku + e]);
+      vf[e] = __bfloat162float(a.vb[ku + e]);
+      dk[e] = 0.f;
+      dv[e] = 0.f;
+    }
+    for (int hh = 0; hh < G; ++hh) {
+      const int h = g * G + hh;
+      for (int t = (a.mode == 0 ? u : 0); t < a.B; ++t) {
+        // bitmask: row t sees key u iff bit u of its word
+        if (a.mode == 2 && !((a.bmask[int64_t(b) * a.B + t] >> u) & 1ull)) continue;
+        const int64_t qo = ((int64_t(b) * a.B + t) * a.Hq + h) * D + lane * E;
+        float qf[E], df[E];
+        float s = 0.f, dp = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          qf[e] = __bfloat162float(a.qb[qo + e]);
+          df[e] = __bfloat162float(a.dob[qo + e]);
+          s = fmaf(qf[e], kf[e], s);
+          dp = fmaf(df[e], vf[e], dp);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          s += __shfl_xor_sync(0xffffffffu, s, off);
+          dp += __shfl_xor_sync(0xffffffffu, dp, off);
+        }
+        const int64_t row = base_row + t;
+        const float P = expf(s * a.scale - a.lse[int64_t(h) * a.rows + row]);
+        const float dS = P * (dp - a.drow[int64_t(h) * a.rows + row]);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          dv[e] = fmaf(P, df[e], dv[e]);
+          dk[e] = fmaf(dS, qf[e], dk[e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      a.dkb[ku + e] = __float2bfloat16_rn(dk[e] * a.scale);
+      a.dvb[ku + e] = __float2bfloat16_rn(dv[e]);
+    }
+  }
+}
+
 // Shared memory of one branch-key block: q, dO [B][G][D], k, v [B][D] (bf16),
 // L, D [B][G] (fp32, padded to 8 bytes) and the copy barrier.
 size_t branch_bwd_smem(int B, int G, int d) {
@@ -268,7 +330,13 @@ cudaError_t launch_branch_bwd(const BranchBwdArgs& a, int d, cudaStream_t st) {
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
   const int warps = a.B < 8 ? a.B : 8;
   const size_t smem = branch_bwd_smem(a.B, a.Hq / a.Hkv, d);
-  if (smem > 232448) return cudaErrorInvalidValue;  // B x G too large for one block's rows
+  if (smem > 232448) {  // B x G too large for one block's rows in shared memory
+    if (d == 128)
+      branch_bwd_rows_kernel<128><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(a);
+    else
+      branch_bwd_rows_kernel<64><<<static_cast<unsigned>(blocks), warps * 32, 0, st>>>(a);
+    return cudaGetLastError();
+  }
   cudaError_t e = d == 128 ? cudaFuncSetAttribute(branch_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))
                            : cudaFuncSetAttribute(branch_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
